@@ -1,0 +1,320 @@
+"""PyTorch-facing binding of the Twilight sm_100a library.
+
+Every function here only checks tensor dtypes / shapes, allocates outputs with
+PyTorch (device memory and streams are the only things PyTorch provides) and
+calls the C ABI on the current CUDA stream.  All computation happens in the
+CUDA kernels of libtwilight.so.
+
+Method: "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning"
+(arXiv 2502.02770): Quest page pre-selection, top-p pruning of the candidates'
+attention weights estimated from a 4-bit key cache, exact sparse attention over
+the survivors.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _capi
+from ._capi import TwKv, TwStep, check
+
+HEAD_DIM = 128
+PAGE = 16
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclasses.dataclass
+class KVCache:
+    """fp16 K/V in the contiguous [B][Hk][N][128] layout, or a paged pool
+    [pages][Hk][16][128] with page_table [B][max_pages]."""
+    k: torch.Tensor
+    v: Optional[torch.Tensor]
+    seq_lens: torch.Tensor
+    page_table: Optional[torch.Tensor] = None
+
+    def __post_init__(self):
+        _need(self.k, torch.float16, "k")
+        if self.v is not None:
+            _need(self.v, torch.float16, "v")
+            if self.v.shape != self.k.shape:
+                raise ValueError("k and v must have the same shape")
+        _need(self.seq_lens, torch.int32, "seq_lens")
+        if self.k.shape[-1] != HEAD_DIM:
+            raise ValueError("head_dim must be 128")
+        if self.page_table is not None:
+            _need(self.page_table, torch.int32, "page_table")
+            if self.k.dim() != 4 or self.k.shape[2] != PAGE:
+                raise ValueError("paged k must be [pages][Hk][16][128]")
+        elif self.k.dim() != 4:
+            raise ValueError("contiguous k must be [B][Hk][N][128]")
+
+    @property
+    def paged(self) -> bool:
+        return self.page_table is not None
+
+    @property
+    def B(self) -> int:
+        return int(self.seq_lens.shape[0])
+
+    @property
+    def Hk(self) -> int:
+        return int(self.k.shape[1])
+
+    @property
+    def N(self) -> int:
+        return int(self.page_table.shape[1]) * PAGE if self.paged else int(self.k.shape[2])
+
+    @property
+    def max_pages(self) -> int:
+        return (self.N + PAGE - 1) // PAGE
+
+    def struct(self) -> TwKv:
+        s = TwKv()
+        s.k = _ptr(self.k)
+        s.v = _ptr(self.v)
+        s.batch = self.B
+        s.num_kv_heads = self.Hk
+        s.max_seq_len = self.N
+        s.seq_lens = _ptr(self.seq_lens)
+        s.page_table = _ptr(self.page_table)
+        s.max_pages_per_seq = int(self.page_table.shape[1]) if self.paged else 0
+        s.num_pool_pages = int(self.k.shape[0]) if self.paged else 0
+        s.page_size = PAGE
+        s.head_dim = HEAD_DIM
+        return s
+
+    def row_shape(self, last: int):
+        """Shape of a per-token companion array (codes, scales, zeros)."""
+        if self.paged:
+            return (self.k.shape[0], self.Hk, PAGE, last)
+        return (self.B, self.Hk, self.N, last)
+
+    def meta_shape(self):
+        if self.paged:
+            return (self.k.shape[0], self.Hk, 2, HEAD_DIM)
+        return (self.B, self.Hk, self.max_pages, 2, HEAD_DIM)
+
+    @classmethod
+    def from_workload(cls, w) -> "KVCache":
+        return cls(w.k, w.v, w.seq_lens, w.page_table)
+
+
+@dataclasses.dataclass
+class Int4Keys:
+    codes: torch.Tensor    # uint8  [..][64]
+    scales: torch.Tensor   # fp16   [..][4]
+    zeros: torch.Tensor    # fp16   [..][4]
+
+
+def quantize_keys(kv: KVCache, out: Optional[Int4Keys] = None, stream=None) -> Int4Keys:
+    """4-bit per-token asymmetric key cache (group 32): tw_quantize_keys."""
+    lib = _capi.load()
+    if out is None:
+        out = Int4Keys(torch.zeros(kv.row_shape(64), dtype=torch.uint8, device=kv.k.device),
+                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=kv.k.device),
+                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=kv.k.device))
+    s = kv.struct()
+    check(lib.tw_quantize_keys(ctypes.byref(s), _ptr(out.codes), _ptr(out.scales),
+                               _ptr(out.zeros), _stream(stream)), "tw_quantize_keys")
+    return out
+
+
+def page_meta(kv: KVCache, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Quest per-page channel-wise key min / max: tw_page_meta."""
+    lib = _capi.load()
+    if out is None:
+        out = torch.zeros(kv.meta_shape(), dtype=torch.float16, device=kv.k.device)
+    s = kv.struct()
+    check(lib.tw_page_meta(ctypes.byref(s), _ptr(out), _stream(stream)), "tw_page_meta")
+    return out
+
+
+def workspace_bytes(B: int, Hq: int, Hk: int, N: int, capacity: int) -> int:
+    lib = _capi.load()
+    n = ctypes.c_size_t(0)
+    check(lib.tw_workspace_size(B, Hq, Hk, N, capacity, ctypes.byref(n)), "tw_workspace_size")
+    return int(n.value)
+
+
+def new_workspace(B, Hq, Hk, N, capacity, device) -> torch.Tensor:
+    return torch.empty(max(workspace_bytes(B, Hq, Hk, N, capacity), 256), dtype=torch.uint8,
+                       device=device)
+
+
+def budget_pages(budget_tokens: Optional[int], kv: KVCache) -> int:
+    return min(budget_tokens // PAGE, kv.max_pages)
+
+
+def select_pages(q: torch.Tensor, kv: KVCache, meta: torch.Tensor, budget_tokens: int,
+                 ws: Optional[torch.Tensor] = None, stream=None):
+    """Quest top-K_p pages per (b, KV head): tw_select_pages -> (cand_pages, ncand)."""
+    lib = _capi.load()
+    _need(q, torch.float16, "q")
+    Hq = int(q.shape[1])
+    stride = max(1, budget_pages(budget_tokens, kv))
+    cand = torch.zeros((kv.B, kv.Hk, stride), dtype=torch.int32, device=q.device)
+    ncand = torch.zeros((kv.B, kv.Hk), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = new_workspace(kv.B, Hq, kv.Hk, kv.N, 1, q.device)
+    s = kv.struct()
+    check(lib.tw_select_pages(_ptr(q), Hq, ctypes.byref(s), _ptr(meta), int(budget_tokens),
+                              _ptr(cand), stride, _ptr(ncand), _ptr(ws), ws.numel(),
+                              _stream(stream)), "tw_select_pages")
+    return cand, ncand
+
+
+def num_sets(kv: KVCache, Hq: int, group_mode: int) -> int:
+    return kv.B * kv.Hk if (group_mode or Hq == kv.Hk) else kv.B * Hq
+
+
+def topp_prune(q: torch.Tensor, kv: KVCache, keys: Int4Keys, cand: Optional[torch.Tensor],
+               ncand: Optional[torch.Tensor], p: float, group_mode: int = 0,
+               capacity: Optional[int] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Twilight top-p pruning of the candidates: tw_topp_prune -> (idx, count)."""
+    lib = _capi.load()
+    _need(q, torch.float16, "q")
+    Hq = int(q.shape[1])
+    stride = int(cand.shape[-1]) if cand is not None else 0
+    if capacity is None:
+        capacity = min(stride, kv.max_pages) * PAGE if cand is not None else kv.N
+        capacity = max(capacity, 1)
+    U = num_sets(kv, Hq, group_mode)
+    idx = torch.zeros((U, capacity), dtype=torch.int32, device=q.device)
+    count = torch.zeros((U,), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = new_workspace(kv.B, Hq, kv.Hk, kv.N, capacity, q.device)
+    s = kv.struct()
+    check(lib.tw_topp_prune(_ptr(q), Hq, ctypes.byref(s), _ptr(keys.codes), _ptr(keys.scales),
+                            _ptr(keys.zeros), _ptr(cand), stride, _ptr(ncand), float(p),
+                            int(group_mode), _ptr(idx), capacity, _ptr(count), _ptr(ws),
+                            ws.numel(), _stream(stream)), "tw_topp_prune")
+    return idx, count
+
+
+def sparse_decode(q: torch.Tensor, kv: KVCache, idx: torch.Tensor, count: torch.Tensor,
+                  group_mode: int = 0, ws: Optional[torch.Tensor] = None, with_lse: bool = True,
+                  stream=None):
+    """Exact attention over the selected tokens: tw_sparse_decode -> (out, lse)."""
+    lib = _capi.load()
+    _need(q, torch.float16, "q")
+    _need(idx, torch.int32, "idx")
+    Hq = int(q.shape[1])
+    capacity = int(idx.shape[-1])
+    out = torch.empty((kv.B, Hq, HEAD_DIM), dtype=torch.float16, device=q.device)
+    lse = torch.empty((kv.B, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    if ws is None:
+        ws = new_workspace(kv.B, Hq, kv.Hk, kv.N, capacity, q.device)
+    s = kv.struct()
+    check(lib.tw_sparse_decode(_ptr(q), Hq, ctypes.byref(s), _ptr(idx), capacity, _ptr(count),
+                               int(group_mode), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                               _stream(stream)), "tw_sparse_decode")
+    return out, lse
+
+
+class DecodeStep:
+    """Pre-allocated buffers for repeated tw_decode_step calls on one shape.
+
+    budget_tokens None (or <= 0) means base = full attention (every token is a
+    candidate); otherwise Quest keeps budget_tokens // 16 pages first."""
+
+    def __init__(self, kv: KVCache, keys: Int4Keys, meta: Optional[torch.Tensor], Hq: int,
+                 budget_tokens: Optional[int], p: float, group_mode: int = 0,
+                 with_lse: bool = True):
+        self.kv, self.keys, self.meta = kv, keys, meta
+        self.Hq = Hq
+        self.budget = int(budget_tokens) if budget_tokens and budget_tokens > 0 else 0
+        self.p = float(p)
+        self.group_mode = int(group_mode)
+        dev = kv.k.device
+        if self.budget:
+            self.cand_stride = max(1, budget_pages(self.budget, kv))
+            self.capacity = self.cand_stride * PAGE
+        else:
+            self.cand_stride = 1
+            self.capacity = max(kv.N, 1)
+        self.cand = torch.zeros((kv.B, kv.Hk, self.cand_stride), dtype=torch.int32, device=dev)
+        self.ncand = torch.zeros((kv.B, kv.Hk), dtype=torch.int32, device=dev)
+        U = num_sets(kv, Hq, group_mode)
+        self.idx = torch.zeros((U, self.capacity), dtype=torch.int32, device=dev)
+        self.count = torch.zeros((U,), dtype=torch.int32, device=dev)
+        self.out = torch.zeros((kv.B, Hq, HEAD_DIM), dtype=torch.float16, device=dev)
+        self.lse = torch.zeros((kv.B, Hq), dtype=torch.float32, device=dev) if with_lse else None
+        self.ws = new_workspace(kv.B, Hq, kv.Hk, kv.N, self.capacity, dev)
+        self._q = None
+        self._s = None
+
+    def _struct(self, q: torch.Tensor) -> TwStep:
+        if self._s is not None and self._q is q:
+            return self._s
+        _need(q, torch.float16, "q")
+        if tuple(q.shape) != (self.kv.B, self.Hq, HEAD_DIM):
+            raise ValueError(f"q must be [{self.kv.B}][{self.Hq}][128]")
+        s = TwStep()
+        s.q = _ptr(q)
+        s.num_q_heads = self.Hq
+        s.kv = self.kv.struct()
+        s.codes, s.scales, s.zeros = (_ptr(self.keys.codes), _ptr(self.keys.scales),
+                                      _ptr(self.keys.zeros))
+        s.meta = _ptr(self.meta)
+        s.budget_tokens = self.budget
+        s.p = self.p
+        s.group_mode = self.group_mode
+        s.cand_pages, s.cand_stride, s.ncand = _ptr(self.cand), self.cand_stride, _ptr(self.ncand)
+        s.idx, s.capacity, s.count = _ptr(self.idx), self.capacity, _ptr(self.count)
+        s.out, s.lse = _ptr(self.out), _ptr(self.lse)
+        s.ws, s.ws_bytes = _ptr(self.ws), self.ws.numel()
+        self._q, self._s = q, s
+        return s
+
+    def __call__(self, q: torch.Tensor, stream=None) -> torch.Tensor:
+        lib = _capi.load()
+        s = self._struct(q)
+        check(lib.tw_decode_step(ctypes.byref(s), _stream(stream)), "tw_decode_step")
+        return self.out
+
+    def kernel_names(self):
+        lib = _capi.load()
+        s = self._struct(self._q) if self._q is not None else None
+        if s is None:
+            raise RuntimeError("call the step once before asking for kernel names")
+        n = lib.tw_decode_step_num_kernels(ctypes.byref(s))
+        return [lib.tw_decode_step_kernel_name(ctypes.byref(s), i).decode() for i in range(n)]
+
+    def profiled(self, q: torch.Tensor, events, stream=None) -> None:
+        """Run one step recording events[0] before and events[i+1] after kernel i."""
+        lib = _capi.load()
+        s = self._struct(q)
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        check(lib.tw_decode_step_profiled(ctypes.byref(s), arr, len(events), _stream(stream)),
+              "tw_decode_step_profiled")
+
+
+def prepare(w, device=None):
+    """Move a workload to the GPU and build its int4 key cache and page metadata
+    with the library.  Returns (kv, keys, meta, q)."""
+    if device is not None:
+        w = w.to(device)
+    kv = KVCache.from_workload(w)
+    keys = quantize_keys(kv)
+    meta = page_meta(kv)
+    return kv, keys, meta, w.q

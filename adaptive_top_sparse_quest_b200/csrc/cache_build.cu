@@ -1,0 +1,153 @@
+// Cache-build kernels (prefill time, once per token): the 4-bit key cache and
+// the Quest page metadata.
+//
+// 4-bit key cache: Twilight estimates attention weights from INT4 keys
+// (atlas.scime.ai summary of "Twilight: Adaptive Attention Sparsity with
+// Hierarchical Top-p Pruning", "Approach"; 4-bit preferred to 2-bit in its
+// table of measured effects).  Quest page metadata: per-page channel-wise key
+// min / max, the layout Quest's page selection works on ("Surprising findings").
+//
+// Both kernels stream K once with 16-byte loads; one half-warp owns one token
+// row (or one page), lane l owns channels 8l..8l+7, so a group of 32 channels
+// is 4 adjacent lanes and its min / max needs two xor-shuffles.
+#include "tw_common.cuh"
+#include "tw_kernels.h"
+
+namespace tw {
+
+__global__ void __launch_bounds__(256)
+k_quantize_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ codes,
+                __half* __restrict__ scales, __half* __restrict__ zeros) {
+  const int lane = threadIdx.x & 31;
+  const int l16 = lane & 15;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const int64_t total = (int64_t)L.B * L.Hk * L.N;
+  const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 4);
+  for (int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4); i < total;
+       i += step) {
+    const int t = (int)(i % L.N);
+    const int64_t bh = i / L.N;
+    const int h = (int)(bh % L.Hk);
+    const int b = (int)(bh / L.Hk);
+    if (t >= L.len(b)) continue;  // uniform across the half-warp
+    const int64_t row = L.row(b, h, t);
+    const uint4 raw = ld_stream16(K + row * kHeadDim + l16 * 8);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    int kmin = 0x7FFFFFFF, kmax = -0x7FFFFFFF - 1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int kk = h_key((w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+      kmin = min(kmin, kk);
+      kmax = max(kmax, kk);
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      kmin = min(kmin, __shfl_xor_sync(hmask, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(hmask, kmax, o));
+    }
+    const uint32_t mn_bits = h_from_key(kmin);
+    const uint32_t mx_bits = h_from_key(kmax);
+    const float mnf = __half2float(__ushort_as_half((unsigned short)mn_bits));
+    const float mxf = __half2float(__ushort_as_half((unsigned short)mx_bits));
+    const float s32 = __fdiv_rn(__fsub_rn(mxf, mnf), 15.0f);
+    const __half sc = __float2half_rn(s32);
+    const float scf = __half2float(sc);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x =
+          __half2float(__ushort_as_half((unsigned short)((w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu)));
+      int c = 0;
+      if (scf != 0.0f) {
+        c = __float2int_rn(__fdiv_rn(__fsub_rn(x, mnf), scf));
+        c = min(max(c, 0), 15);
+      }
+      packed |= (uint32_t)c << (4 * j);
+    }
+    *reinterpret_cast<uint32_t*>(codes + row * (kHeadDim / 2) + l16 * 4) = packed;
+    // gather the 4 groups' scale / zero to lane 0 of the half-warp: one 8-byte store each
+    const uint32_t sc_bits = __half_as_ushort(sc);
+    const int base = lane & 16;
+    uint32_t s[4], z[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      s[g] = __shfl_sync(hmask, sc_bits, base + 4 * g);
+      z[g] = __shfl_sync(hmask, mn_bits, base + 4 * g);
+    }
+    if (l16 == 0) {
+      *reinterpret_cast<uint2*>(scales + row * kGroups) =
+          make_uint2(s[0] | (s[1] << 16), s[2] | (s[3] << 16));
+      *reinterpret_cast<uint2*>(zeros + row * kGroups) =
+          make_uint2(z[0] | (z[1] << 16), z[2] | (z[3] << 16));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+k_page_meta(Layout L, const __half* __restrict__ K, __half* __restrict__ meta) {
+  const int l16 = threadIdx.x & 15;
+  const int64_t total = (int64_t)L.B * L.Hk * L.max_pages;
+  const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 4);
+  for (int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4); i < total;
+       i += step) {
+    const int pg = (int)(i % L.max_pages);
+    const int64_t bh = i / L.max_pages;
+    const int h = (int)(bh % L.Hk);
+    const int b = (int)(bh / L.Hk);
+    const int n = min(kPage, L.len(b) - pg * kPage);
+    if (n <= 0) continue;
+    const int64_t row0 = L.page_row(b, h, pg);
+    const __half* src = K + row0 * kHeadDim + l16 * 8;
+    uint4 raw[kPage];
+#pragma unroll
+    for (int r = 0; r < kPage; ++r)
+      if (r < n) raw[r] = ld_stream16(src + (int64_t)r * kHeadDim);
+    int kmin[8], kmax[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      kmin[j] = 0x7FFFFFFF;
+      kmax[j] = -0x7FFFFFFF - 1;
+    }
+#pragma unroll
+    for (int r = 0; r < kPage; ++r) {
+      if (r < n) {
+        const uint32_t w[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int kk = h_key((w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+          kmin[j] = min(kmin[j], kk);
+          kmax[j] = max(kmax[j], kk);
+        }
+      }
+    }
+    uint32_t mn[4], mx[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      mn[j] = h_from_key(kmin[2 * j]) | (h_from_key(kmin[2 * j + 1]) << 16);
+      mx[j] = h_from_key(kmax[2 * j]) | (h_from_key(kmax[2 * j + 1]) << 16);
+    }
+    __half* dst = meta + L.meta_index(b, h, pg) * (2 * kHeadDim) + l16 * 8;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+    *reinterpret_cast<uint4*>(dst + kHeadDim) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
+  }
+}
+
+void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __half* scales,
+                          __half* zeros, cudaStream_t st, int num_sms) {
+  const int64_t rows = (int64_t)L.B * L.Hk * L.N;
+  const int64_t want = (rows + 15) / 16;
+  const int64_t cap_blocks = (int64_t)num_sms * 8;
+  const int blocks = (int)(want < 1 ? 1 : (want < cap_blocks ? want : cap_blocks));
+  k_quantize_keys<<<blocks, 256, 0, st>>>(L, K, codes, scales, zeros);
+}
+
+void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream_t st,
+                      int num_sms) {
+  const int64_t pages = (int64_t)L.B * L.Hk * L.max_pages;
+  const int64_t want = (pages + 15) / 16;
+  const int64_t cap_blocks = (int64_t)num_sms * 8;
+  const int blocks = (int)(want < 1 ? 1 : (want < cap_blocks ? want : cap_blocks));
+  k_page_meta<<<blocks, 256, 0, st>>>(L, K, meta);
+}
+
+}  // namespace tw

@@ -1,0 +1,401 @@
+// C ABI of the Twilight decode path (declared in include/twilight.h): host-side
+// argument checks, workspace carving and kernel launches.  Nothing here
+// allocates device memory, synchronises, or reads device results.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "twilight.h"
+#include "tw_kernels.h"
+
+namespace {
+
+thread_local int g_last_cuda = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda = (int)e;
+  return TW_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Per-device cache: 0 = unknown, -1 = unsupported, >0 = SM count.
+std::atomic<int> g_dev_sms[128];
+
+int device_check(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 128) return TW_ERR_UNSUPPORTED;
+  int v = g_dev_sms[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    v = (major == 10 && minor == 0 && sms > 0) ? sms : -1;
+    g_dev_sms[dev].store(v, std::memory_order_relaxed);
+  }
+  if (v < 0) return TW_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = v;
+  return TW_OK;
+}
+
+int check_kv(const tw_kv* kv, bool need_k, bool need_v, tw::Layout* L) {
+  if (!kv) return TW_ERR_INVALID_ARG;
+  if (kv->head_dim != tw::kHeadDim || kv->page_size != tw::kPage) return TW_ERR_UNSUPPORTED;
+  if (kv->batch < 0 || kv->num_kv_heads < 1 || kv->max_seq_len < 0) return TW_ERR_INVALID_ARG;
+  if (need_k && (!kv->k || !aligned(kv->k, 16))) return TW_ERR_INVALID_ARG;
+  if (need_v && (!kv->v || !aligned(kv->v, 16))) return TW_ERR_INVALID_ARG;
+  if (kv->seq_lens && !aligned(kv->seq_lens, 4)) return TW_ERR_INVALID_ARG;
+  if (kv->page_table) {
+    if (!aligned(kv->page_table, 4) || kv->max_pages_per_seq < 1 || kv->num_pool_pages < 1 ||
+        (int64_t)kv->max_seq_len != (int64_t)kv->max_pages_per_seq * tw::kPage)
+      return TW_ERR_INVALID_ARG;
+  }
+  L->B = kv->batch;
+  L->Hk = kv->num_kv_heads;
+  L->N = kv->max_seq_len;
+  L->seq_lens = kv->seq_lens;
+  L->page_table = kv->page_table;
+  L->max_pages = kv->page_table ? kv->max_pages_per_seq : (kv->max_seq_len + tw::kPage - 1) / tw::kPage;
+  L->pool_pages = kv->page_table ? kv->num_pool_pages : 0;
+  return TW_OK;
+}
+
+int check_heads(int Hq, int Hk) {
+  if (Hq < 1 || Hq % Hk != 0) return TW_ERR_INVALID_ARG;
+  const int G = Hq / Hk;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TW_ERR_UNSUPPORTED;
+  return TW_OK;
+}
+
+// Workspace regions, in order: page scores | logits | tile stats | split partials.
+struct Plan {
+  size_t scores_off, logits_off, stats_off, part_off;
+  size_t scores_end, topp_end, total;
+  int lcap;
+};
+
+Plan make_plan(int B, int Hq, int Hk, int N, int cap) {
+  Plan p;
+  const int G = Hq / Hk;
+  const int64_t pmax = (N + tw::kPage - 1) / tw::kPage;
+  p.lcap = (int)(((int64_t)cap + tw::kEstTile - 1) / tw::kEstTile * tw::kEstTile);
+  p.scores_off = 0;
+  p.scores_end = align256((size_t)B * Hk * pmax * sizeof(float));
+  p.logits_off = p.scores_end;
+  p.stats_off = p.logits_off + align256((size_t)B * Hk * p.lcap * G * sizeof(float));
+  p.topp_end = p.stats_off + align256((size_t)B * Hk * (p.lcap / tw::kEstTile) * G * sizeof(float2));
+  p.part_off = p.topp_end;
+  int S = 0;
+  for (int gs = 0; gs < 2; ++gs) {
+    const int sets = gs ? B * Hk : B * Hq;
+    const int T = tw::decode_split_tokens(sets, cap);
+    const int s = (cap + T - 1) / T;
+    if (s > S) S = s;
+  }
+  p.total = p.part_off + align256((size_t)B * Hq * S * tw::kPartStride * sizeof(float));
+  return p;
+}
+
+char* wsp(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
+
+struct Marker {
+  void* const* ev;
+  int n;
+  cudaStream_t st;
+  int next = 0;
+  cudaError_t mark() {
+    if (!ev) return cudaSuccess;
+    if (next >= n) return cudaErrorInvalidValue;
+    return cudaEventRecord(static_cast<cudaEvent_t>(ev[next++]), st);
+  }
+};
+
+int check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TW_OK : cuda_fail(e);
+}
+
+#define TW_TRY(x)               \
+  do {                          \
+    const int _s = (x);         \
+    if (_s != TW_OK) return _s; \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Argument checks shared by the single calls and the fused step.
+
+int check_select(const uint16_t* q, int Hq, const tw::Layout& L, const uint16_t* meta,
+                 int budget, const int32_t* cand, int cand_stride, const int32_t* ncand) {
+  TW_TRY(check_heads(Hq, L.Hk));
+  if (!q || !aligned(q, 16) || !meta || !aligned(meta, 16)) return TW_ERR_INVALID_ARG;
+  if (budget < tw::kPage) return TW_ERR_INVALID_ARG;
+  if (!cand || !aligned(cand, 4) || !ncand || !aligned(ncand, 4)) return TW_ERR_INVALID_ARG;
+  const int kp = budget / tw::kPage < L.max_pages ? budget / tw::kPage : L.max_pages;
+  if (cand_stride < kp || cand_stride < 1) return TW_ERR_CAPACITY;
+  return TW_OK;
+}
+
+int candidates_max(const tw::Layout& L, const int32_t* cand, int cand_stride) {
+  if (!cand) return L.N;
+  const int rows = cand_stride < L.max_pages ? cand_stride : L.max_pages;
+  return rows * tw::kPage;
+}
+
+int check_topp(const uint16_t* q, int Hq, const tw::Layout& L, const uint8_t* codes,
+               const uint16_t* scales, const uint16_t* zeros, const int32_t* cand,
+               int cand_stride, const int32_t* ncand, double p, int group_mode, int32_t* idx,
+               int capacity, int32_t* count) {
+  TW_TRY(check_heads(Hq, L.Hk));
+  if (!q || !aligned(q, 16)) return TW_ERR_INVALID_ARG;
+  if (!codes || !aligned(codes, 16) || !scales || !aligned(scales, 16) || !zeros ||
+      !aligned(zeros, 16))
+    return TW_ERR_INVALID_ARG;
+  if (cand && (!aligned(cand, 4) || !ncand || !aligned(ncand, 4) || cand_stride < 1))
+    return TW_ERR_INVALID_ARG;
+  if (!(p > 0.0) || !(p <= 1.0)) return TW_ERR_INVALID_ARG;
+  if (group_mode != 0 && group_mode != 1) return TW_ERR_INVALID_ARG;
+  if (!idx || !aligned(idx, 4) || !count || !aligned(count, 4) || capacity < 1)
+    return TW_ERR_INVALID_ARG;
+  const int cmax = candidates_max(L, cand, cand_stride);
+  if (capacity < cmax) return TW_ERR_CAPACITY;
+  if (cmax > tw::kMaxSetCandidates) return TW_ERR_UNSUPPORTED;
+  return TW_OK;
+}
+
+int check_decode(const uint16_t* q, int Hq, const tw::Layout& L, const int32_t* idx,
+                 int capacity, const int32_t* count, int group_mode, uint16_t* out,
+                 float* lse) {
+  TW_TRY(check_heads(Hq, L.Hk));
+  if (!q || !aligned(q, 16) || !idx || !aligned(idx, 4) || !count || !aligned(count, 4))
+    return TW_ERR_INVALID_ARG;
+  if (capacity < 1 || (group_mode != 0 && group_mode != 1)) return TW_ERR_INVALID_ARG;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return TW_ERR_INVALID_ARG;
+  return TW_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return TW_OK;
+  if (!ws || !aligned(ws, 256)) return TW_ERR_INVALID_ARG;
+  if (ws_bytes < need) return TW_ERR_CAPACITY;
+  return TW_OK;
+}
+
+int group_sets_of(int Hq, int Hk, int group_mode) { return (group_mode || Hq == Hk) ? 1 : 0; }
+
+// The fused step, optionally recording an event before the first kernel and
+// after each kernel.
+int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaStream_t st) {
+  if (!s) return TW_ERR_INVALID_ARG;
+  tw::Layout L;
+  TW_TRY(check_kv(&s->kv, true, true, &L));
+  const int Hq = s->num_q_heads;
+  const bool use_select = s->budget_tokens > 0;
+  if (use_select)
+    TW_TRY(check_select(s->q, Hq, L, s->meta, s->budget_tokens, s->cand_pages, s->cand_stride,
+                        s->ncand));
+  const int32_t* cand = use_select ? s->cand_pages : nullptr;
+  TW_TRY(check_topp(s->q, Hq, L, s->codes, s->scales, s->zeros, cand, s->cand_stride, s->ncand,
+                    s->p, s->group_mode, s->idx, s->capacity, s->count));
+  TW_TRY(check_decode(s->q, Hq, L, s->idx, s->capacity, s->count, s->group_mode, s->out, s->lse));
+  if (L.B == 0) return TW_OK;
+  const Plan plan = make_plan(L.B, Hq, L.Hk, L.N, s->capacity);
+  TW_TRY(check_ws(s->ws, s->ws_bytes, plan.total));
+  TW_TRY(device_check(nullptr));
+  const int gs = group_sets_of(Hq, L.Hk, s->group_mode);
+  const auto* q = reinterpret_cast<const __half*>(s->q);
+  Marker mk{events, n_events, st};
+  cudaError_t e;
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  float* scores = reinterpret_cast<float*>(wsp(s->ws, plan.scores_off));
+  if (use_select) {
+    tw::launch_page_scores(L, q, Hq, reinterpret_cast<const __half*>(s->meta), scores, st);
+    if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+    tw::launch_page_topk(L, scores, s->budget_tokens / tw::kPage, s->cand_pages, s->cand_stride,
+                         s->ncand, st);
+    if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  }
+  float* logits = reinterpret_cast<float*>(wsp(s->ws, plan.logits_off));
+  float2* stats = reinterpret_cast<float2*>(wsp(s->ws, plan.stats_off));
+  const int cmax = candidates_max(L, cand, s->cand_stride);
+  tw::launch_estimate(L, q, Hq, s->codes, reinterpret_cast<const __half*>(s->scales),
+                      reinterpret_cast<const __half*>(s->zeros), cand, s->cand_stride, s->ncand,
+                      plan.lcap, cmax, logits, stats, st);
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  e = tw::launch_topp(L, Hq, gs, cand, s->cand_stride, s->ncand, plan.lcap, cmax, logits, stats,
+                      s->p, s->idx, s->capacity, s->count, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  float* part = reinterpret_cast<float*>(wsp(s->ws, plan.part_off));
+  const auto* K = reinterpret_cast<const __half*>(s->kv.k);
+  const auto* V = reinterpret_cast<const __half*>(s->kv.v);
+  auto* out = reinterpret_cast<__half*>(s->out);
+  tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, out, s->lse,
+                           st, false, true);
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, out, s->lse,
+                           st, true, false);
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tw_status_string(int status) {
+  switch (status) {
+    case TW_OK: return "TW_OK";
+    case TW_ERR_INVALID_ARG: return "TW_ERR_INVALID_ARG: null/misaligned pointer or bad parameter";
+    case TW_ERR_UNSUPPORTED: return "TW_ERR_UNSUPPORTED: shape or device not supported";
+    case TW_ERR_CAPACITY: return "TW_ERR_CAPACITY: output or workspace buffer too small";
+    case TW_ERR_CUDA: return "TW_ERR_CUDA: a CUDA call failed";
+    case TW_ERR_TIMEOUT: return "TW_ERR_TIMEOUT: a bounded device wait gave up";
+    default: return "unknown tw_status";
+  }
+}
+
+int tw_last_cuda_error(void) { return g_last_cuda; }
+
+int tw_version(void) { return 100; }
+
+int tw_quantize_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                     void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, true, false, &L));
+  if (!codes || !aligned(codes, 16) || !scales || !aligned(scales, 16) || !zeros ||
+      !aligned(zeros, 16))
+    return TW_ERR_INVALID_ARG;
+  if ((int64_t)L.B * L.N == 0) return TW_OK;
+  int sms = 0;
+  TW_TRY(device_check(&sms));
+  tw::launch_quantize_keys(L, reinterpret_cast<const __half*>(kv->k), codes,
+                           reinterpret_cast<__half*>(scales), reinterpret_cast<__half*>(zeros),
+                           static_cast<cudaStream_t>(stream), sms);
+  return check_launch();
+}
+
+int tw_page_meta(const tw_kv* kv, uint16_t* meta, void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, true, false, &L));
+  if (!meta || !aligned(meta, 16)) return TW_ERR_INVALID_ARG;
+  if ((int64_t)L.B * L.N == 0) return TW_OK;
+  int sms = 0;
+  TW_TRY(device_check(&sms));
+  tw::launch_page_meta(L, reinterpret_cast<const __half*>(kv->k), reinterpret_cast<__half*>(meta),
+                       static_cast<cudaStream_t>(stream), sms);
+  return check_launch();
+}
+
+int tw_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t max_seq_len, int32_t capacity, size_t* bytes) {
+  if (!bytes || batch < 0 || num_kv_heads < 1 || max_seq_len < 0 || capacity < 1)
+    return TW_ERR_INVALID_ARG;
+  TW_TRY(check_heads(num_q_heads, num_kv_heads));
+  *bytes = make_plan(batch, num_q_heads, num_kv_heads, max_seq_len, capacity).total;
+  return TW_OK;
+}
+
+int tw_select_pages(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                    const uint16_t* meta, int32_t budget_tokens, int32_t* cand_pages,
+                    int32_t cand_stride, int32_t* ncand, void* ws, size_t ws_bytes,
+                    void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, false, false, &L));
+  TW_TRY(check_select(q, num_q_heads, L, meta, budget_tokens, cand_pages, cand_stride, ncand));
+  if (L.B == 0) return TW_OK;
+  const Plan plan = make_plan(L.B, num_q_heads, L.Hk, L.N, 1);
+  TW_TRY(check_ws(ws, ws_bytes, plan.scores_end));
+  TW_TRY(device_check(nullptr));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = reinterpret_cast<float*>(wsp(ws, plan.scores_off));
+  tw::launch_page_scores(L, reinterpret_cast<const __half*>(q), num_q_heads,
+                         reinterpret_cast<const __half*>(meta), scores, st);
+  tw::launch_page_topk(L, scores, budget_tokens / tw::kPage, cand_pages, cand_stride, ncand, st);
+  return check_launch();
+}
+
+int tw_topp_prune(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                  const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                  const int32_t* cand_pages, int32_t cand_stride, const int32_t* ncand,
+                  double p, int32_t group_mode, int32_t* idx, int32_t capacity, int32_t* count,
+                  void* ws, size_t ws_bytes, void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, false, false, &L));
+  TW_TRY(check_topp(q, num_q_heads, L, codes, scales, zeros, cand_pages, cand_stride, ncand, p,
+                    group_mode, idx, capacity, count));
+  if (L.B == 0) return TW_OK;
+  const Plan plan = make_plan(L.B, num_q_heads, L.Hk, L.N, capacity);
+  TW_TRY(check_ws(ws, ws_bytes, plan.topp_end));
+  TW_TRY(device_check(nullptr));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* logits = reinterpret_cast<float*>(wsp(ws, plan.logits_off));
+  float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.stats_off));
+  const auto* qh = reinterpret_cast<const __half*>(q);
+  const int cmax = candidates_max(L, cand_pages, cand_stride);
+  tw::launch_estimate(L, qh, num_q_heads, codes, reinterpret_cast<const __half*>(scales),
+                      reinterpret_cast<const __half*>(zeros), cand_pages, cand_stride, ncand,
+                      plan.lcap, cmax, logits, stats, st);
+  const cudaError_t e =
+      tw::launch_topp(L, num_q_heads, group_sets_of(num_q_heads, L.Hk, group_mode), cand_pages,
+                      cand_stride, ncand, plan.lcap, cmax, logits, stats, p, idx, capacity, count,
+                      st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                     const int32_t* idx, int32_t capacity, const int32_t* count,
+                     int32_t group_mode, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                     void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, true, true, &L));
+  TW_TRY(check_decode(q, num_q_heads, L, idx, capacity, count, group_mode, out, lse));
+  if (L.B == 0) return TW_OK;
+  const Plan plan = make_plan(L.B, num_q_heads, L.Hk, L.N, capacity);
+  TW_TRY(check_ws(ws, ws_bytes, plan.total));
+  TW_TRY(device_check(nullptr));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* part = reinterpret_cast<float*>(wsp(ws, plan.part_off));
+  const int gs = group_sets_of(num_q_heads, L.Hk, group_mode);
+  const auto* K = reinterpret_cast<const __half*>(kv->k);
+  const auto* V = reinterpret_cast<const __half*>(kv->v);
+  tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V, idx,
+                           capacity, count, part, reinterpret_cast<__half*>(out), lse, st, false,
+                           false);
+  return check_launch();
+}
+
+int tw_decode_step(const tw_step* step, void* stream) {
+  return decode_step_impl(step, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+int tw_decode_step_num_kernels(const tw_step* step) {
+  if (!step) return -TW_ERR_INVALID_ARG;
+  return step->budget_tokens > 0 ? 6 : 4;
+}
+
+const char* tw_decode_step_kernel_name(const tw_step* step, int32_t i) {
+  static const char* with_select[6] = {"page_scores", "page_topk", "estimate",
+                                       "topp", "sparse_decode", "merge"};
+  static const char* no_select[4] = {"estimate", "topp", "sparse_decode", "merge"};
+  if (!step) return nullptr;
+  if (step->budget_tokens > 0) return (i >= 0 && i < 6) ? with_select[i] : nullptr;
+  return (i >= 0 && i < 4) ? no_select[i] : nullptr;
+}
+
+int tw_decode_step_profiled(const tw_step* step, void* const* events, int32_t n_events,
+                            void* stream) {
+  if (!events || n_events < tw_decode_step_num_kernels(step) + 1) return TW_ERR_INVALID_ARG;
+  return decode_step_impl(step, events, n_events, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,41 @@
+// Internal launch interface between the C ABI (capi.cu) and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tw_common.cuh"
+
+namespace tw {
+
+constexpr int kEstTile = 256;        // candidates per estimate block (and per tile statistic)
+constexpr int kPartStride = 132;     // floats per split record: m, l, 2 pad, acc[128]
+constexpr int kPartAcc = 4;
+constexpr int kTargetSms = 148;      // B200 SM count used to size decode splits
+constexpr int kMaxSetCandidates = 8 * 512 * 32;   // cluster of 8 x 512 threads x 32 weights
+
+void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __half* scales,
+                          __half* zeros, cudaStream_t st, int num_sms);
+void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream_t st,
+                      int num_sms);
+void launch_page_scores(const Layout& L, const __half* q, int Hq, const __half* meta,
+                        float* scores, cudaStream_t st);
+void launch_page_topk(const Layout& L, const float* scores, int budget_pages, int32_t* cand,
+                      int cand_stride, int32_t* ncand, cudaStream_t st);
+void launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
+                     const __half* scales, const __half* zeros, const int32_t* cand,
+                     int cand_stride, const int32_t* ncand, int cap, int cmax, float* logits,
+                     float2* stats, cudaStream_t st);
+int topp_cluster_shape(int cmax, int* R, int* CS);
+cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* cand,
+                        int cand_stride, const int32_t* ncand, int lcap, int cmax,
+                        const float* logits, const float2* stats, double p, int32_t* idx,
+                        int icap, int32_t* count, cudaStream_t st);
+int decode_split_tokens(int sets, int icap);
+void launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
+                          const __half* K, const __half* V, const int32_t* idx, int icap,
+                          const int32_t* count, float* part, __half* out, float* lse,
+                          cudaStream_t st, bool merge_only, bool decode_only);
+
+}  // namespace tw

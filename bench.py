@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of one Twilight decode step per layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one decode layer: Quest page
+scores + top-K_p pages -> int4 weight estimate + top-p threshold + index
+compaction -> split-K sparse attention + log-sum-exp merge (the KV cache, its
+4-bit key companion and the page metadata are built beforehand, as at
+prefill).  The default workload is the Llama-2-7B-shaped MHA layer: batch 1, 32
+heads, context 32768, Quest budget 8192 tokens, p = 0.85.
+
+The timed region replays the step over R independent copies of the cache in
+rotation, so the bytes touched between two visits of a copy exceed the 126 MB
+L2.  Times are CUDA events on the launching stream, max over ranks.  With N > 1
+(torchrun) each rank runs an independent replica on its own GPU: the path has
+no exchange step, so there is no collective on the data path.
+
+--impl reference times the CPU oracle on the host cores on a bounded sample of
+the same workload and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs per decode step (top-p prune + sparse attn) per layer; achieved HBM GB/s"
+UNIT = "us/step"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="llama2_mha",
+                    choices=["llama2_mha", "llama3_gqa", "batched_paged", "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def make_workload(name, device):
+    import workloads as W
+    return W.CONFIGS[name](device=device)
+
+
+def workload_config(w, copies=None, copy_bytes=None):
+    c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hk,
+         "context": w.N, "paged": w.paged, "budget_tokens": w.budget_tokens, "p": w.p,
+         "group_mode": w.group_mode, "head_dim": 128, "page_size": 16, "int4_group": 32}
+    if copies:
+        c["l2"] = (f"inputs larger than L2: {copies} rotating cache copies, "
+                   f"{copy_bytes / 1e9:.2f} GB each")
+    return c
+
+
+def src_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "adaptive_top_sparse_quest_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        pk = json.load(open(PEAKS_PATH))
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while load runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_step_sample(w_cpu, seconds: float, max_units=None):
+    """Time the oracle's decode step (page scores, top-K_p, int4 estimate, top-p,
+    sparse attention) on (b, kv head) units of the workload until `seconds` of
+    CPU work; the int4 cache and page metadata are built first, untimed, as at
+    prefill.  Returns (us per full step, units timed, total units, threads)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:
+        limiter = None
+    import numpy as np
+
+    import oracle as O
+    x = O.SeqInputs.from_workload(w_cpu)
+    G = x.Hq // x.Hk
+    units = [(b, h) for b in range(x.B) for h in range(x.Hk)]
+    rng = np.random.default_rng(0)
+    order = rng.permutation(len(units))
+    spent, n = 0.0, 0
+    for ui in order:
+        if max_units is not None and n >= max_units:
+            break
+        b, hk = units[ui]
+        L = int(x.seq_lens[b])
+        k_seq = O.sequence_rows(x.k, x.page_table, b, hk, L)
+        v_seq = O.sequence_rows(x.v, x.page_table, b, hk, L)
+        codes, scales, zeros = O.quantize_keys(k_seq)
+        meta = O.page_meta(k_seq, L) if w_cpu.budget_tokens else None
+        qg = x.q[b, hk * G:(hk + 1) * G]
+        t0 = time.perf_counter()
+        pages = None
+        if w_cpu.budget_tokens:
+            pages = O.select_pages(O.quest_page_scores(qg, meta), w_cpu.budget_tokens)
+        toks = O.candidate_tokens(pages, L)
+        lg = O.estimate_logits(qg, codes[toks], scales[toks], zeros[toks])
+        if w_cpu.group_mode and G > 1:
+            sel = O.topp_select(O.group_weights(lg), w_cpu.p)[0]
+            sels = [sel] * G
+        else:
+            sels = [O.topp_select(O.softmax_weights(lg[:, g]), w_cpu.p)[0] for g in range(G)]
+        for g in range(G):
+            t = toks[sels[g]]
+            O.sparse_attention(qg[g], k_seq[t], v_seq[t])
+        spent += time.perf_counter() - t0
+        n += 1
+        if spent >= seconds:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    return spent / n * len(units) * 1e6, n, len(units), 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    w = make_workload(args.config, "cpu")
+    per = []
+    for i in range(args.warmup + args.steps):
+        us, n, tot, cores = cpu_step_sample(w, 0.0, max_units=1)
+        if i >= args.warmup:
+            per.append(us)
+    value = statistics.mean(per)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": value / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step: 1 random (sequence, KV head) unit of {tot}, "
+                                   "scaled by the unit count"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def algorithmic_bytes(w, step):
+    """Bytes the step must move (per kernel): page metadata scanned (512 B per
+    page per KV head), int4 candidate keys (80 B per candidate token per KV
+    head) and fp16 K+V rows of the selected tokens (512 B per token per set)."""
+    import torch
+    lens = w.seq_lens.to(torch.int64).cpu()
+    pages = (lens + 15) // 16
+    meta_b = int(pages.sum()) * w.Hk * 512 if w.budget_tokens else 0
+    if w.budget_tokens:
+        nc = step.ncand.to(torch.int64).cpu()          # [B][Hk] pages
+        cand_tokens = 0
+        for b in range(w.B):
+            for h in range(w.Hk):
+                # every candidate page is full except possibly the sequence's last page
+                n = int(nc[b, h]) * 16
+                last = int(lens[b]) - (int(pages[b]) - 1) * 16
+                sel = step.cand[b, h, :int(nc[b, h])].cpu()
+                if int(pages[b]) - 1 in sel.tolist():
+                    n -= 16 - last
+                cand_tokens += n
+    else:
+        cand_tokens = int(lens.sum()) * w.Hk
+    int4_b = cand_tokens * 80
+    kept = step.count.to(torch.int64).cpu()
+    kv_b = int(kept.sum()) * 512
+    return {"page_scores": meta_b, "estimate": int4_b, "sparse_decode": kv_b}, cand_tokens, kept
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from adaptive_top_sparse_quest_b200 import DecodeStep, KVCache, _capi, page_meta, quantize_keys
+    from adaptive_top_sparse_quest_b200 import build as _b
+    _b.build()
+    _capi.load()
+
+    w = make_workload(args.config, dev)
+    kv0 = KVCache.from_workload(w)
+    keys0 = quantize_keys(kv0)
+    meta0 = page_meta(kv0)
+    torch.cuda.synchronize()
+    copy_bytes = sum(t.numel() * t.element_size() for t in
+                     (w.k, w.v, keys0.codes, keys0.scales, keys0.zeros, meta0))
+    touched_est = 114e6
+    R = 1
+    while R * min(copy_bytes, 4 * touched_est) < 4 * L2_BYTES and R < 16:
+        R += 1
+    R = max(R, 4)
+
+    # cache-build kernels timed once (GB/s over K read + int4/meta written)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    quantize_keys(kv0, keys0)
+    ev[1].record()
+    page_meta(kv0, meta0)
+    ev[2].record()
+    torch.cuda.synchronize()
+    build_ms = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]))
+
+    steps = []
+    for r in range(R):
+        if r == 0:
+            kv, keys, meta = kv0, keys0, meta0
+        else:
+            kv = KVCache(w.k.clone(), w.v.clone(), w.seq_lens.clone(),
+                         None if w.page_table is None else w.page_table.clone())
+            keys = type(keys0)(keys0.codes.clone(), keys0.scales.clone(), keys0.zeros.clone())
+            meta = meta0.clone()
+        steps.append(DecodeStep(kv, keys, meta, w.Hq, w.budget_tokens, w.p, w.group_mode))
+    q = w.q.contiguous()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.warmup):
+        steps[i % R](q)
+    barrier()
+    t_start = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        steps[i % R](q)
+    e1.record(stream)
+    e1.synchronize()
+    barrier()
+    t_end = time.time()
+    elapsed_ms = e0.elapsed_time(e1)
+    # keep the GPU under the same load long enough for nvidia-smi to sample clocks
+    t_load_end = t_end
+    if sampler and t_end - t_start < 0.6:
+        n_extra = 0
+        while time.time() - t_end < 0.6:
+            for _ in range(200):
+                steps[n_extra % R](q)
+                n_extra += 1
+            torch.cuda.synchronize()
+        t_load_end = time.time()
+    t_max = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+    us_per_step = elapsed_ms * 1e3 / args.steps
+    value = us_per_step / world
+
+    # per-kernel durations: the same step with an event after each kernel
+    names = steps[0].kernel_names()
+    nk = len(names)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(4)]
+    for es in evs:
+        for e in es:
+            e.record(stream)
+    torch.cuda.synchronize()
+    per = [[] for _ in range(nk)]
+    nprof = max(8, min(args.steps, 400))
+    for i in range(nprof):
+        es = evs[i % 4]
+        steps[i % R].profiled(q, es)
+        if i % 4 == 3 or i == nprof - 1:
+            torch.cuda.synchronize()
+            for j in range(i - (i % 4), i + 1):
+                ej = evs[j % 4]
+                for k in range(nk):
+                    per[k].append(ej[k].elapsed_time(ej[k + 1]) * 1e3)
+    kernel_us = {names[k]: statistics.mean(per[k]) for k in range(nk)}
+
+    # end to end through the public API with host buffers: q from pinned host
+    # memory in, the attention output back to pinned host memory, every step
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty(steps[0].out.shape, dtype=steps[0].out.dtype).pin_memory()
+    q_dev = torch.empty_like(q)
+    for i in range(max(3, args.warmup)):
+        q_dev.copy_(q_host, non_blocking=True)
+        o = steps[i % R](q_dev)
+        out_host.copy_(o, non_blocking=True)
+    barrier()
+    e0.record(stream)
+    for i in range(args.steps):
+        q_dev.copy_(q_host, non_blocking=True)
+        o = steps[i % R](q_dev)
+        out_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    e1.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    t2 = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_us = float(t2.item()) * 1e3 / args.steps / world
+
+    if sampler:
+        sampler.stop()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    kb, cand_tokens, kept = algorithmic_bytes(w, steps[0])
+    toks_total = int(w.seq_lens.to(torch.int64).sum()) * w.Hk
+    pages_total = int(((w.seq_lens.to(torch.int64) + 15) // 16).sum()) * w.Hk
+    total_b = sum(kb.values())
+    peak, peak_kind = hbm_peak()
+    dom = max(kb, key=lambda k: kernel_us.get(k, 0.0) if kb[k] > 0 else -1)
+    dom_us = kernel_us[dom]
+    achieved = kb[dom] / (dom_us * 1e-6) / 1e9
+    traffic = None
+    try:
+        tr = json.load(open(TRAFFIC_PATH))
+        if tr.get("src_hash") == src_hash() and tr.get("workload") == w.name and \
+                tr.get("kernel") == dom:
+            traffic = tr.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    clocks = sampler.summary(t_start - 0.05, t_load_end + 0.05) if sampler else None
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        w_cpu = w.to("cpu")
+        cpu_us, n_units, tot_units, cores = cpu_step_sample(w_cpu, args.cpu_seconds)
+        cpu = {"value": cpu_us, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n_units} of {tot_units} (sequence, KV head) units of the same "
+                         f"workload, single-threaded numpy, scaled to the full step"}
+
+    sets = kept.numel()
+    cands_per_set = cand_tokens / max(1, w.B * w.Hk)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, R, copy_bytes),
+        "hbm_gbs": total_b / (us_per_step * 1e-6) / 1e9,
+        "hbm_frac_of_measured": total_b / (us_per_step * 1e-6) / 1e9 / peak,
+        "bytes_per_step": total_b,
+        "kv_tokens_scanned_per_s": cand_tokens / (us_per_step * 1e-6),
+        "kept_tokens": {"mean": float(kept.double().mean()), "min": int(kept.min()),
+                        "max": int(kept.max()), "sets": sets,
+                        "candidates_per_set": cands_per_set},
+        "pruned_frac": 1.0 - float(kept.double().mean()) / max(1.0, cands_per_set),
+        "kernel_us": kernel_us,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": kb[dom]},
+        "cache_build": {
+            "quantize_keys_gbs": toks_total * (256 + 80) / (build_ms[0] * 1e-3) / 1e9,
+            "page_meta_gbs": (toks_total * 256 + pages_total * 512) / (build_ms[1] * 1e-3) / 1e9},
+        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": q.numel() * q.element_size(),
+                "d2h_bytes_per_step": steps[0].out.numel() * steps[0].out.element_size()},
+        "gpu_launches": args.steps * nk,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

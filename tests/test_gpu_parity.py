@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle on
+the same seeded inputs.
+
+Bars: bit-exact int4 codes, scales, zeros, page metadata and page ids; the
+selected index set exact except tokens whose oracle weight is within 1e-6
+relative of the oracle threshold (plus, counted separately, one token at the
+cut when the oracle's cumulative mass there is within 1e-5 of p); attention
+output max abs error <= 2e-3 against the oracle's fp64 result on the GPU's own
+selection."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from _parity import check_attention, compare_selection, gpu_meta, gpu_rows, np16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from adaptive_top_sparse_quest_b200 import _capi, build
+    build.build()
+    _capi.load()
+
+
+def run_gpu(w, budget, p, gm):
+    from adaptive_top_sparse_quest_b200 import DecodeStep, prepare
+    kv, keys, meta, q = prepare(w, "cuda")
+    step = DecodeStep(kv, keys, meta, w.Hq, budget, p, gm)
+    step(q)
+    torch.cuda.synchronize()
+    return dict(codes=np16(keys.codes), scales=np16(keys.scales), zeros=np16(keys.zeros),
+                meta=np16(meta), cand=np16(step.cand), ncand=np16(step.ncand),
+                idx=np16(step.idx), count=np16(step.count), out=np16(step.out),
+                lse=np16(step.lse), step=step, kv=kv, keys=keys, meta_t=meta, q=q)
+
+
+def check_units(w, g, budget, p, gm, units, check_cache=True):
+    x = O.SeqInputs.from_workload(w)
+    table = x.page_table
+    G = w.Hq // w.Hk
+    group_sets = gm == 1 or G == 1
+    stats = {"near": 0, "cut": 0, "sets": 0, "max_err": 0.0}
+    for (b, hk) in units:
+        res = O.oracle_unit(x, b, hk, budget, p, gm)
+        L = res["len"]
+        if check_cache:
+            assert np.array_equal(gpu_rows(g["codes"], table, b, hk, L), res["codes"])
+            assert np.array_equal(gpu_rows(g["scales"], table, b, hk, L).view(np.uint16),
+                                  res["scales"].view(np.uint16))
+            assert np.array_equal(gpu_rows(g["zeros"], table, b, hk, L).view(np.uint16),
+                                  res["zeros"].view(np.uint16))
+            assert np.array_equal(gpu_meta(g["meta"], table, b, hk, L).view(np.uint16),
+                                  res["meta"].view(np.uint16))
+        if budget:
+            n = int(g["ncand"][b, hk])
+            assert g["cand"][b, hk, :n].tolist() == res["pages"].tolist()
+        heads = list(range(hk * G, (hk + 1) * G))
+        for hq in heads:
+            s = b * w.Hk + hk if group_sets else b * w.Hq + hq
+            cnt = int(g["count"][s])
+            toks = g["idx"][s, :cnt]
+            if group_sets and hq != heads[0]:
+                pass
+            else:
+                near, cut = compare_selection(toks, res, hq, p)
+                stats["near"] += near
+                stats["cut"] += cut
+                stats["sets"] += 1
+            err = check_attention(g["out"][b, hq], float(g["lse"][b, hq]), x, b, hq, toks, hk)
+            stats["max_err"] = max(stats["max_err"], err)
+    return stats
+
+
+SMALL = [
+    dict(seed=1, B=2, Hq=2, Hk=2, N=777, paged=False, budget=160, p=0.85, gm=0),
+    dict(seed=2, B=3, Hq=8, Hk=2, N=1000, paged=True, budget=256, p=0.85, gm=1),
+    dict(seed=3, B=2, Hq=8, Hk=2, N=900, paged=False, budget=320, p=0.9, gm=0),
+    dict(seed=4, B=2, Hq=4, Hk=4, N=1500, paged=True, budget=None, p=0.85, gm=0),
+    dict(seed=5, B=1, Hq=8, Hk=1, N=2049, paged=False, budget=None, p=0.7, gm=1),
+    dict(seed=6, B=4, Hq=4, Hk=2, N=333, paged=True, budget=48, p=0.95, gm=1),
+    dict(seed=7, B=2, Hq=4, Hk=2, N=5000, paged=False, budget=4096, p=0.99, gm=1),
+]
+
+
+@pytest.mark.parametrize("c", SMALL, ids=lambda c: f"s{c['seed']}")
+def test_small_parity(c):
+    w = W.random_small(c["seed"], B=c["B"], Hq=c["Hq"], Hk=c["Hk"], N=c["N"], paged=c["paged"],
+                       budget_tokens=c["budget"], p=c["p"], group_mode=c["gm"])
+    g = run_gpu(w, c["budget"], c["p"], c["gm"])
+    units = [(b, h) for b in range(w.B) for h in range(w.Hk)]
+    st = check_units(w, g, c["budget"], c["p"], c["gm"], units)
+    assert st["cut"] <= max(1, st["sets"] // 20)
+
+
+def test_tiny_single_head_full_size():
+    w = W.tiny(device="cpu")
+    g = run_gpu(w, None, 0.85, 0)
+    st = check_units(w, g, None, 0.85, 0, [(0, 0)])
+    assert set(w.heavy[(0, 0)]) <= set(g["idx"][0, :g["count"][0]].tolist())
+
+
+def test_single_calls_match_fused_step():
+    from adaptive_top_sparse_quest_b200 import select_pages, sparse_decode, topp_prune
+    w = W.random_small(11, B=2, Hq=8, Hk=2, N=1200, paged=True, budget_tokens=256, group_mode=1)
+    g = run_gpu(w, 256, 0.85, 1)
+    kv, keys, meta, q = g["kv"], g["keys"], g["meta_t"], g["q"]
+    cand, ncand = select_pages(q, kv, meta, 256)
+    idx, count = topp_prune(q, kv, keys, cand, ncand, 0.85, 1)
+    out, lse = sparse_decode(q, kv, idx, count, 1)
+    torch.cuda.synchronize()
+    assert np.array_equal(np16(ncand), g["ncand"])
+    for b in range(w.B):
+        for h in range(w.Hk):
+            n = int(g["ncand"][b, h])
+            assert np.array_equal(np16(cand)[b, h, :n], g["cand"][b, h, :n])
+    assert np.array_equal(np16(count), g["count"])
+    for s in range(count.shape[0]):
+        n = int(g["count"][s])
+        assert np.array_equal(np16(idx)[s, :n], g["idx"][s, :n])
+    assert np.array_equal(np16(out).view(np.uint16), g["out"].view(np.uint16))
+    assert np.array_equal(np16(lse), g["lse"])
+
+
+def test_empty_and_one_token_sequences():
+    w = W.random_small(12, B=3, Hq=4, Hk=2, N=64, paged=True, budget_tokens=32, group_mode=1)
+    w.seq_lens[:] = torch.tensor([0, 1, 17], dtype=torch.int32)
+    g = run_gpu(w, 32, 0.85, 1)
+    assert g["count"][0] == 0 and g["count"][1] == 0
+    assert np.all(g["out"][0] == 0) and np.all(np.isneginf(g["lse"][0]))
+    assert g["count"][2] == 1 and g["count"][3] == 1
+    check_units(w, g, 32, 0.85, 1, [(1, 0), (1, 1), (2, 0), (2, 1)])
+
+
+def _pin_workload(n, seed, mode):
+    w = W.random_small(seed, B=1, Hq=1, Hk=1, N=n, ragged=False, budget_tokens=None, n_heavy=0)
+    if mode == "uniform":
+        w.k[0, 0, :] = w.k[0, 0, 0].clone()
+    elif mode == "spike":
+        qf = w.q[0, 0].float()
+        w.k[0, 0, n // 3] = (qf * (60.0 * math.sqrt(128) / float(qf @ qf))).half()
+    return w
+
+
+@pytest.mark.parametrize("p", [0.5, 0.85, 0.9, 0.999])
+def test_pin_uniform_keeps_ceil_pn(p):
+    n = 1000
+    g = run_gpu(_pin_workload(n, 21, "uniform"), None, p, 0)
+    k = math.ceil(p * n - 1e-9)
+    assert int(g["count"][0]) == k
+    assert g["idx"][0, :k].tolist() == list(range(k))
+
+
+@pytest.mark.parametrize("p", [0.5, 0.85, 0.99, 0.999999])
+def test_pin_spike_keeps_one(p):
+    n = 3000
+    g = run_gpu(_pin_workload(n, 22, "spike"), None, p, 0)
+    assert int(g["count"][0]) == 1 and int(g["idx"][0, 0]) == n // 3
+
+
+def test_pin_p_one_keeps_all_and_is_dense():
+    w = W.random_small(23, B=2, Hq=4, Hk=2, N=700, budget_tokens=None, group_mode=1)
+    g = run_gpu(w, None, 1.0, 1)
+    lens = w.seq_lens.tolist()
+    for b in range(2):
+        for h in range(2):
+            s = b * 2 + h
+            assert g["count"][s] == lens[b]
+            assert g["idx"][s, :lens[b]].tolist() == list(range(lens[b]))
+    check_units(w, g, None, 1.0, 1, [(0, 0), (1, 1)], check_cache=False)
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads, in the launch configuration the benchmark times, checked
+# on sampled (sequence, KV head) units.
+
+def _full(w, units, budget, p, gm):
+    g = run_gpu(w, budget, p, gm)
+    st = check_units(w, g, budget, p, gm, units)
+    assert st["cut"] <= max(1, st["sets"] // 10), st
+    return st
+
+
+@pytest.mark.slow
+def test_full_llama2_mha_32k():
+    w = W.llama2_mha(device="cuda")
+    _full(w, [(0, 0), (0, 17), (0, 31)], w.budget_tokens, w.p, 0)
+
+
+@pytest.mark.slow
+def test_full_llama3_gqa_128k():
+    w = W.llama3_gqa(device="cuda")
+    _full(w, [(0, 0), (0, 3), (0, 7)], w.budget_tokens, w.p, 1)
+
+
+@pytest.mark.slow
+def test_full_batched_paged():
+    w = W.batched_paged(device="cuda")
+    _full(w, [(0, 0), (7, 12), (15, 31)], w.budget_tokens, w.p, 0)
+
+
+@pytest.mark.slow
+def test_full_concentration_sweep():
+    base = W.concentration_sweep(device="cuda")
+    i = 0
+    for tau in W.SWEEP_TAU:
+        for p in W.SWEEP_P:
+            w = W.sweep_point(base, tau, p)
+            _full(w, [(i % 4, (3 * i) % 8)], None, p, 1)
+            i += 1
