@@ -76,9 +76,10 @@ int check_heads(int Hq, int Hk) {
   return TW_OK;
 }
 
-// Workspace regions, in order: page scores | logits | tile stats | split partials.
+// Workspace regions, in order: page scores | logits | softmax statistics |
+// per-set completion counters | attention partial records.
 struct Plan {
-  size_t scores_off, logits_off, stats_off, part_off;
+  size_t scores_off, logits_off, stats_off, done_off, part_off;
   size_t scores_end, topp_end, total;
   int lcap;
 };
@@ -92,16 +93,12 @@ Plan make_plan(int B, int Hq, int Hk, int N, int cap) {
   p.scores_end = align256((size_t)B * Hk * pmax * sizeof(float));
   p.logits_off = p.scores_end;
   p.stats_off = p.logits_off + align256((size_t)B * Hk * p.lcap * G * sizeof(float));
-  p.topp_end = p.stats_off + align256((size_t)B * Hk * (p.lcap / tw::kEstTile) * G * sizeof(float2));
-  p.part_off = p.topp_end;
-  int S = 0;
-  for (int gs = 0; gs < 2; ++gs) {
-    const int sets = gs ? B * Hk : B * Hq;
-    const int T = tw::decode_split_tokens(sets, cap);
-    const int s = (cap + T - 1) / T;
-    if (s > S) S = s;
-  }
-  p.total = p.part_off + align256((size_t)B * Hq * S * tw::kPartStride * sizeof(float));
+  p.topp_end = p.stats_off +
+               align256((size_t)B * Hk * (p.lcap / tw::kStatSpan) * G * sizeof(float2));
+  p.done_off = p.topp_end;
+  const size_t nsets = (size_t)B * (Hq > Hk ? Hq : Hk);
+  p.part_off = p.done_off + align256(nsets * sizeof(int32_t));
+  p.total = p.part_off + align256(tw::decode_part_floats(B, Hq, Hk) * sizeof(float));
   return p;
 }
 
@@ -209,41 +206,44 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   if (L.B == 0) return TW_OK;
   const Plan plan = make_plan(L.B, Hq, L.Hk, L.N, s->capacity);
   TW_TRY(check_ws(s->ws, s->ws_bytes, plan.total));
-  TW_TRY(device_check(nullptr));
+  int sms = 0;
+  TW_TRY(device_check(&sms));
   const int gs = group_sets_of(Hq, L.Hk, s->group_mode);
   const auto* q = reinterpret_cast<const __half*>(s->q);
+  // programmatic dependent launch overlaps each kernel's launch with its
+  // predecessor's tail; the profiled variant runs them strictly in order so
+  // that each event pair brackets exactly one kernel
+  const bool pdl = events == nullptr;
   Marker mk{events, n_events, st};
   cudaError_t e;
   if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   float* scores = reinterpret_cast<float*>(wsp(s->ws, plan.scores_off));
   if (use_select) {
-    tw::launch_page_scores(L, q, Hq, reinterpret_cast<const __half*>(s->meta), scores, st);
-    if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
-    tw::launch_page_topk(L, scores, s->budget_tokens / tw::kPage, s->cand_pages, s->cand_stride,
-                         s->ncand, st);
-    if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+    e = tw::launch_page_scores(L, q, Hq, reinterpret_cast<const __half*>(s->meta), scores, st,
+                               sms, pdl);
+    if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+    e = tw::launch_page_topk(L, scores, s->budget_tokens / tw::kPage, s->cand_pages,
+                             s->cand_stride, s->ncand, st, pdl);
+    if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   }
   float* logits = reinterpret_cast<float*>(wsp(s->ws, plan.logits_off));
   float2* stats = reinterpret_cast<float2*>(wsp(s->ws, plan.stats_off));
   const int cmax = candidates_max(L, cand, s->cand_stride);
-  tw::launch_estimate(L, q, Hq, s->codes, reinterpret_cast<const __half*>(s->scales),
-                      reinterpret_cast<const __half*>(s->zeros), cand, s->cand_stride, s->ncand,
-                      plan.lcap, cmax, logits, stats, st);
-  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  e = tw::launch_estimate(L, q, Hq, s->codes, reinterpret_cast<const __half*>(s->scales),
+                          reinterpret_cast<const __half*>(s->zeros), cand, s->cand_stride,
+                          s->ncand, plan.lcap, cmax, logits, stats, st, sms, pdl);
+  if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  int32_t* done = reinterpret_cast<int32_t*>(wsp(s->ws, plan.done_off));
   e = tw::launch_topp(L, Hq, gs, cand, s->cand_stride, s->ncand, plan.lcap, cmax, logits, stats,
-                      s->p, s->idx, s->capacity, s->count, st);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+                      s->p, s->idx, s->capacity, s->count, done, st, pdl);
+  if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   float* part = reinterpret_cast<float*>(wsp(s->ws, plan.part_off));
   const auto* K = reinterpret_cast<const __half*>(s->kv.k);
   const auto* V = reinterpret_cast<const __half*>(s->kv.v);
   auto* out = reinterpret_cast<__half*>(s->out);
-  tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, out, s->lse,
-                           st, false, true);
-  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
-  tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, out, s->lse,
-                           st, true, false);
-  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  e = tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, done, out,
+                               s->lse, st, pdl);
+  if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 
@@ -314,12 +314,17 @@ int tw_select_pages(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   if (L.B == 0) return TW_OK;
   const Plan plan = make_plan(L.B, num_q_heads, L.Hk, L.N, 1);
   TW_TRY(check_ws(ws, ws_bytes, plan.scores_end));
-  TW_TRY(device_check(nullptr));
+  int sms = 0;
+  TW_TRY(device_check(&sms));
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(wsp(ws, plan.scores_off));
-  tw::launch_page_scores(L, reinterpret_cast<const __half*>(q), num_q_heads,
-                         reinterpret_cast<const __half*>(meta), scores, st);
-  tw::launch_page_topk(L, scores, budget_tokens / tw::kPage, cand_pages, cand_stride, ncand, st);
+  cudaError_t e = tw::launch_page_scores(L, reinterpret_cast<const __half*>(q), num_q_heads,
+                                         reinterpret_cast<const __half*>(meta), scores, st, sms,
+                                         false);
+  if (e == cudaSuccess)
+    e = tw::launch_page_topk(L, scores, budget_tokens / tw::kPage, cand_pages, cand_stride,
+                             ncand, st, false);
+  if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 
@@ -335,19 +340,21 @@ int tw_topp_prune(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   if (L.B == 0) return TW_OK;
   const Plan plan = make_plan(L.B, num_q_heads, L.Hk, L.N, capacity);
   TW_TRY(check_ws(ws, ws_bytes, plan.topp_end));
-  TW_TRY(device_check(nullptr));
+  int sms = 0;
+  TW_TRY(device_check(&sms));
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* logits = reinterpret_cast<float*>(wsp(ws, plan.logits_off));
   float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.stats_off));
-  const auto* qh = reinterpret_cast<const __half*>(q);
   const int cmax = candidates_max(L, cand_pages, cand_stride);
-  tw::launch_estimate(L, qh, num_q_heads, codes, reinterpret_cast<const __half*>(scales),
-                      reinterpret_cast<const __half*>(zeros), cand_pages, cand_stride, ncand,
-                      plan.lcap, cmax, logits, stats, st);
-  const cudaError_t e =
-      tw::launch_topp(L, num_q_heads, group_sets_of(num_q_heads, L.Hk, group_mode), cand_pages,
-                      cand_stride, ncand, plan.lcap, cmax, logits, stats, p, idx, capacity, count,
-                      st);
+  cudaError_t e = tw::launch_estimate(L, reinterpret_cast<const __half*>(q), num_q_heads, codes,
+                                      reinterpret_cast<const __half*>(scales),
+                                      reinterpret_cast<const __half*>(zeros), cand_pages,
+                                      cand_stride, ncand, plan.lcap, cmax, logits, stats, st, sms,
+                                      false);
+  if (e == cudaSuccess)
+    e = tw::launch_topp(L, num_q_heads, group_sets_of(num_q_heads, L.Hk, group_mode), cand_pages,
+                        cand_stride, ncand, plan.lcap, cmax, logits, stats, p, idx, capacity,
+                        count, nullptr, st, false);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
@@ -365,12 +372,17 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   TW_TRY(device_check(nullptr));
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* part = reinterpret_cast<float*>(wsp(ws, plan.part_off));
+  int32_t* done = reinterpret_cast<int32_t*>(wsp(ws, plan.done_off));
   const int gs = group_sets_of(num_q_heads, L.Hk, group_mode);
+  const int nsets = gs ? L.B * L.Hk : L.B * num_q_heads;
   const auto* K = reinterpret_cast<const __half*>(kv->k);
   const auto* V = reinterpret_cast<const __half*>(kv->v);
-  tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V, idx,
-                           capacity, count, part, reinterpret_cast<__half*>(out), lse, st, false,
-                           false);
+  cudaError_t e = cudaMemsetAsync(done, 0, (size_t)nsets * sizeof(int32_t), st);
+  if (e == cudaSuccess)
+    e = tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V, idx,
+                                 capacity, count, part, done, reinterpret_cast<__half*>(out), lse,
+                                 st, false);
+  if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 
@@ -380,16 +392,16 @@ int tw_decode_step(const tw_step* step, void* stream) {
 
 int tw_decode_step_num_kernels(const tw_step* step) {
   if (!step) return -TW_ERR_INVALID_ARG;
-  return step->budget_tokens > 0 ? 6 : 4;
+  return step->budget_tokens > 0 ? 5 : 3;
 }
 
 const char* tw_decode_step_kernel_name(const tw_step* step, int32_t i) {
-  static const char* with_select[6] = {"page_scores", "page_topk", "estimate",
-                                       "topp", "sparse_decode", "merge"};
-  static const char* no_select[4] = {"estimate", "topp", "sparse_decode", "merge"};
+  static const char* with_select[5] = {"page_scores", "page_topk", "estimate", "topp",
+                                       "sparse_decode"};
+  static const char* no_select[3] = {"estimate", "topp", "sparse_decode"};
   if (!step) return nullptr;
-  if (step->budget_tokens > 0) return (i >= 0 && i < 6) ? with_select[i] : nullptr;
-  return (i >= 0 && i < 4) ? no_select[i] : nullptr;
+  if (step->budget_tokens > 0) return (i >= 0 && i < 5) ? with_select[i] : nullptr;
+  return (i >= 0 && i < 3) ? no_select[i] : nullptr;
 }
 
 int tw_decode_step_profiled(const tw_step* step, void* const* events, int32_t n_events,

@@ -1,39 +1,169 @@
 // Exact attention over the tokens that survive Twilight's top-p pruning:
-// split-K flash decoding with a log-sum-exp merge.
+// load-balanced split-K flash decoding with a fused log-sum-exp merge.
 //
 // After pruning, attention runs only over the selected tokens' fp16 K/V
 // ("Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning",
 // atlas.scime.ai summary, "Approach": select-then-prune, then sparse attention;
 // its kernels build on FlashInfer, "Experimental setup").
 //
-// k_sparse_decode: block (split, set); the split covers idx[split*T, split*T+T).
-//   Each warp walks every 4th selected token; lane l owns channels 4l..4l+3,
-//   so a gathered 256-byte K or V row is one coalesced 8-byte load per lane.
-//   Rows for 8 tokens are loaded before any math (64 B of K + V per lane in
-//   flight per batch).  The NH query heads that share the set reuse every
-//   gathered row.  Online softmax in the log2 domain; the 4 warps' partial
-//   (max, sum, acc) are combined in shared memory and one record per (query
-//   head, split) is written: {m, l, -, -, acc[128]} fp32.
-// k_merge: one block per (b, query head); out = sum_s 2^(m_s-M) acc_s /
-//   sum_s 2^(m_s-M) l_s, lse = ln 2 * (M + log2 sum_s 2^(m_s-M) l_s).
+// Work split.  The selected-token counts are only known on the device and
+// differ per set (head or KV group) by an order of magnitude, so a fixed split
+// per set leaves most of the GPU idle.  The selected tokens of all sets are
+// viewed as one concatenated list of S tokens and a fixed grid of kDecCtas
+// CTAs takes equal contiguous ranges: CTA c owns [c*S/n, (c+1)*S/n).  Each CTA
+// derives the set offsets from the counts.  For every set its range touches,
+// the CTA writes one partial record {m, l, acc[128]} per query head to slot
+// (c + set), unique because (c, set) pairs advance monotonically along the
+// list.
+//
+// Data path.  The set's token ids for a window of the range are staged in
+// shared memory once; the gathered 256-byte K and V rows then stream through a
+// 4-stage cp.async ring of 16 tokens per stage (32 KB in flight per CTA), so
+// a CTA pays one dependent round trip per window instead of one per batch.
+// Each half-warp takes 2 tokens of a stage; lane l of the half-warp holds
+// channels 8l..8l+7, the scores are reduced with 4 xor-shuffles and the online
+// softmax is kept in the log2 domain.  The NH query heads of a KV group reuse
+// every staged row.
+//
+// Merge.  After writing its record for a set, a CTA bumps the set's counter;
+// the CTA that completes the set folds all of its records:
+//   out = sum_r 2^(m_r-M) acc_r / sum_r 2^(m_r-M) l_r,
+//   lse = ln 2 * (M + log2 sum_r 2^(m_r-M) l_r),
+// and resets the counter.  Sets with no selected token get out = 0, lse = -inf.
 #include "tw_common.cuh"
 #include "tw_kernels.h"
 
 namespace tw {
 
 constexpr int kDecThreads = 128;
-constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kDecBatch = 8;
+constexpr int kDecHW = kDecThreads / 16;       // half-warps
+constexpr int kStageTok = 16;                  // tokens per pipeline stage
+constexpr int kStages = 4;
+constexpr int kWin = 512;                      // token ids staged per window
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void h4_to_f4(uint2 r, float* f) {
-  const __half2 a = *reinterpret_cast<const __half2*>(&r.x);
-  const __half2 b = *reinterpret_cast<const __half2*>(&r.y);
-  const float2 fa = __half22float2(a), fb = __half22float2(b);
-  f[0] = fa.x;
-  f[1] = fa.y;
-  f[2] = fb.x;
-  f[3] = fb.y;
+__device__ __forceinline__ void h8_to_f8(uint4 r, float* f) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ int64_t block_sum_i64(int64_t v, int64_t* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  int64_t t = 0;
+#pragma unroll
+  for (int i = 0; i < kDecThreads / 32; ++i) t += sh[i];
+  return t;
+}
+
+__device__ __forceinline__ bool range_has(int64_t c, int64_t S, int n, int64_t off, int cnt) {
+  const int64_t lo = c * S / n, hi = (c + 1) * S / n;
+  return lo < hi && lo < off + cnt && hi > off;
+}
+
+template <int NH>
+struct DecSmem {
+  int ids[kWin];
+  union {
+    __half kv[kStages][kStageTok][2][kHeadDim];                 // K row, V row
+    struct {
+      float m[kDecHW][NH], l[kDecHW][NH];
+      float acc[kDecHW][NH][kHeadDim];
+    } comb;
+    struct {
+      float f[kDecThreads];
+      float red[kDecThreads / 32];
+    } merge;
+  } u;
+  int64_t red64[kDecThreads / 32];
+  int list_set[kDecThreads];
+  long long list_off[kDecThreads];
+  unsigned wcnt[kDecThreads / 32];
+  int nlist;
+  int last;
+};
+
+// Fold the records of `set` into out / lse (called by the CTA that completes it).
+template <int NH>
+__device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_t S, int n_ctas,
+                          int Hq, int hq0, int b, const float* part, __half* out, float* lse) {
+  const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  const int64_t c0 = ((off + 1) * n_ctas + S - 1) / S - 1;
+  const int64_t c1 = ((off + cnt) * n_ctas + S - 1) / S - 1;
+  const int nrec = (int)(c1 - c0 + 1);
+  for (int h = 0; h < NH; ++h) {
+    float mx = -INFINITY;
+    for (int r = d; r < nrec; r += kDecThreads)
+      if (range_has(c0 + r, S, n_ctas, off, cnt))
+        mx = fmaxf(mx, part[((c0 + r + set) * NH + h) * kPartStride]);
+    mx = warp_max(mx);
+    __syncthreads();
+    if (lane == 0) sm.u.merge.red[warp] = mx;
+    __syncthreads();
+    float M = sm.u.merge.red[0];
+#pragma unroll
+    for (int i = 1; i < kDecThreads / 32; ++i) M = fmaxf(M, sm.u.merge.red[i]);
+    float Ls = 0.f, A = 0.f;
+    for (int r0 = 0; r0 < nrec; r0 += kDecThreads) {
+      const int r = r0 + d;
+      float f = 0.f;
+      if (r < nrec && range_has(c0 + r, S, n_ctas, off, cnt)) {
+        const float* rec = part + ((c0 + r + set) * NH + h) * kPartStride;
+        if (rec[0] != -INFINITY) {
+          f = exp2f(rec[0] - M);
+          Ls += rec[1] * f;
+        }
+      }
+      __syncthreads();
+      sm.u.merge.f[d] = f;
+      __syncthreads();
+      const int nr = min(kDecThreads, nrec - r0);
+      int i = 0;
+      for (; i + 8 <= nr; i += 8) {
+        float a8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          a8[j] = sm.u.merge.f[i + j] != 0.f
+                      ? part[((c0 + r0 + i + j + set) * NH + h) * kPartStride + kPartAcc + d]
+                      : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) A += a8[j] * sm.u.merge.f[i + j];
+      }
+      for (; i < nr; ++i)
+        if (sm.u.merge.f[i] != 0.f)
+          A += part[((c0 + r0 + i + set) * NH + h) * kPartStride + kPartAcc + d] * sm.u.merge.f[i];
+    }
+    Ls = warp_sum(Ls);
+    __syncthreads();
+    if (lane == 0) sm.u.merge.red[warp] = Ls;
+    __syncthreads();
+    Ls = 0.f;
+#pragma unroll
+    for (int i = 0; i < kDecThreads / 32; ++i) Ls += sm.u.merge.red[i];
+    const int64_t bh = (int64_t)b * Hq + hq0 + h;
+    out[bh * kHeadDim + d] = __float2half_rn(Ls > 0.f ? A / Ls : 0.f);
+    if (lse && d == 0) lse[bh] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  }
 }
 
 template <int NH>
@@ -41,174 +171,278 @@ __global__ void __launch_bounds__(kDecThreads)
 k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group_sets,
                 const __half* __restrict__ K, const __half* __restrict__ V,
                 const int32_t* __restrict__ idx, int icap, const int32_t* __restrict__ count,
-                int T, int S, float* __restrict__ part) {
-  __shared__ float sm_m[kDecWarps][NH], sm_l[kDecWarps][NH];
-  __shared__ __align__(16) float sm_acc[kDecWarps][NH][kHeadDim];
-  const int set = blockIdx.y, split = blockIdx.x;
-  const int n = min(count[set], icap);
-  const int start = split * T;
-  if (start >= n) return;
-  const int end = min(n, start + T);
-  int b, hk, hq0;
-  if (group_sets) {
-    b = set / L.Hk;
-    hk = set % L.Hk;
-    hq0 = hk * G;
-  } else {
-    b = set / Hq;
-    hq0 = set % Hq;
-    hk = hq0 / G;
-  }
-  const int len = L.len(b);
+                int nsets, float* __restrict__ part, int32_t* __restrict__ done,
+                __half* __restrict__ out, float* __restrict__ lse) {
+  __shared__ __align__(16) DecSmem<NH> sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float qscale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
-  float qf[NH][4];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    const uint2 r = *reinterpret_cast<const uint2*>(q + ((int64_t)b * Hq + hq0 + h) * kHeadDim + 4 * lane);
-    h4_to_f4(r, qf[h]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) qf[h][j] *= qscale;
-  }
-  float m[NH], l[NH], acc[NH][4];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[h][j] = 0.f;
-  }
-  const int32_t* ids = idx + (int64_t)set * icap;
-  for (int i0 = start + warp; i0 < end; i0 += kDecWarps * kDecBatch) {
-    uint2 kr[kDecBatch], vr[kDecBatch];
-    bool ok[kDecBatch];
-#pragma unroll
-    for (int j = 0; j < kDecBatch; ++j) {
-      const int i = i0 + j * kDecWarps;
-      ok[j] = false;
-      if (i < end) {
-        const int t = ids[i];
-        ok[j] = (unsigned)t < (unsigned)len;   // ids outside [0, len) are ignored
-        if (ok[j]) {
-          const int64_t row = L.row(b, hk, t);
-          kr[j] = ld_stream8(K + row * kHeadDim + 4 * lane);
-          vr[j] = ld_stream8(V + row * kHeadDim + 4 * lane);
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kDecBatch; ++j) {
-      if (!ok[j]) continue;   // uniform across the warp
-      float kf[4], vf[4];
-      h4_to_f4(kr[j], kf);
-      h4_to_f4(vr[j], vf);
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float s = qf[h][0] * kf[0];
-        s = __fmaf_rn(qf[h][1], kf[1], s);
-        s = __fmaf_rn(qf[h][2], kf[2], s);
-        s = __fmaf_rn(qf[h][3], kf[3], s);
-        s = warp_sum(s);
-        const float mn = fmaxf(m[h], s);
-        const float corr = exp2f(m[h] - mn);
-        const float pr = exp2f(s - mn);
-        l[h] = l[h] * corr + pr;
-#pragma unroll
-        for (int d = 0; d < 4; ++d) acc[h][d] = __fmaf_rn(pr, vf[d], acc[h][d] * corr);
-        m[h] = mn;
-      }
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    if (lane == 0) {
-      sm_m[warp][h] = m[h];
-      sm_l[warp][h] = l[h];
-    }
-    *reinterpret_cast<float4*>(&sm_acc[warp][h][4 * lane]) =
-        make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-  }
-  __syncthreads();
-  // thread tid combines channel tid of every head across the 4 warps
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][h]);
-    float Ls = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-      const float f = sm_m[w][h] == -INFINITY ? 0.f : exp2f(sm_m[w][h] - M);
-      Ls += sm_l[w][h] * f;
-      A += sm_acc[w][h][tid] * f;
-    }
-    float* rec = part + (((int64_t)b * Hq + hq0 + h) * S + split) * kPartStride;
-    rec[kPartAcc + tid] = A;
-    if (tid == 0) {
-      rec[0] = M;
-      rec[1] = Ls;
-    }
-  }
-}
+  const int hw = tid >> 4, l16 = tid & 15;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const int n = gridDim.x, c = blockIdx.x;
+  griddep_wait();
 
-__global__ void __launch_bounds__(kHeadDim)
-k_merge(int Hq, int Hk, int G, int group_sets, const int32_t* __restrict__ count, int icap, int T,
-        int S, const float* __restrict__ part, __half* __restrict__ out, float* __restrict__ lse) {
-  const int bh = blockIdx.x;
-  const int b = bh / Hq, hq = bh % Hq;
-  const int set = group_sets ? b * Hk + hq / G : bh;
-  const int n = max(0, min(count[set], icap));
-  const int ns = (n + T - 1) / T;
-  const int d = threadIdx.x;
-  const float* rec = part + (int64_t)bh * S * kPartStride;
-  if (ns == 0) {
-    out[(int64_t)bh * kHeadDim + d] = __float2half_rn(0.f);
-    if (lse && d == 0) lse[bh] = -INFINITY;
+  auto set_heads = [&](int set, int& b, int& hk, int& hq0) {
+    if (group_sets) {
+      b = set / L.Hk;
+      hk = set % L.Hk;
+      hq0 = hk * G;
+    } else {
+      b = set / Hq;
+      hq0 = set % Hq;
+      hk = hq0 / G;
+    }
+  };
+
+  // total selected tokens; sets with none get out = 0 here (one CTA each)
+  int64_t loc = 0;
+  for (int s = tid; s < nsets; s += kDecThreads) loc += max(0, min(count[s], icap));
+  const int64_t S = block_sum_i64(loc, sm.red64);
+  for (int s = c; s < nsets; s += n) {
+    if (max(0, min(count[s], icap)) == 0) {
+      int b, hk, hq0;
+      set_heads(s, b, hk, hq0);
+      for (int h = 0; h < NH; ++h) {
+        const int64_t bh = (int64_t)b * Hq + hq0 + h;
+        out[bh * kHeadDim + tid] = __float2half_rn(0.f);
+        if (lse && tid == 0) lse[bh] = -INFINITY;
+      }
+    }
+  }
+  const int64_t begin = (int64_t)c * S / n, end = (int64_t)(c + 1) * S / n;
+  if (begin >= end) {
+    griddep_launch();
     return;
   }
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, rec[s * kPartStride]);
-  float Ls = 0.f, A = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const float ms = rec[s * kPartStride];
-    const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
-    Ls += rec[s * kPartStride + 1] * f;
-    A += rec[s * kPartStride + kPartAcc + d] * f;
+  const float qscale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+
+  int64_t running = 0;
+  for (int base = 0; base < nsets && running < end; base += kDecThreads) {
+    // offsets of this chunk of sets, and the sets that overlap [begin, end)
+    const int s = base + tid;
+    const int cnt = s < nsets ? max(0, min(count[s], icap)) : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    __syncthreads();
+    if (lane == 31) sm.wcnt[warp] = incl;
+    if (tid == 0) sm.nlist = 0;
+    __syncthreads();
+    int wbefore = 0, chunk = 0;
+#pragma unroll
+    for (int i = 0; i < kDecThreads / 32; ++i) {
+      const int v = (int)sm.wcnt[i];
+      if (i < warp) wbefore += v;
+      chunk += v;
+    }
+    const int64_t off = running + wbefore + incl - cnt;
+    const bool hit = cnt > 0 && off < end && off + cnt > begin;
+    const unsigned bal = __ballot_sync(0xffffffffu, hit);
+    __syncthreads();
+    if (lane == 0 && bal) sm.wcnt[warp] = atomicAdd(&sm.nlist, __popc(bal));
+    __syncthreads();
+    if (hit) {
+      const int slot = sm.wcnt[warp] + __popc(bal & ((1u << lane) - 1u));
+      sm.list_set[slot] = s;
+      sm.list_off[slot] = off;
+    }
+    __syncthreads();
+    const int nl = sm.nlist;   // record slots depend only on (c, set): order does not matter
+    running += chunk;
+    for (int li = 0; li < nl; ++li) {
+      const int set = sm.list_set[li];
+      const int64_t soff = sm.list_off[li];
+      const int scnt = max(0, min(count[set], icap));
+      const int64_t lo = max(begin, soff), hi = min(end, soff + scnt);
+      int b, hk, hq0;
+      set_heads(set, b, hk, hq0);
+      const int len = L.len(b);
+      float qf[NH][8];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const uint4 r = *reinterpret_cast<const uint4*>(q + ((int64_t)b * Hq + hq0 + h) * kHeadDim + 8 * l16);
+        h8_to_f8(r, qf[h]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qf[h][j] *= qscale;
+      }
+      float m[NH], l[NH], acc[NH][8];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
+      }
+      const int32_t* ids = idx + (int64_t)set * icap;
+      for (int64_t w0 = lo; w0 < hi; w0 += kWin) {
+        const int wn = (int)min((int64_t)kWin, hi - w0);
+        __syncthreads();   // previous window's ids and ring are no longer read
+        for (int i = tid; i < wn; i += kDecThreads) {
+          const int tk = ids[w0 - soff + i];
+          sm.ids[i] = (unsigned)tk < (unsigned)len ? tk : -1;   // ids outside [0, len) are ignored
+        }
+        __syncthreads();
+        const int nst = (wn + kStageTok - 1) / kStageTok;
+        auto issue = [&](int st) {
+          if (st < nst) {
+            const int slot = st % kStages;
+#pragma unroll
+            for (int x = tid; x < kStageTok * 32; x += kDecThreads) {
+              const int j = x >> 5, part_ = x & 31;
+              const int pos = st * kStageTok + j;
+              const int tk = pos < wn ? sm.ids[pos] : -1;
+              if (tk >= 0) {
+                const int64_t row = L.row(b, hk, tk);
+                const __half* src = (part_ < 16 ? K : V) + row * kHeadDim + (part_ & 15) * 8;
+                cp_async16(&sm.u.kv[slot][j][part_ >> 4][(part_ & 15) * 8], src);
+              }
+            }
+          }
+          cp_async_commit();
+        };
+#pragma unroll
+        for (int st = 0; st < kStages - 1; ++st) issue(st);
+        for (int st = 0; st < nst; ++st) {
+          issue(st + kStages - 1);
+          cp_async_wait<kStages - 1>();
+          __syncthreads();
+          const int slot = st % kStages;
+          float sc[NH][2];
+          bool ok[2];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * hw + jj;
+            const int pos = st * kStageTok + j;
+            ok[jj] = pos < wn && sm.ids[pos] >= 0;
+            float kf[8];
+            h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][j][0][8 * l16])
+                            : make_uint4(0u, 0u, 0u, 0u),
+                     kf);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              float s0 = qf[h][0] * kf[0];
+#pragma unroll
+              for (int dd = 1; dd < 8; ++dd) s0 = __fmaf_rn(qf[h][dd], kf[dd], s0);
+              sc[h][jj] = s0;
+            }
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              sc[h][0] += __shfl_xor_sync(hmask, sc[h][0], o, 16);
+              sc[h][1] += __shfl_xor_sync(hmask, sc[h][1], o, 16);
+            }
+          if (ok[0] || ok[1]) {   // uniform across the half-warp
+            float vf[2][8];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+              h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][2 * hw + jj][1][8 * l16])
+                              : make_uint4(0u, 0u, 0u, 0u),
+                       vf[jj]);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              float mb = m[h];
+              if (ok[0]) mb = fmaxf(mb, sc[h][0]);
+              if (ok[1]) mb = fmaxf(mb, sc[h][1]);
+              const float corr = exp2f(m[h] - mb);
+              const float p0 = ok[0] ? exp2f(sc[h][0] - mb) : 0.f;
+              const float p1 = ok[1] ? exp2f(sc[h][1] - mb) : 0.f;
+              l[h] = l[h] * corr + (p0 + p1);
+#pragma unroll
+              for (int dd = 0; dd < 8; ++dd)
+                acc[h][dd] = __fmaf_rn(p1, vf[1][dd], __fmaf_rn(p0, vf[0][dd], acc[h][dd] * corr));
+              m[h] = mb;
+            }
+          }
+          __syncthreads();   // this slot is refilled by a later issue()
+        }
+        cp_async_wait<0>();
+      }
+      // fold the 8 half-warps and write this CTA's record for the set
+      __syncthreads();
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (l16 == 0) {
+          sm.u.comb.m[hw][h] = m[h];
+          sm.u.comb.l[hw][h] = l[h];
+        }
+        *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16]) =
+            make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+        *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16 + 4]) =
+            make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+      }
+      __syncthreads();
+      float* rec = part + ((int64_t)(c + set) * NH) * kPartStride;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecHW; ++w) M = fmaxf(M, sm.u.comb.m[w][h]);
+        float Ls = 0.f, A = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecHW; ++w) {
+          const float f = sm.u.comb.m[w][h] == -INFINITY ? 0.f : exp2f(sm.u.comb.m[w][h] - M);
+          Ls += sm.u.comb.l[w][h] * f;
+          A += sm.u.comb.acc[w][h][tid] * f;
+        }
+        rec[h * kPartStride + kPartAcc + tid] = A;
+        if (tid == 0) {
+          rec[h * kPartStride] = M;
+          rec[h * kPartStride + 1] = Ls;
+        }
+      }
+      // publish the record; the CTA that completes the set merges it
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        const int64_t c0 = ((soff + 1) * n + S - 1) / S - 1;
+        const int64_t c1 = ((soff + scnt) * n + S - 1) / S - 1;
+        int nrec = 0;
+        if (S >= n) {
+          nrec = (int)(c1 - c0 + 1);
+        } else {
+          for (int64_t cc = c0; cc <= c1; ++cc) nrec += range_has(cc, S, n, soff, scnt) ? 1 : 0;
+        }
+        const int prev = atomicAdd(&done[set], 1);
+        sm.last = (prev == nrec - 1);
+      }
+      __syncthreads();
+      if (sm.last) {
+        __threadfence();
+        merge_set<NH>(sm, set, soff, scnt, S, n, Hq, hq0, b, part, out, lse);
+        if (tid == 0) done[set] = 0;   // ready for the next call
+      }
+    }
+    __syncthreads();
   }
-  out[(int64_t)bh * kHeadDim + d] = __float2half_rn(Ls > 0.f ? A / Ls : 0.f);
-  if (lse && d == 0) lse[bh] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  griddep_launch();
 }
 
-int decode_split_tokens(int sets, int icap) {
-  int T = 1024;
-  while (T > 64 && (int64_t)sets * ((icap + T - 1) / T) < 4 * kTargetSms) T >>= 1;
-  return T;
+size_t decode_part_floats(int B, int Hq, int Hk) {
+  const int G = Hq / Hk;
+  const size_t grp = (size_t)(kDecCtas + B * Hk) * G * kPartStride;
+  const size_t head = (size_t)(kDecCtas + B * Hq) * kPartStride;
+  return grp > head ? grp : head;
 }
 
-void launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
-                          const __half* K, const __half* V, const int32_t* idx, int icap,
-                          const int32_t* count, float* part, __half* out, float* lse,
-                          cudaStream_t st, bool merge_only, bool decode_only) {
+cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
+                                 const __half* K, const __half* V, const int32_t* idx, int icap,
+                                 const int32_t* count, float* part, int32_t* done, __half* out,
+                                 float* lse, cudaStream_t st, bool pdl) {
   const int G = Hq / L.Hk;
   const int NH = group_sets ? G : 1;
-  const int sets = group_sets ? L.B * L.Hk : L.B * Hq;
-  const int T = decode_split_tokens(sets, icap);
-  const int S = (icap + T - 1) / T;
-  if (!merge_only) {
-    dim3 grid(S, sets);
-    switch (NH) {
-#define TW_DEC(NN)                                                                          \
-  case NN:                                                                                  \
-    k_sparse_decode<NN><<<grid, kDecThreads, 0, st>>>(L, q, Hq, G, group_sets, K, V, idx,    \
-                                                      icap, count, T, S, part);              \
-    break;
-      TW_DEC(1) TW_DEC(2) TW_DEC(4) TW_DEC(8)
+  const int nsets = group_sets ? L.B * L.Hk : L.B * Hq;
+  switch (NH) {
+#define TW_DEC(NN)                                                                           \
+  case NN:                                                                                   \
+    return launch_k(k_sparse_decode<NN>, dim3(kDecCtas), dim3(kDecThreads), 0, st, pdl, L, q, \
+                    Hq, G, group_sets, K, V, idx, icap, count, nsets, part, done, out, lse);
+    TW_DEC(1) TW_DEC(2) TW_DEC(4) TW_DEC(8)
 #undef TW_DEC
-    }
   }
-  if (!decode_only)
-    k_merge<<<L.B * Hq, kHeadDim, 0, st>>>(Hq, L.Hk, G, group_sets, count, icap, T, S, part, out,
-                                           lse);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace tw

@@ -102,4 +102,14 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p) {
   return r;
 }
 
+// Programmatic dependent launch: wait until the preceding kernel in the stream
+// has completed and its writes are visible (a no-op without the launch
+// attribute), and let the next kernel begin launching.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace tw

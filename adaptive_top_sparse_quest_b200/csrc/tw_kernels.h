@@ -5,11 +5,33 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "tw_common.cuh"
 
 namespace tw {
 
-constexpr int kEstTile = 256;        // candidates per estimate block (and per tile statistic)
+// Launch with an optional programmatic-stream-serialization attribute (PDL):
+// the kernel may start while its predecessor drains; it calls griddep_wait()
+// before touching anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
+constexpr int kEstTile = 256;        // candidates per estimate work item
+constexpr int kStatSpan = 32;        // candidates per softmax-statistics record
 constexpr int kPartStride = 132;     // floats per split record: m, l, 2 pad, acc[128]
 constexpr int kPartAcc = 4;
 constexpr int kTargetSms = 148;      // B200 SM count used to size decode splits
@@ -19,23 +41,26 @@ void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __ha
                           __half* zeros, cudaStream_t st, int num_sms);
 void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream_t st,
                       int num_sms);
-void launch_page_scores(const Layout& L, const __half* q, int Hq, const __half* meta,
-                        float* scores, cudaStream_t st);
-void launch_page_topk(const Layout& L, const float* scores, int budget_pages, int32_t* cand,
-                      int cand_stride, int32_t* ncand, cudaStream_t st);
-void launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
-                     const __half* scales, const __half* zeros, const int32_t* cand,
-                     int cand_stride, const int32_t* ncand, int cap, int cmax, float* logits,
-                     float2* stats, cudaStream_t st);
-int topp_cluster_shape(int cmax, int* R, int* CS);
+cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
+                            const __half* scales, const __half* zeros, const int32_t* cand,
+                            int cand_stride, const int32_t* ncand, int lcap, int cmax,
+                            float* logits, float2* stats, cudaStream_t st, int num_sms,
+                            bool pdl);
+int topp_shape(int cmax, int* R, int* CS);
 cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* cand,
                         int cand_stride, const int32_t* ncand, int lcap, int cmax,
                         const float* logits, const float2* stats, double p, int32_t* idx,
-                        int icap, int32_t* count, cudaStream_t st);
-int decode_split_tokens(int sets, int icap);
-void launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
-                          const __half* K, const __half* V, const int32_t* idx, int icap,
-                          const int32_t* count, float* part, __half* out, float* lse,
-                          cudaStream_t st, bool merge_only, bool decode_only);
+                        int icap, int32_t* count, int32_t* done, cudaStream_t st, bool pdl);
+constexpr int kDecCtas = 4 * kTargetSms;   // CTAs sharing the concatenated selected tokens
+size_t decode_part_floats(int B, int Hq, int Hk);
+cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
+                                 const __half* K, const __half* V, const int32_t* idx, int icap,
+                                 const int32_t* count, float* part, int32_t* done, __half* out,
+                                 float* lse, cudaStream_t st, bool pdl);
+cudaError_t launch_page_scores(const Layout& L, const __half* q, int Hq, const __half* meta,
+                               float* scores, cudaStream_t st, int num_sms, bool pdl);
+cudaError_t launch_page_topk(const Layout& L, const float* scores, int budget_pages,
+                             int32_t* cand, int cand_stride, int32_t* ncand, cudaStream_t st,
+                             bool pdl);
 
 }  // namespace tw

@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--copies", type=int, default=0,
+                    help="rotating cache copies (0: enough to exceed L2 several times)")
     return ap.parse_args()
 
 
@@ -292,6 +294,8 @@ def main():
     while R * min(copy_bytes, 4 * touched_est) < 4 * L2_BYTES and R < 16:
         R += 1
     R = max(R, 4)
+    if args.copies > 0:
+        R = args.copies
 
     # cache-build kernels timed once (GB/s over K read + int4/meta written)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
