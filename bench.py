@@ -83,6 +83,23 @@ def src_hash():
     return h.hexdigest()[:16]
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (the job's time is its slowest rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_step(max_elapsed_ms: float, steps: int, world: int) -> float:
+    """Replicas: every rank runs `steps` independent decode steps, so the job
+    completes steps * world steps in the slowest rank's time."""
+    return max_elapsed_ms * 1e3 / (steps * world)
+
+
 def hbm_peak():
     try:
         pk = json.load(open(PEAKS_PATH))
@@ -353,12 +370,9 @@ def main():
                 n_extra += 1
             torch.cuda.synchronize()
         t_load_end = time.time()
-    t_max = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = reduce_max(elapsed_ms, world, dev)
     us_per_step = elapsed_ms * 1e3 / args.steps
-    value = us_per_step / world
+    value = whole_job_us_per_step(elapsed_ms, args.steps, world)
 
     # per-kernel durations: the same step with an event after each kernel
     names = steps[0].kernel_names()
@@ -399,11 +413,7 @@ def main():
     e1.record(stream)
     e1.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    t2 = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_us = float(t2.item()) * 1e3 / args.steps / world
+    e2e_us = whole_job_us_per_step(reduce_max(e0.elapsed_time(e1), world, dev), args.steps, world)
 
     if sampler:
         sampler.stop()
