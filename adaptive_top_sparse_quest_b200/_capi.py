@@ -59,6 +59,9 @@ _SIGS = {
                                      c_size, c_vp]),
     "tw_sparse_decode": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_i32, c_vp,
                                         c_i32, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "tw_topp_prune_noalloc": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_vp, c_vp,
+                                             c_vp, c_i32, c_vp, ctypes.c_double, c_i32, c_vp,
+                                             c_i32, c_vp, c_vp]),
     "tw_decode_step": (ctypes.c_int, [ctypes.POINTER(TwStep), c_vp]),
     "tw_decode_step_num_kernels": (ctypes.c_int, [ctypes.POINTER(TwStep)]),
     "tw_decode_step_kernel_name": (ctypes.c_char_p, [ctypes.POINTER(TwStep), c_i32]),

@@ -179,6 +179,28 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
                      int32_t group_mode, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
                      void* stream);
 
+/*
+ * tw_topp_prune without a workspace, for callers that cannot allocate device
+ * memory (a runtime recording the step into a CUDA graph with allocation
+ * forbidden, a plugin whose enqueue hook may not allocate, a server that fixes
+ * its device memory at start-up).  The paper has no counterpart to this call:
+ * it exists only for that calling constraint.
+ * Same inputs, outputs and results as tw_topp_prune; the scratch is one fixed
+ * array of TW_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library, resident
+ * on every GPU that loads it until the process exits.  Shapes whose scratch
+ * (logits and softmax statistics: about B * Hk * capacity * G * 4 bytes) does
+ * not fit return TW_ERR_CAPACITY before any device work.  The first call on a
+ * device looks up the array's device address (TW_ERR_CUDA if that fails), so
+ * make it before any stream capture.  Every call shares the array: calls that
+ * overlap on the GPU race.  Nothing in it needs to start at zero.
+ */
+#define TW_NOALLOC_SCRATCH_BYTES (8u << 20)
+int tw_topp_prune_noalloc(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                          const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                          const int32_t* cand_pages, int32_t cand_stride, const int32_t* ncand,
+                          double p, int32_t group_mode, int32_t* idx, int32_t capacity,
+                          int32_t* count, void* stream);
+
 /* One decode step: tw_select_pages (skipped when budget_tokens <= 0, every token
  * is then a candidate) -> tw_topp_prune -> tw_sparse_decode, enqueued back to
  * back on one stream with no host synchronisation. */
