@@ -76,10 +76,11 @@ int check_heads(int Hq, int Hk) {
   return TW_OK;
 }
 
-// Workspace regions, in order: page scores | logits | softmax statistics |
-// per-set completion counters | attention partial records.
+// Workspace regions, in order: status word | page scores | logits | softmax
+// statistics | per-set completion counters | attention partial records.  The
+// status word collects device-side error bits (a bounded wait that gave up).
 struct Plan {
-  size_t scores_off, logits_off, stats_off, done_off, part_off;
+  size_t status_off, scores_off, logits_off, stats_off, done_off, part_off;
   size_t scores_end, topp_end, total;
   int lcap;
 };
@@ -89,8 +90,9 @@ Plan make_plan(int B, int Hq, int Hk, int N, int cap) {
   const int G = Hq / Hk;
   const int64_t pmax = (N + tw::kPage - 1) / tw::kPage;
   p.lcap = (int)(((int64_t)cap + tw::kEstTile - 1) / tw::kEstTile * tw::kEstTile);
-  p.scores_off = 0;
-  p.scores_end = align256((size_t)B * Hk * pmax * sizeof(float));
+  p.status_off = 0;
+  p.scores_off = 256;
+  p.scores_end = p.scores_off + align256((size_t)B * Hk * pmax * sizeof(float));
   p.logits_off = p.scores_end;
   p.stats_off = p.logits_off + align256((size_t)B * Hk * p.lcap * G * sizeof(float));
   p.topp_end = p.stats_off +

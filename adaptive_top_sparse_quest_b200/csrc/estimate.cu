@@ -5,91 +5,79 @@
 //
 // For candidate i, query head h and 32-channel group g with scale s, zero z:
 //   k_hat = z + s * c = (z + 8 s) + s * (c - 8),  c in 0..15
-//   l[i,h] = sum_g ( s_ig * D[h,g,i] + (z_ig + 8 s_ig) * Q[h,g] ) / sqrt(128)
-//   D[h,g,i] = sum_{j in g} q_hj * (c_ij - 8),   Q[h,g] = sum_{j in g} q_hj
+//   l[i,h] = sum_g ( s_ig * D[i,h,g] + (z_ig + 8 s_ig) * Q[h,g] ) / sqrt(128)
+//   D[i,h,g] = sum_{j in g} (c_ij - 8) * q_hj,   Q[h,g] = sum_{j in g} q_hj
 // The D terms are a small dense contraction, run on the tensor cores with
 // mma.sync m16n8k16 (fp16 operands, fp32 accumulation): (c - 8) and the fp16
-// queries are exact in fp16 and their products exact in fp32.  The MMA's M
-// rows are (head, group) pairs (row 4h + g), N is 8 candidates, K is 16
-// channels per step; each row keeps only its own group's channels, so after 8
-// K-steps every row holds one D[h,g,*] and the per-group scales are applied in
-// the fp32 epilogue.  The K order is permuted so that lane (gid, t) feeds
-// exactly the codes of candidate gid, group t it loaded: 16 B of codes become
-// 8 half2 B-fragments with one shift, one LOP3 (nibbles -> 0x6400|c, i.e.
-// 1024 + c) and one half2 subtract of 1032 each.  M = 16 rows cover 4 heads
-// (GQA 4:1); 8 heads take two row blocks.
+// queries are exact in fp16 and their products exact in fp32.  M = 16
+// candidates, N = 8 columns = (head, group) pairs of two heads, K = 16
+// channels per step; column (h, g) keeps only group g's channels of q_h, so
+// after 8 K-steps every column holds one D[*,h,g] and the per-group scales are
+// applied in the fp32 epilogue, where one xor-shuffle adds the lane pair that
+// holds the other two groups.  The K order is permuted so that lane (gid, t)
+// feeds exactly the 16 B of codes of candidates gid and gid+8, group t, it
+// reads: each code pair becomes a half2 A-fragment with one shift, one LOP3
+// (nibbles -> 0x6400|c, i.e. 1024 + c) and one half2 subtract of 1032.
+// Logits are kept in log2 units (log2(e) folded into the 1/sqrt(128) factor),
+// so the statistics and the top-p kernel use exp2.
 //
-// Persistent kernel: each CTA owns a contiguous block of (kv unit,
-// 256-candidate) items, 32 candidates per warp (4 MMA tiles of 8), and loads
-// item i+1's codes and item i+2's candidate page ids while computing item i.
-// Each warp writes the per-head max and sum exp(l - max) of its 32 logits so
-// the top-p kernel starts from softmax statistics without another pass.
+// Data path.  Persistent CTAs (two per SM) each own a contiguous block of
+// work items (kv unit, 16 candidate pages = 256 candidates: 16 KB of codes +
+// 2 KB of scales + 2 KB of zeros).  A 4-stage shared-memory ring is filled
+// with cp.async by all threads (16-byte chunks of codes, 8-byte rows of
+// scales and zeros) three items ahead, and warp 0 looks up the page ids of the
+// item after that, so the id lookups and the row gathers both stay off the
+// critical path.  Each of the eight warps then takes 32 candidates (two MMA
+// tiles) and writes the fp32 logits [unit][cap][G] plus its per-head
+// (max, sum 2^(l - max)).
 #include "tw_common.cuh"
 #include "tw_kernels.h"
 
 namespace tw {
 
 constexpr int kEstThreads = 256;
-constexpr int kEstTiles = 4;                  // 4 MMA tiles x 8 candidates = 32 per warp
-constexpr float kInvSqrtD = 0.08838834764831845f;
+constexpr int kEstStages = 4;
+constexpr int kEstTiles = 2;                             // MMA tiles of 16 candidates per warp
+constexpr int kPagesPerItem = kEstTile / kPage;          // 16
+constexpr float kL2Scale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
 
-struct EstLoad {
-  uint4 cw[kEstTiles];       // 16 B of codes: candidate gid of tile k, group t
-  uint32_t sz[kEstTiles];    // fp16 scale (low half) and zero (high half) of that group
+struct EstStage {
+  uint8_t codes[kEstTile][kHeadDim / 2];
+  __half scales[kEstTile][kGroups];
+  __half zeros[kEstTile][kGroups];
 };
 
-struct EstIds {
-  int len, C;
-  int pg[kEstTiles];
+// Where the 16 pages of an item live: first global row and valid rows (0 = none).
+struct EstPages {
+  long long row0[kPagesPerItem];
+  int rows[kPagesPerItem];
 };
 
-__device__ __forceinline__ void est_issue_ids(const Layout& L, const int32_t* cand,
-                                              int cand_stride, const int32_t* ncand, int cmax,
-                                              int tiles, int it, int warp, int gid, EstIds& r) {
-  const int u = it / tiles;
-  const int b = u / L.Hk;
-  r.len = L.len(b);
-  r.C = cand ? ncand[u] * kPage : r.len;
-#pragma unroll
-  for (int k = 0; k < kEstTiles; ++k) {
-    const int c = (it % tiles) * kEstTile + warp * 32 + k * 8 + gid;
-    r.pg[k] = 0;
-    if (cand && (c >> 4) < cand_stride && c < cmax) r.pg[k] = cand[(int64_t)u * cand_stride + (c >> 4)];
-  }
-}
+struct EstSmem {
+  EstStage st[kEstStages];
+  EstPages pg[kEstStages + 1];
+};
 
-__device__ __forceinline__ void est_tokens(const EstIds& r, bool has_cand, int cmax, int tiles,
-                                           int it, int warp, int gid, int tok[kEstTiles]) {
-  const int C = min(r.C, cmax);
-#pragma unroll
-  for (int k = 0; k < kEstTiles; ++k) {
-    const int c = (it % tiles) * kEstTile + warp * 32 + k * 8 + gid;
-    int t = -1;
-    if (c < C) {
-      t = has_cand ? r.pg[k] * kPage + (c & 15) : c;
-      if (t < 0 || t >= r.len) t = -1;
-    }
-    tok[k] = t;
-  }
-}
+constexpr size_t kEstSmemBytes = sizeof(EstSmem);
 
-__device__ __forceinline__ void est_issue_codes(const Layout& L, const uint8_t* codes,
-                                                const __half* scales, const __half* zeros,
-                                                int tiles, int it, int t,
-                                                const int tok[kEstTiles], EstLoad& d) {
-  const int u = it / tiles;
-  const int b = u / L.Hk, hk = u % L.Hk;
-#pragma unroll
-  for (int k = 0; k < kEstTiles; ++k) {
-    d.cw[k] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-    d.sz[k] = 0u;
-    if (tok[k] >= 0) {
-      const int64_t row = L.row(b, hk, tok[k]);
-      d.cw[k] = ld_stream16(codes + row * (kHeadDim / 2) + t * 16);
-      d.sz[k] = (uint32_t)__half_as_ushort(scales[row * kGroups + t]) |
-                ((uint32_t)__half_as_ushort(zeros[row * kGroups + t]) << 16);
-    }
-  }
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (unsigned)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                   (unsigned)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -113,14 +101,60 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-// RB: 16-row blocks of (head, group) pairs, ceil(G / 4).
+// Page lookup of item `it` (lanes 0..15 of one warp): global first row and
+// valid rows of each of its 16 candidate pages.
+__device__ __forceinline__ void est_pages(const Layout& L, const int32_t* cand, int cand_stride,
+                                          const int32_t* ncand, int cmax, int tiles, int it,
+                                          int lane, EstPages& out) {
+  if (lane >= kPagesPerItem) return;
+  const int u = it / tiles;
+  const int b = u / L.Hk, hk = u % L.Hk;
+  const int len = L.len(b);
+  const int C = min(cand ? ncand[u] * kPage : len, cmax);
+  const int lp = (it % tiles) * kPagesPerItem + lane;   // logical candidate page
+  int rows = 0;
+  long long row0 = 0;
+  if (lp * kPage < C) {
+    const int page = cand ? (lp < cand_stride ? cand[(int64_t)u * cand_stride + lp] : -1) : lp;
+    if (page >= 0 && page < L.max_pages) {
+      rows = max(0, min(kPage, len - page * kPage));
+      if (rows > 0) row0 = L.page_row(b, hk, page);
+    }
+  }
+  out.rows[lane] = rows;
+  out.row0[lane] = row0;
+}
+
+// All threads: gather item `it` (pages already looked up) into a ring stage.
+__device__ __forceinline__ void est_issue(const EstPages& pg, const uint8_t* codes,
+                                          const __half* scales, const __half* zeros,
+                                          EstStage& st) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {   // codes: 1024 chunks of 16 B
+    const int x = tid + k * kEstThreads;
+    const int c = x >> 2, part = x & 3, p = c >> 4, r = c & 15;
+    if (r < pg.rows[p])
+      cp_async16(&st.codes[c][16 * part], codes + (pg.row0[p] + r) * (kHeadDim / 2) + 16 * part);
+  }
+  {   // scales and zeros: one 8-byte row each per thread
+    const int c = tid, p = c >> 4, r = c & 15;
+    if (r < pg.rows[p]) {
+      cp_async8(&st.scales[c][0], scales + (pg.row0[p] + r) * kGroups);
+      cp_async8(&st.zeros[c][0], zeros + (pg.row0[p] + r) * kGroups);
+    }
+  }
+}
+
 template <int G>
-__global__ void __launch_bounds__(kEstThreads)
+__global__ void __launch_bounds__(kEstThreads, 2)
 k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __restrict__ codes,
            const __half* __restrict__ scales, const __half* __restrict__ zeros,
            const int32_t* __restrict__ cand, int cand_stride, const int32_t* __restrict__ ncand,
            int lcap, int cmax, float* __restrict__ logits, float2* __restrict__ stats) {
-  constexpr int RB = (G + 3) / 4;
+  constexpr int HP = (G + 1) / 2;   // head pairs: one MMA N-block of 8 (head, group) columns each
+  extern __shared__ __align__(128) unsigned char est_smem_raw[];
+  EstSmem& sm = *reinterpret_cast<EstSmem*>(est_smem_raw);
   const int tiles = lcap / kEstTile;
   const int items = L.B * L.Hk * tiles;
   const int per = (items + gridDim.x - 1) / gridDim.x;
@@ -128,180 +162,161 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
   const int it1 = min(items, it0 + per);
   if (it0 >= it1) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, t = lane & 3;
-  const int g = gid & 3;                 // group of the MMA rows this lane holds
-  const int nspan = lcap / kStatSpan;
-  const bool has_cand = cand != nullptr;
-
-  int tokA[kEstTiles], tokB[kEstTiles];
-  EstIds ids;
-  EstLoad A, B;
   griddep_wait();
-  est_issue_ids(L, cand, cand_stride, ncand, cmax, tiles, it0, warp, gid, ids);
-  est_tokens(ids, has_cand, cmax, tiles, it0, warp, gid, tokA);
-  est_issue_codes(L, codes, scales, zeros, tiles, it0, t, tokA, A);
-  if (it0 + 1 < it1) {
-    est_issue_ids(L, cand, cand_stride, ncand, cmax, tiles, it0 + 1, warp, gid, ids);
-    est_tokens(ids, has_cand, cmax, tiles, it0 + 1, warp, gid, tokB);
+  // pipeline prologue: page lookups for items it0 .. it0+S-1, then their gathers
+  if (warp == 0)
+    for (int j = 0; j < kEstStages && it0 + j < it1; ++j)
+      est_pages(L, cand, cand_stride, ncand, cmax, tiles, it0 + j, lane, sm.pg[j]);
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kEstStages - 1; ++j) {
+    if (it0 + j < it1) est_issue(sm.pg[j], codes, scales, zeros, sm.st[j]);
+    cp_async_commit();
   }
-  uint32_t afr[RB][8][4];
-  float qsum[RB][2];
+  const int gid = lane >> 2, t = lane & 3;
+  const int g0 = 2 * (t & 1);            // this lane's two groups in the epilogue: g0, g0 + 1
+  const int nspan = lcap / kStatSpan;
+  uint32_t bfr[HP][8][2];                // B fragments: column gid = (head 2hp + gid/4, group gid%4)
+  float Qv[HP][2];                       // Q[h][g0], Q[h][g0+1] for the lane's epilogue head
   int staged = -1;
   for (int it = it0; it < it1; ++it) {
-    if (it + 1 < it1) est_issue_codes(L, codes, scales, zeros, tiles, it + 1, t, tokB, B);
-    if (it + 2 < it1) est_issue_ids(L, cand, cand_stride, ncand, cmax, tiles, it + 2, warp, gid, ids);
+    const int j = it - it0, slot = j % kEstStages;
+    // refill: gather item j+S-1 into the slot item j-1 used, and look up the
+    // pages of item j+S (their ring entries were last read one iteration ago)
+    __syncthreads();
+    if (it + kEstStages - 1 < it1)
+      est_issue(sm.pg[(j + kEstStages - 1) % (kEstStages + 1)], codes, scales, zeros,
+                sm.st[(j + kEstStages - 1) % kEstStages]);
+    cp_async_commit();
+    if (warp == 0 && it + kEstStages < it1)
+      est_pages(L, cand, cand_stride, ncand, cmax, tiles, it + kEstStages, lane,
+                sm.pg[(j + kEstStages) % (kEstStages + 1)]);
     const int u = it / tiles;
     const int b = u / L.Hk, hk = u % L.Hk;
     if (u != staged) {
-      // A fragments: row gid = (head rb*4 + gid/4, group g), row gid+8 = head + 2.
-      // They are non-zero only where the K slots belong to the row's group (t == g).
 #pragma unroll
-      for (int rb = 0; rb < RB; ++rb) {
-        const int h0 = rb * 4 + (gid >> 2), h1 = h0 + 2;
-        const __half* q0 = q + ((int64_t)b * Hq + hk * G + h0) * kHeadDim;
-        const __half* q1 = q + ((int64_t)b * Hq + hk * G + h1) * kHeadDim;
-        const bool on = (t == g);
-        const bool v0 = on && h0 < G, v1 = on && h1 < G;
-        float s0 = 0.f, s1 = 0.f;
+      for (int hp = 0; hp < HP; ++hp) {
+        const int hb = 2 * hp + (gid >> 2);   // head of B column gid
+        const bool on = ((gid & 3) == t) && hb < G;
+        const __half* qb = q + ((int64_t)b * Hq + hk * G + min(hb, G - 1)) * kHeadDim;
+        const __half z = __float2half_rn(0.f);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const int e = (s & 1) * 2, base = 32 * t + 8 * (s >> 1);
-          const __half z = __float2half_rn(0.f);
-          const __half x00 = v0 ? q0[base + e] : z, x01 = v0 ? q0[base + e + 4] : z;
-          const __half x02 = v0 ? q0[base + e + 1] : z, x03 = v0 ? q0[base + e + 5] : z;
-          const __half x10 = v1 ? q1[base + e] : z, x11 = v1 ? q1[base + e + 4] : z;
-          const __half x12 = v1 ? q1[base + e + 1] : z, x13 = v1 ? q1[base + e + 5] : z;
-          afr[rb][s][0] = pack_h2(x00, x01);
-          afr[rb][s][1] = pack_h2(x10, x11);
-          afr[rb][s][2] = pack_h2(x02, x03);
-          afr[rb][s][3] = pack_h2(x12, x13);
-          s0 += (__half2float(x00) + __half2float(x01)) + (__half2float(x02) + __half2float(x03));
-          s1 += (__half2float(x10) + __half2float(x11)) + (__half2float(x12) + __half2float(x13));
+          bfr[hp][s][0] = pack_h2(on ? qb[base + e] : z, on ? qb[base + e + 4] : z);
+          bfr[hp][s][1] = pack_h2(on ? qb[base + e + 1] : z, on ? qb[base + e + 5] : z);
         }
-        qsum[rb][0] = s0;   // Q[h0][g] on lanes with t == g
-        qsum[rb][1] = s1;
+        const int he = 2 * hp + (t >> 1);     // head of this lane's epilogue columns
+        const __half* qe = q + ((int64_t)b * Hq + hk * G + min(he, G - 1)) * kHeadDim;
+        float s0 = 0.f, s1 = 0.f;
+        for (int d = 0; d < kGroup; ++d) {
+          s0 += __half2float(qe[g0 * kGroup + d]);
+          s1 += __half2float(qe[(g0 + 1) * kGroup + d]);
+        }
+        Qv[hp][0] = s0;
+        Qv[hp][1] = s1;
       }
       staged = u;
     }
-    const int cw0 = (it % tiles) * kEstTile + warp * 32;
-    const int Cu = min(has_cand ? __ldg(ncand + u) * kPage : L.len(b), cmax);
-    float mlo[RB], mhi[RB];
-    float lgv[kEstTiles][RB][4];
-#pragma unroll
-    for (int rb = 0; rb < RB; ++rb) mlo[rb] = mhi[rb] = -INFINITY;
+    cp_async_wait<kEstStages - 1>();
+    __syncthreads();
+    const EstPages& pgs = sm.pg[j % (kEstStages + 1)];
+    const EstStage& st = sm.st[slot];
+    const int cw0 = (it % tiles) * kEstTile + warp * 32;   // this warp's first candidate
+    const int Cu = min(cand ? __ldg(ncand + u) * kPage : L.len(b), cmax);
+    float lg[kEstTiles][HP][2];
 #pragma unroll
     for (int k = 0; k < kEstTiles; ++k) {
-      float acc[RB][4];
+      const int ca = warp * 32 + k * 16 + gid, cb = ca + 8;   // candidates (rows gid, gid+8)
+      const uint4 wa = *reinterpret_cast<const uint4*>(&st.codes[ca][16 * t]);
+      const uint4 wb = *reinterpret_cast<const uint4*>(&st.codes[cb][16 * t]);
+      const bool va = (ca & 15) < pgs.rows[ca >> 4];
+      const bool vb = (cb & 15) < pgs.rows[cb >> 4];
+      float acc[HP][4];
 #pragma unroll
-      for (int rb = 0; rb < RB; ++rb) acc[rb][0] = acc[rb][1] = acc[rb][2] = acc[rb][3] = 0.f;
-      const uint32_t w[4] = {A.cw[k].x, A.cw[k].y, A.cw[k].z, A.cw[k].w};
+      for (int hp = 0; hp < HP; ++hp) acc[hp][0] = acc[hp][1] = acc[hp][2] = acc[hp][3] = 0.f;
+      const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const uint32_t W = w[s >> 1];
         const int e = (s & 1) * 2;
-        const uint32_t b0 = nib_pair(W, e), b1 = nib_pair(W, e + 1);
+        const uint32_t a[4] = {nib_pair(WA[s >> 1], e), nib_pair(WB[s >> 1], e),
+                               nib_pair(WA[s >> 1], e + 1), nib_pair(WB[s >> 1], e + 1)};
 #pragma unroll
-        for (int rb = 0; rb < RB; ++rb) mma16816(acc[rb], afr[rb][s], b0, b1);
+        for (int hp = 0; hp < HP; ++hp) mma16816(acc[hp], a, bfr[hp][s][0], bfr[hp][s][1]);
       }
-      // epilogue: this lane holds rows (h0, g), (h1, g) for candidates 2t, 2t+1
-      const uint32_t sz0 = __shfl_sync(0xffffffffu, A.sz[k], (2 * t) * 4 + g);
-      const uint32_t sz1 = __shfl_sync(0xffffffffu, A.sz[k], (2 * t + 1) * 4 + g);
-      const int tk0 = __shfl_sync(0xffffffffu, tokA[k], (2 * t) * 4);
-      const int tk1 = __shfl_sync(0xffffffffu, tokA[k], (2 * t + 1) * 4);
-      const float sc0 = __half2float(__ushort_as_half((unsigned short)(sz0 & 0xFFFF)));
-      const float sc1 = __half2float(__ushort_as_half((unsigned short)(sz1 & 0xFFFF)));
-      const float zz0 = __fmaf_rn(8.f, sc0, __half2float(__ushort_as_half((unsigned short)(sz0 >> 16))));
-      const float zz1 = __fmaf_rn(8.f, sc1, __half2float(__ushort_as_half((unsigned short)(sz1 >> 16))));
+      // scales / zeros of groups g0, g0+1 for both candidates (fp16 pairs)
+      const __half2 sa = *reinterpret_cast<const __half2*>(&st.scales[ca][g0]);
+      const __half2 za = *reinterpret_cast<const __half2*>(&st.zeros[ca][g0]);
+      const __half2 sb = *reinterpret_cast<const __half2*>(&st.scales[cb][g0]);
+      const __half2 zb = *reinterpret_cast<const __half2*>(&st.zeros[cb][g0]);
+      const float2 fsa = __half22float2(sa), fza = __half22float2(za);
+      const float2 fsb = __half22float2(sb), fzb = __half22float2(zb);
+      const float zza0 = __fmaf_rn(8.f, fsa.x, fza.x), zza1 = __fmaf_rn(8.f, fsa.y, fza.y);
+      const float zzb0 = __fmaf_rn(8.f, fsb.x, fzb.x), zzb1 = __fmaf_rn(8.f, fsb.y, fzb.y);
 #pragma unroll
-      for (int rb = 0; rb < RB; ++rb) {
-        const float Qlo = __shfl_sync(0xffffffffu, qsum[rb][0], gid * 4 + g);
-        const float Qhi = __shfl_sync(0xffffffffu, qsum[rb][1], gid * 4 + g);
-        float v[4];
-        v[0] = __fmaf_rn(sc0, acc[rb][0], zz0 * Qlo);
-        v[1] = __fmaf_rn(sc1, acc[rb][1], zz1 * Qlo);
-        v[2] = __fmaf_rn(sc0, acc[rb][2], zz0 * Qhi);
-        v[3] = __fmaf_rn(sc1, acc[rb][3], zz1 * Qhi);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[j] += __shfl_xor_sync(0xffffffffu, v[j], 4);
-          v[j] += __shfl_xor_sync(0xffffffffu, v[j], 8);
-        }
-        lgv[k][rb][0] = tk0 >= 0 ? v[0] * kInvSqrtD : -INFINITY;
-        lgv[k][rb][1] = tk1 >= 0 ? v[1] * kInvSqrtD : -INFINITY;
-        lgv[k][rb][2] = tk0 >= 0 ? v[2] * kInvSqrtD : -INFINITY;
-        lgv[k][rb][3] = tk1 >= 0 ? v[3] * kInvSqrtD : -INFINITY;
-        mlo[rb] = fmaxf(mlo[rb], fmaxf(lgv[k][rb][0], lgv[k][rb][1]));
-        mhi[rb] = fmaxf(mhi[rb], fmaxf(lgv[k][rb][2], lgv[k][rb][3]));
+      for (int hp = 0; hp < HP; ++hp) {
+        float pa = __fmaf_rn(fsa.x, acc[hp][0], zza0 * Qv[hp][0]);
+        pa = __fmaf_rn(fsa.y, acc[hp][1], __fmaf_rn(zza1, Qv[hp][1], pa));
+        float pb = __fmaf_rn(fsb.x, acc[hp][2], zzb0 * Qv[hp][0]);
+        pb = __fmaf_rn(fsb.y, acc[hp][3], __fmaf_rn(zzb1, Qv[hp][1], pb));
+        pa += __shfl_xor_sync(0xffffffffu, pa, 1);   // + the other two groups
+        pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+        lg[k][hp][0] = va ? pa * kL2Scale : -INFINITY;
+        lg[k][hp][1] = vb ? pb * kL2Scale : -INFINITY;
       }
     }
     if (cw0 < Cu) {
-      // logits [unit][lcap][G], written by the lanes with g == 0
-      if (g == 0) {
+      const bool owner = (t & 1) == 0;   // lanes t and t^1 hold the same logits
 #pragma unroll
-        for (int k = 0; k < kEstTiles; ++k) {
-          const int c0 = cw0 + k * 8 + 2 * t;
-#pragma unroll
-          for (int rb = 0; rb < RB; ++rb) {
-            const int h0 = rb * 4 + (gid >> 2), h1 = h0 + 2;
-            float* lp = logits + ((int64_t)u * lcap + c0) * G;
-            if (h0 < G) {
-              if (c0 < Cu) lp[h0] = lgv[k][rb][0];
-              if (c0 + 1 < Cu) lp[G + h0] = lgv[k][rb][1];
-            }
-            if (h1 < G) {
-              if (c0 < Cu) lp[h1] = lgv[k][rb][2];
-              if (c0 + 1 < Cu) lp[G + h1] = lgv[k][rb][3];
-            }
-          }
-        }
-      }
-      // this warp's softmax statistics per head (32 candidates)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int rb = h >> 2, hh = h & 3;   // head hh of block rb: slot lo if hh < 2, gid>>2 == hh & 1
-        const bool mine = g == 0 && ((gid >> 2) == (hh & 1));
-        const bool lo = hh < 2;
-        float m = mine ? (lo ? mlo[rb] : mhi[rb]) : -INFINITY;
-        m = warp_max(m);
-        float z = 0.f;
-        if (mine && m != -INFINITY) {
+      for (int hp = 0; hp < HP; ++hp) {
+        const int he = 2 * hp + (t >> 1);
+        const bool hv = he < G;
+        // logits [unit][lcap][G]
+        if (owner && hv) {
 #pragma unroll
           for (int k = 0; k < kEstTiles; ++k) {
-            const float a = lo ? lgv[k][rb][0] : lgv[k][rb][2];
-            const float c = lo ? lgv[k][rb][1] : lgv[k][rb][3];
-            if (a != -INFINITY) z += expf(a - m);
-            if (c != -INFINITY) z += expf(c - m);
+            const int c0 = cw0 + k * 16 + gid;
+            if (c0 < Cu) logits[((int64_t)u * lcap + c0) * G + he] = lg[k][hp][0];
+            if (c0 + 8 < Cu) logits[((int64_t)u * lcap + c0 + 8) * G + he] = lg[k][hp][1];
           }
         }
-        z = warp_sum(z);
-        if (lane == 0) stats[((int64_t)u * nspan + cw0 / kStatSpan) * G + h] = make_float2(m, z);
-      }
-    }
-    if (it + 2 < it1) est_tokens(ids, has_cand, cmax, tiles, it + 2, warp, gid, tokA);
-    // rotate the pipeline: A <- B (item it+1), tokB <- candidates of item it+2
+        // (max, sum 2^(l - max)) over this warp's 32 candidates for head he
+        float m = -INFINITY;
+        if (owner && hv) {
 #pragma unroll
-    for (int k = 0; k < kEstTiles; ++k) {
-      const int t2 = tokA[k];
-      tokA[k] = tokB[k];
-      tokB[k] = t2;
-      A.cw[k] = B.cw[k];
-      A.sz[k] = B.sz[k];
+          for (int k = 0; k < kEstTiles; ++k) m = fmaxf(m, fmaxf(lg[k][hp][0], lg[k][hp][1]));
+        }
+        float z = 0.f;
+        if (m != -INFINITY) {
+#pragma unroll
+          for (int k = 0; k < kEstTiles; ++k) {
+            if (lg[k][hp][0] != -INFINITY) z += exp2f(lg[k][hp][0] - m);
+            if (lg[k][hp][1] != -INFINITY) z += exp2f(lg[k][hp][1] - m);
+          }
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {   // fold the 8 lanes (gid) that share t
+          const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+          const float zo = __shfl_xor_sync(0xffffffffu, z, o);
+          const float mn = fmaxf(m, mo);
+          z = (m == -INFINITY ? 0.f : z * exp2f(m - mn)) + (mo == -INFINITY ? 0.f : zo * exp2f(mo - mn));
+          m = mn;
+        }
+        if (gid == 0 && owner && hv)
+          stats[((int64_t)u * nspan + cw0 / kStatSpan) * G + he] = make_float2(m, z);
+      }
     }
   }
   griddep_launch();
 }
 
 template <int G>
-static int est_grid(int num_sms) {
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_estimate<G>, kEstThreads, 0) !=
-            cudaSuccess || n < 1)
-      n = 1;
-    per_sm = n;
-  }
-  return num_sms * per_sm;
+static cudaError_t est_prepare() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaErrorNotReady)
+    done = cudaFuncSetAttribute(k_estimate<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kEstSmemBytes);
+  return done;
 }
 
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
@@ -311,13 +326,15 @@ cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint
                             bool pdl) {
   const int G = Hq / L.Hk;
   const int items = L.B * L.Hk * (lcap / kEstTile);
+  const int grid = items < 2 * num_sms ? items : 2 * num_sms;
   switch (G) {
 #define TW_EST(GG)                                                                          \
   case GG: {                                                                                \
-    const int grid = items < est_grid<GG>(num_sms) ? items : est_grid<GG>(num_sms);        \
-    return launch_k(k_estimate<GG>, dim3(grid), dim3(kEstThreads), 0, st, pdl, L, q, Hq,    \
-                    codes, scales, zeros, cand, cand_stride, ncand, lcap, cmax, logits,     \
-                    stats);                                                                 \
+    const cudaError_t e = est_prepare<GG>();                                                \
+    if (e != cudaSuccess) return e;                                                         \
+    return launch_k(k_estimate<GG>, dim3(grid), dim3(kEstThreads), kEstSmemBytes, st, pdl, \
+                    L, q, Hq, codes, scales, zeros, cand, cand_stride, ncand, lcap, cmax,   \
+                    logits, stats);                                                         \
   }
     TW_EST(1) TW_EST(2) TW_EST(4) TW_EST(8)
 #undef TW_EST

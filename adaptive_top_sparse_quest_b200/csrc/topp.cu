@@ -9,9 +9,10 @@
 // One CTA per selection set (or a thread-block cluster of up to 8 CTAs when a
 // set has more than 8192 candidates).  The set's weights stay in registers, R
 // consecutive candidates per thread:
-//   w = exp(l - m) / Z               (per-head sets)
-//   w = mean_h exp(l_h - m_h) / Z_h  (group sets)
-// with m, Z merged from the estimate kernel's per-32-candidate statistics.
+//   w = 2^(l - m) / Z               (per-head sets)
+//   w = mean_h 2^(l_h - m_h) / Z_h  (group sets)
+// with logits l in log2 units (the estimate kernel folds log2(e) into its
+// scale) and m, Z merged from that kernel's per-32-candidate statistics.
 // The threshold theta is the largest weight value whose retained mass
 // sum_{w >= theta} w reaches p.  Weights lie in [0, 1], so their fp32 bit
 // patterns order like their values and use 30 bits; theta is found most
@@ -26,7 +27,9 @@
 // through distributed shared memory.  Every weight above theta is kept, plus
 // the lowest-position weights equal to theta needed to reach p; the kept token
 // ids are compacted in ascending order by one block scan (and one exchange of
-// per-CTA totals in a cluster).
+// per-CTA totals in a cluster).  Each round costs two block barriers: the
+// replicated histogram is summed, scanned and its digit chosen by one warp
+// while the other warps clear the next round's buffer.
 #include <cooperative_groups.h>
 
 #include "tw_common.cuh"
@@ -79,14 +82,6 @@ __device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* sh, un
   return r;
 }
 
-// Candidate position c of kv unit ukv -> token id, or -1 if not a valid token.
-__device__ __forceinline__ int topp_token(const int32_t* cand, int cand_stride, int64_t ukv,
-                                          int c, int C, int len) {
-  if (c >= C) return -1;
-  int t = c;
-  if (cand) t = cand[ukv * cand_stride + (c >> 4)] * kPage + (c & 15);
-  return (t >= 0 && t < len) ? t : -1;
-}
 
 // NH: heads averaged into one set (1 for per-head sets, G for group sets).
 template <int NH, int R, bool CLUSTER>
@@ -96,9 +91,9 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
        const float* __restrict__ logits, const float2* __restrict__ stats, double p,
        int32_t* __restrict__ idx, int icap, int32_t* __restrict__ count,
        int32_t* __restrict__ done) {
-  __shared__ uint32_t hlo[kHistReps][256], hhi[kHistReps][256];
-  __shared__ unsigned long long hloc[2][256];
-  __shared__ unsigned long long wsuf[8];
+  constexpr int NPG = (R + kPage - 1) / kPage;   // candidate pages a thread's R positions span
+  __shared__ uint32_t hlo[2][kHistReps][256], hhi[2][kHistReps][256];   // double-buffered
+  __shared__ unsigned long long hloc[2][256];                           // per-CTA totals (cluster)
   __shared__ unsigned long long sh_total, sh_above;
   __shared__ int sh_d;
   __shared__ unsigned sh_scan[kToppWarps + 1];
@@ -126,14 +121,38 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
     h0 = (set % Hq) % G;
   }
   const int64_t ukv = (int64_t)b * L.Hk + hk;
-  const int len = L.len(b);
+  const int cbase = cr * (kToppThreads * R) + tid * R;   // this thread's R consecutive candidates
   griddep_wait();
+  // Loads that do not depend on the candidate count go out first: the page ids
+  // of this thread's candidates and their logits (masked by the count below).
+  int pgid[NPG];
+#pragma unroll
+  for (int k = 0; k < NPG; ++k) {
+    const int pgl = (cbase >> 4) + k;
+    pgid[k] = cand ? (pgl < cand_stride ? cand[ukv * cand_stride + pgl] : -1) : pgl;
+  }
+  // small sets of logits are loaded now, into registers; large ones when used
+  constexpr bool kPre = NH * R <= 64;
+  float lv[kPre ? R : 1][kPre ? NH : 1];
+  if (kPre) {
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        lv[kPre ? i : 0][kPre ? h : 0] =
+            (cbase + i < lcap) ? logits[(ukv * lcap + cbase + i) * G + h0 + h] : -INFINITY;
+  }
+  const int len = L.len(b);
   const int C = min(cand ? ncand[ukv] * kPage : len, cmax);
   const int nspans = (C + kStatSpan - 1) / kStatSpan;
-  const int spans_cap = lcap / kStatSpan;
-  const float2* st = stats + ukv * spans_cap * G + h0;
+  const float2* st = stats + ukv * (lcap / kStatSpan) * G + h0;
+  {   // round 0's histogram starts at zero
+    uint32_t* a = &hlo[0][0][0];
+    uint32_t* c = &hhi[0][0][0];
+    for (int i = tid; i < kHistReps * 256; i += kToppThreads) a[i] = c[i] = 0u;
+  }
 
-  // 1. merge the statistics records into each head's max and 1 / sum exp
+  // 1. merge the statistics records into each head's max and 1 / sum 2^(l - max)
   float mloc[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h) mloc[h] = -INFINITY;
@@ -158,8 +177,8 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   for (int t = tid; t < nspans; t += kToppThreads)
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
-      const float2 s = st[(int64_t)t * G + h];
-      if (s.x != -INFINITY) zloc[h] += s.y * expf(s.x - sh_m[h]);
+      const float2 s2 = st[(int64_t)t * G + h];
+      if (s2.x != -INFINITY) zloc[h] += s2.y * exp2f(s2.x - sh_m[h]);
     }
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
@@ -174,21 +193,20 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   }
   __syncthreads();
 
-  // 2. this thread's R consecutive candidates -> weights (-1 marks an invalid slot)
-  const int cbase = cr * (kToppThreads * R) + tid * R;
+  // 2. weights (-1 marks an invalid slot)
   float w[R];
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const int c = cbase + i;
     w[i] = -1.0f;
-    if (c < C) {
+    if (cbase + i < C) {
       float acc = 0.f;
       bool ok = true;
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        const float l = logits[(ukv * lcap + c) * G + h0 + h];
+        const float l = kPre ? lv[kPre ? i : 0][kPre ? h : 0]
+                             : logits[(ukv * lcap + cbase + i) * G + h0 + h];
         ok = ok && (l != -INFINITY);
-        acc += expf(l - sh_m[h]) * sh_iz[h];
+        acc += exp2f(l - sh_m[h]) * sh_iz[h];
       }
       if (ok) w[i] = NH == 1 ? acc : acc * (1.0f / NH);
     }
@@ -202,17 +220,11 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   if (!keep_all) {
     uint32_t prefix = 0, pmask = 0;
     unsigned long long A = 0, T = 0;   // A: mass strictly above the current prefix range
-    uint32_t* hlo_flat = &hlo[0][0];
-    uint32_t* hhi_flat = &hhi[0][0];
     const int rep = lane & (kHistReps - 1);
     for (int round = 0; round < 4; ++round) {
+      const int buf = round & 1;
       const int shift = digit_shift(round);
       const uint32_t dm = digit_mask(round);
-      for (int i = tid; i < kHistReps * 256; i += kToppThreads) {
-        hlo_flat[i] = 0u;
-        hhi_flat[i] = 0u;
-      }
-      __syncthreads();
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         if (w[i] >= 0.f) {
@@ -223,44 +235,83 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
             const unsigned long long F = mass_of(w[i]);
             const uint32_t dg = (key >> shift) & dm;
             const uint32_t lo = (uint32_t)F;
-            const uint32_t old = atomicAdd(&hlo[rep][dg], lo);
+            const uint32_t old = atomicAdd(&hlo[buf][rep][dg], lo);
             const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
-            if (up) atomicAdd(&hhi[rep][dg], up);
+            if (up) atomicAdd(&hhi[buf][rep][dg], up);
           }
         }
       }
+      {   // the other buffer is not read in this round: clear it for the next one
+        uint32_t* a = &hlo[buf ^ 1][0][0];
+        uint32_t* c = &hhi[buf ^ 1][0][0];
+        for (int i = tid; i < kHistReps * 256; i += kToppThreads) a[i] = c[i] = 0u;
+      }
       __syncthreads();
-      unsigned long long v = 0;
-      if (tid < 256) {
+      // warp 0: per-digit mass over the CTA (and cluster), suffix sums, the digit
+      unsigned long long v[8];
+      if (warp == 0) {
 #pragma unroll
-        for (int r = 0; r < kHistReps; ++r)
-          v += ((unsigned long long)hhi[r][tid] << 32) | hlo[r][tid];
+        for (int k = 0; k < 8; ++k) {
+          const int j = 8 * lane + k;
+          unsigned long long x = 0;
+#pragma unroll
+          for (int r = 0; r < kHistReps; ++r)
+            x += ((unsigned long long)hhi[buf][r][j] << 32) | hlo[buf][r][j];
+          v[k] = x;
+          if (CLUSTER) hloc[buf][j] = x;
+        }
       }
       if (CLUSTER) {
         cg::cluster_group cl = cg::this_cluster();
-        if (tid < 256) hloc[round & 1][tid] = v;
         cl.sync();
-        if (tid < 256) {
-          v = 0;
-          for (int r = 0; r < CS; ++r) v += cl.map_shared_rank(&hloc[round & 1][0], r)[tid];
+        if (warp == 0) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            unsigned long long x = 0;
+            for (int r = 0; r < CS; ++r) x += cl.map_shared_rank(&hloc[buf][0], r)[8 * lane + k];
+            v[k] = x;
+          }
         }
       }
-      // suffix sums over the digits: suf[j] = mass of digits >= j
-      unsigned long long suf = v;
-      if (tid < 256) {
+      if (warp == 0) {
+        unsigned long long sl[8];   // suffix within this lane's 8 digits
+        sl[7] = v[7];
+#pragma unroll
+        for (int k = 6; k >= 0; --k) sl[k] = v[k] + sl[k + 1];
+        unsigned long long incl = sl[0];   // suffix over lanes >= this one
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long t = __shfl_down_sync(0xffffffffu, suf, o);
-          if (lane + o < 32) suf += t;
+          const unsigned long long t = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += t;
         }
-        if (lane == 0) wsuf[warp] = suf;
+        const unsigned long long after = incl - sl[0];   // mass of digits above this lane's
+        if (round == 0) {
+          total = __shfl_sync(0xffffffffu, incl, 0);
+          const double tf = ceil((p - kMassEps) * (double)total);
+          T = tf < 1.0 ? 1ull : (unsigned long long)tf;
+          if (T > total) T = total;
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cnt += (A + sl[k] + after >= T) ? 1 : 0;
+        cnt = warp_sum(cnt);
+        const int d = cnt - 1;   // largest digit whose suffix mass reaches T
+        const int dn = d + 1;
+        unsigned long long ab = 0;
+        if (dn < 256 && lane == (dn >> 3)) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k == (dn & 7)) ab = sl[k] + after;
+        }
+        ab = __shfl_sync(0xffffffffu, ab, dn < 256 ? (dn >> 3) : 0);
+        if (lane == 0) {
+          sh_d = d;
+          sh_above = dn < 256 ? ab : 0ull;
+          if (round == 0) sh_total = total;
+        }
       }
       __syncthreads();
-      if (tid < 256)
-        for (int ww = warp + 1; ww < 8; ++ww) suf += wsuf[ww];
       if (round == 0) {
-        if (tid == 0) sh_total = suf;
-        __syncthreads();
         total = sh_total;
         if (total == 0) break;   // no valid candidate (uniform over the cluster)
         const double tf = ceil((p - kMassEps) * (double)total);
@@ -268,15 +319,9 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
         if (T > total) T = total;
         have = true;
       }
-      const int cnt = __syncthreads_count(tid < 256 && A + suf >= T);
-      const int d = cnt - 1;
-      if (tid == d + 1) sh_above = suf;   // mass of digits strictly above d
-      if (tid == 0) sh_d = d;
-      __syncthreads();
-      A += (d == 255) ? 0ull : sh_above;
+      A += sh_above;
       prefix |= (uint32_t)sh_d << shift;
       pmask |= dm << shift;
-      __syncthreads();
     }
     if (have) {
       theta = prefix;
@@ -348,7 +393,10 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
       sel = true;
       ++taken;
     }
-    if (sel) out[pos++] = topp_token(cand, cand_stride, ukv, cbase + i, C, len);
+    if (sel) {
+      const int c = cbase + i;
+      out[pos++] = cand ? pgid[(c >> 4) - (cbase >> 4)] * kPage + (c & 15) : c;
+    }
   }
   if (cr == 0 && tid == 0) {
     count[set] = (int32_t)(gt_all + (unsigned)min(r_need, (unsigned long long)eq_all));
