@@ -59,6 +59,10 @@ int check_kv(const tw_kv* kv, bool need_k, bool need_v, tw::Layout* L) {
         (int64_t)kv->max_seq_len != (int64_t)kv->max_pages_per_seq * tw::kPage)
       return TW_ERR_INVALID_ARG;
   }
+  // physical rows are 32-bit indices (row lists between the kernels)
+  const int64_t nrows = kv->page_table ? (int64_t)kv->num_pool_pages * kv->num_kv_heads * tw::kPage
+                                       : (int64_t)kv->batch * kv->num_kv_heads * kv->max_seq_len;
+  if (nrows >= (int64_t)tw::kNoRow) return TW_ERR_UNSUPPORTED;
   L->B = kv->batch;
   L->Hk = kv->num_kv_heads;
   L->N = kv->max_seq_len;
@@ -76,11 +80,12 @@ int check_heads(int Hq, int Hk) {
   return TW_OK;
 }
 
-// Workspace regions, in order: status word | page scores | logits | softmax
-// statistics | per-set completion counters | attention partial records.  The
+// Workspace regions, in order: status word | page scores | first physical row
+// of each candidate page | logits | softmax statistics | physical rows of the
+// kept tokens | per-set completion counters | attention partial records.  The
 // status word collects device-side error bits (a bounded wait that gave up).
 struct Plan {
-  size_t status_off, scores_off, logits_off, stats_off, done_off, part_off;
+  size_t status_off, scores_off, row0_off, logits_off, stats_off, rows_off, done_off, part_off;
   size_t scores_end, topp_end, total;
   int lcap;
 };
@@ -93,12 +98,14 @@ Plan make_plan(int B, int Hq, int Hk, int N, int cap) {
   p.status_off = 0;
   p.scores_off = 256;
   p.scores_end = p.scores_off + align256((size_t)B * Hk * pmax * sizeof(float));
-  p.logits_off = p.scores_end;
+  p.row0_off = p.scores_end;
+  p.logits_off = p.row0_off + align256((size_t)B * Hk * pmax * sizeof(uint32_t));
   p.stats_off = p.logits_off + align256((size_t)B * Hk * p.lcap * G * sizeof(float));
   p.topp_end = p.stats_off +
                align256((size_t)B * Hk * (p.lcap / tw::kStatSpan) * G * sizeof(float2));
-  p.done_off = p.topp_end;
   const size_t nsets = (size_t)B * (Hq > Hk ? Hq : Hk);
+  p.rows_off = p.topp_end;
+  p.done_off = p.rows_off + align256(nsets * (size_t)cap * sizeof(uint32_t));
   p.part_off = p.done_off + align256(nsets * sizeof(int32_t));
   p.total = p.part_off + align256(tw::decode_part_floats(B, Hq, Hk) * sizeof(float));
   return p;
@@ -220,12 +227,17 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   cudaError_t e;
   if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   float* scores = reinterpret_cast<float*>(wsp(s->ws, plan.scores_off));
+  // physical rows: the selector writes the candidate pages' first rows, the
+  // top-p kernel the kept tokens' rows (without selection the estimate and
+  // top-p kernels compute page rows themselves)
+  uint32_t* row0 = use_select ? reinterpret_cast<uint32_t*>(wsp(s->ws, plan.row0_off)) : nullptr;
+  uint32_t* rows = reinterpret_cast<uint32_t*>(wsp(s->ws, plan.rows_off));
   if (use_select) {
     e = tw::launch_page_scores(L, q, Hq, reinterpret_cast<const __half*>(s->meta), scores, st,
                                sms, pdl);
     if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
     e = tw::launch_page_topk(L, scores, s->budget_tokens / tw::kPage, s->cand_pages,
-                             s->cand_stride, s->ncand, st, pdl);
+                             s->cand_stride, s->ncand, row0, st, pdl);
     if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   }
   float* logits = reinterpret_cast<float*>(wsp(s->ws, plan.logits_off));
@@ -233,17 +245,17 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   const int cmax = candidates_max(L, cand, s->cand_stride);
   e = tw::launch_estimate(L, q, Hq, s->codes, reinterpret_cast<const __half*>(s->scales),
                           reinterpret_cast<const __half*>(s->zeros), cand, s->cand_stride,
-                          s->ncand, plan.lcap, cmax, logits, stats, st, sms, pdl);
+                          s->ncand, row0, plan.lcap, cmax, logits, stats, st, sms, pdl);
   if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   int32_t* done = reinterpret_cast<int32_t*>(wsp(s->ws, plan.done_off));
-  e = tw::launch_topp(L, Hq, gs, cand, s->cand_stride, s->ncand, plan.lcap, cmax, logits, stats,
-                      s->p, s->idx, s->capacity, s->count, done, st, pdl);
+  e = tw::launch_topp(L, Hq, gs, cand, s->cand_stride, s->ncand, row0, plan.lcap, cmax, logits,
+                      stats, s->p, s->idx, rows, s->capacity, s->count, done, st, pdl);
   if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   float* part = reinterpret_cast<float*>(wsp(s->ws, plan.part_off));
   const auto* K = reinterpret_cast<const __half*>(s->kv.k);
   const auto* V = reinterpret_cast<const __half*>(s->kv.v);
   auto* out = reinterpret_cast<__half*>(s->out);
-  e = tw::launch_sparse_decode(L, q, Hq, gs, K, V, s->idx, s->capacity, s->count, part, done, out,
+  e = tw::launch_sparse_decode(L, q, Hq, gs, K, V, rows, s->capacity, s->count, part, done, out,
                                s->lse, st, pdl);
   if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   return check_launch();
@@ -325,7 +337,7 @@ int tw_select_pages(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
                                          false);
   if (e == cudaSuccess)
     e = tw::launch_page_topk(L, scores, budget_tokens / tw::kPage, cand_pages, cand_stride,
-                             ncand, st, false);
+                             ncand, nullptr, st, false);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
@@ -348,15 +360,19 @@ int tw_topp_prune(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   float* logits = reinterpret_cast<float*>(wsp(ws, plan.logits_off));
   float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.stats_off));
   const int cmax = candidates_max(L, cand_pages, cand_stride);
-  cudaError_t e = tw::launch_estimate(L, reinterpret_cast<const __half*>(q), num_q_heads, codes,
-                                      reinterpret_cast<const __half*>(scales),
-                                      reinterpret_cast<const __half*>(zeros), cand_pages,
-                                      cand_stride, ncand, plan.lcap, cmax, logits, stats, st, sms,
-                                      false);
+  // caller-given candidate pages: locate their rows first
+  uint32_t* row0 = cand_pages ? reinterpret_cast<uint32_t*>(wsp(ws, plan.row0_off)) : nullptr;
+  cudaError_t e = cudaSuccess;
+  if (cand_pages) e = tw::launch_resolve_pages(L, cand_pages, cand_stride, row0, st, false);
+  if (e == cudaSuccess)
+    e = tw::launch_estimate(L, reinterpret_cast<const __half*>(q), num_q_heads, codes,
+                            reinterpret_cast<const __half*>(scales),
+                            reinterpret_cast<const __half*>(zeros), cand_pages, cand_stride,
+                            ncand, row0, plan.lcap, cmax, logits, stats, st, sms, false);
   if (e == cudaSuccess)
     e = tw::launch_topp(L, num_q_heads, group_sets_of(num_q_heads, L.Hk, group_mode), cand_pages,
-                        cand_stride, ncand, plan.lcap, cmax, logits, stats, p, idx, capacity,
-                        count, nullptr, st, false);
+                        cand_stride, ncand, row0, plan.lcap, cmax, logits, stats, p, idx,
+                        nullptr, capacity, count, nullptr, st, false);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
@@ -379,11 +395,14 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   const int nsets = gs ? L.B * L.Hk : L.B * num_q_heads;
   const auto* K = reinterpret_cast<const __half*>(kv->k);
   const auto* V = reinterpret_cast<const __half*>(kv->v);
+  uint32_t* rows = reinterpret_cast<uint32_t*>(wsp(ws, plan.rows_off));
   cudaError_t e = cudaMemsetAsync(done, 0, (size_t)nsets * sizeof(int32_t), st);
+  if (e == cudaSuccess)   // caller-given token ids: map them to physical rows first
+    e = tw::launch_resolve_rows(L, num_q_heads, gs, idx, capacity, count, rows, st, false);
   if (e == cudaSuccess)
-    e = tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V, idx,
-                                 capacity, count, part, done, reinterpret_cast<__half*>(out), lse,
-                                 st, false);
+    e = tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V,
+                                 rows, capacity, count, part, done,
+                                 reinterpret_cast<__half*>(out), lse, st, false);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }

@@ -16,7 +16,10 @@
 // (c + set), unique because (c, set) pairs advance monotonically along the
 // list.
 //
-// Data path.  The set's token ids for a window of the range are staged in
+// Data path.  The kept tokens arrive as physical K/V row indices (the top-p
+// kernel, or a resolve kernel for caller-given ids, maps ids through the page
+// table; kNoRow marks an id outside the sequence), so no page-table load sits
+// in front of a gather.  The rows of a window of the range are staged in
 // shared memory once; the gathered 256-byte K and V rows then stream through a
 // 4-stage cp.async ring of 16 tokens per stage (32 KB in flight per CTA), so
 // a CTA pays one dependent round trip per window instead of one per batch.
@@ -39,7 +42,7 @@ constexpr int kDecThreads = 128;
 constexpr int kDecHW = kDecThreads / 16;       // half-warps
 constexpr int kStageTok = 16;                  // tokens per pipeline stage
 constexpr int kStages = 4;
-constexpr int kWin = 512;                      // token ids staged per window
+constexpr int kWin = 512;                      // token rows staged per window
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void h8_to_f8(uint4 r, float* f) {
@@ -81,9 +84,19 @@ __device__ __forceinline__ bool range_has(int64_t c, int64_t S, int n, int64_t o
   return lo < hi && lo < off + cnt && hi > off;
 }
 
+// Merge layout: 32 lanes with a float4 each cover one head's 128 channels.
+// With fewer than 4 heads the warps also split the records (kMergeRS ways);
+// with 8 heads each thread carries two heads.
+template <int NH>
+struct MergeShape {
+  static constexpr int RS = NH >= 4 ? 1 : 4 / NH;    // record split
+  static constexpr int HPT = NH > 4 ? NH / 4 : 1;    // heads per thread
+  static constexpr int U = NH >= 4 ? 8 / HPT : 16;   // records per batch of loads
+};
+
 template <int NH>
 struct DecSmem {
-  int ids[kWin];
+  uint32_t rows[kWin];
   union {
     __half kv[kStages][kStageTok][2][kHeadDim];                 // K row, V row
     struct {
@@ -91,8 +104,9 @@ struct DecSmem {
       float acc[kDecHW][NH][kHeadDim];
     } comb;
     struct {
-      float f[kDecThreads];
-      float red[kDecThreads / 32];
+      float f[NH][kDecThreads];                                 // weights of a chunk of records
+      float red[kDecThreads / 32][NH];
+      float4 acc[MergeShape<NH>::RS][NH][kHeadDim / 4];         // per-split partial sums
     } merge;
   } u;
   int64_t red64[kDecThreads / 32];
@@ -103,74 +117,149 @@ struct DecSmem {
   int last;
 };
 
-// Fold the records of `set` into out / lse (called by the CTA that completes it).
+// Fold the records of `set` into out / lse (called by the CTA that completes
+// it).  All heads are folded together; the records were written by other CTAs
+// of this launch, so they are read through L2 only (ld.global.cg).
 template <int NH>
 __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_t S, int n_ctas,
                           int Hq, int hq0, int b, const float* part, __half* out, float* lse) {
-  const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  using MS = MergeShape<NH>;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t c0 = ((off + 1) * n_ctas + S - 1) / S - 1;
   const int64_t c1 = ((off + cnt) * n_ctas + S - 1) / S - 1;
   const int nrec = (int)(c1 - c0 + 1);
-  for (int h = 0; h < NH; ++h) {
-    float mx = -INFINITY;
-    for (int r = d; r < nrec; r += kDecThreads)
-      if (range_has(c0 + r, S, n_ctas, off, cnt))
-        mx = fmaxf(mx, part[((c0 + r + set) * NH + h) * kPartStride]);
-    mx = warp_max(mx);
-    __syncthreads();
-    if (lane == 0) sm.u.merge.red[warp] = mx;
-    __syncthreads();
-    float M = sm.u.merge.red[0];
+  auto rec_ptr = [&](int r, int h) { return part + ((c0 + r + set) * NH + h) * kPartStride; };
+  // 1. per-head max over the records; the first chunk's (m, l) stay in registers
+  float m0[NH], l0[NH], mx[NH];
+  const bool v0 = t < nrec && range_has(c0 + t, S, n_ctas, off, cnt);
 #pragma unroll
-    for (int i = 1; i < kDecThreads / 32; ++i) M = fmaxf(M, sm.u.merge.red[i]);
-    float Ls = 0.f, A = 0.f;
-    for (int r0 = 0; r0 < nrec; r0 += kDecThreads) {
-      const int r = r0 + d;
-      float f = 0.f;
-      if (r < nrec && range_has(c0 + r, S, n_ctas, off, cnt)) {
-        const float* rec = part + ((c0 + r + set) * NH + h) * kPartStride;
-        if (rec[0] != -INFINITY) {
-          f = exp2f(rec[0] - M);
-          Ls += rec[1] * f;
+  for (int h = 0; h < NH; ++h) {
+    const float2 ml = v0 ? __ldcg(reinterpret_cast<const float2*>(rec_ptr(t, h)))
+                         : make_float2(-INFINITY, 0.f);
+    m0[h] = ml.x;
+    l0[h] = ml.y;
+    mx[h] = ml.x;
+  }
+  for (int r = t + kDecThreads; r < nrec; r += kDecThreads)
+    if (range_has(c0 + r, S, n_ctas, off, cnt))
+#pragma unroll
+      for (int h = 0; h < NH; ++h) mx[h] = fmaxf(mx[h], __ldcg(rec_ptr(r, h)));
+  __syncthreads();   // the shared union was used by the caller
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const float v = warp_max(mx[h]);
+    if (lane == 0) sm.u.merge.red[warp][h] = v;
+  }
+  __syncthreads();
+  float M[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    M[h] = sm.u.merge.red[0][h];
+#pragma unroll
+    for (int w = 1; w < kDecThreads / 32; ++w) M[h] = fmaxf(M[h], sm.u.merge.red[w][h]);
+  }
+  // 2. chunks of 128 records: weights 2^(m_r - M), then the weighted rows
+  const int rs = warp / (NH >= 4 ? 4 : NH) % MS::RS;    // this warp's record split
+  const int hbase = NH >= 4 ? warp : warp % NH;          // first head of this thread
+  float Lp[NH];
+  float4 A[MS::HPT];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) Lp[h] = 0.f;
+#pragma unroll
+  for (int k = 0; k < MS::HPT; ++k) A[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r0 = 0; r0 < nrec; r0 += kDecThreads) {
+    const int r = r0 + t;
+    bool vr = v0;
+    float mr[NH], lr[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      mr[h] = m0[h];
+      lr[h] = l0[h];
+    }
+    if (r0 > 0) {
+      vr = r < nrec && range_has(c0 + r, S, n_ctas, off, cnt);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const float2 ml = vr ? __ldcg(reinterpret_cast<const float2*>(rec_ptr(r, h)))
+                             : make_float2(-INFINITY, 0.f);
+        mr[h] = ml.x;
+        lr[h] = ml.y;
+      }
+      __syncthreads();   // the previous chunk's weights are no longer read
+    }
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const float f = (vr && mr[h] != -INFINITY) ? exp2f(mr[h] - M[h]) : 0.f;
+      Lp[h] += lr[h] * f;
+      sm.u.merge.f[h][t] = f;
+    }
+    __syncthreads();
+    const int nr = min(kDecThreads, nrec - r0);
+    for (int i0 = rs; i0 < nr; i0 += MS::RS * MS::U) {
+      float fv[MS::U][MS::HPT];
+      float4 x[MS::U][MS::HPT];
+#pragma unroll
+      for (int u = 0; u < MS::U; ++u) {
+        const int i = i0 + u * MS::RS;
+#pragma unroll
+        for (int k = 0; k < MS::HPT; ++k) {
+          const int h = hbase + 4 * k;
+          fv[u][k] = i < nr ? sm.u.merge.f[h][i] : 0.f;
+          x[u][k] = fv[u][k] != 0.f
+                        ? __ldcg(reinterpret_cast<const float4*>(rec_ptr(r0 + i, h) + kPartAcc) + lane)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      __syncthreads();
-      sm.u.merge.f[d] = f;
-      __syncthreads();
-      const int nr = min(kDecThreads, nrec - r0);
-      int i = 0;
-      for (; i + 8 <= nr; i += 8) {
-        float a8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          a8[j] = sm.u.merge.f[i + j] != 0.f
-                      ? part[((c0 + r0 + i + j + set) * NH + h) * kPartStride + kPartAcc + d]
-                      : 0.f;
+      for (int u = 0; u < MS::U; ++u)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) A += a8[j] * sm.u.merge.f[i + j];
-      }
-      for (; i < nr; ++i)
-        if (sm.u.merge.f[i] != 0.f)
-          A += part[((c0 + r0 + i + set) * NH + h) * kPartStride + kPartAcc + d] * sm.u.merge.f[i];
+        for (int k = 0; k < MS::HPT; ++k) {
+          A[k].x = __fmaf_rn(fv[u][k], x[u][k].x, A[k].x);
+          A[k].y = __fmaf_rn(fv[u][k], x[u][k].y, A[k].y);
+          A[k].z = __fmaf_rn(fv[u][k], x[u][k].z, A[k].z);
+          A[k].w = __fmaf_rn(fv[u][k], x[u][k].w, A[k].w);
+        }
     }
-    Ls = warp_sum(Ls);
-    __syncthreads();
-    if (lane == 0) sm.u.merge.red[warp] = Ls;
-    __syncthreads();
-    Ls = 0.f;
+  }
+  // 3. totals: sum of l-weights per head, the record splits' partial rows
 #pragma unroll
-    for (int i = 0; i < kDecThreads / 32; ++i) Ls += sm.u.merge.red[i];
-    const int64_t bh = (int64_t)b * Hq + hq0 + h;
-    out[bh * kHeadDim + d] = __float2half_rn(Ls > 0.f ? A / Ls : 0.f);
-    if (lse && d == 0) lse[bh] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+  for (int h = 0; h < NH; ++h) {
+    const float v = warp_sum(Lp[h]);
+    if (lane == 0) sm.u.merge.red[warp][h] = v;
+  }
+#pragma unroll
+  for (int k = 0; k < MS::HPT; ++k) sm.u.merge.acc[rs][hbase + 4 * k][lane] = A[k];
+  __syncthreads();
+  if (rs == 0) {
+#pragma unroll
+    for (int k = 0; k < MS::HPT; ++k) {
+      const int h = hbase + 4 * k;
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecThreads / 32; ++w) Ls += sm.u.merge.red[w][h];
+      float4 a = sm.u.merge.acc[0][h][lane];
+#pragma unroll
+      for (int s2 = 1; s2 < MS::RS; ++s2) {
+        const float4 e = sm.u.merge.acc[s2][h][lane];
+        a.x += e.x;
+        a.y += e.y;
+        a.z += e.z;
+        a.w += e.w;
+      }
+      const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+      const int64_t bh = (int64_t)b * Hq + hq0 + h;
+      __half2 o2[2] = {__floats2half2_rn(a.x * inv, a.y * inv), __floats2half2_rn(a.z * inv, a.w * inv)};
+      *reinterpret_cast<uint2*>(out + bh * kHeadDim + 4 * lane) = *reinterpret_cast<uint2*>(o2);
+      if (lse && lane == 0) lse[bh] = Ls > 0.f ? (M[h] + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+    }
   }
 }
 
 template <int NH>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, NH >= 8 ? 2 : 4)   // 4 CTAs per SM: kDecCtas in one wave
 k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group_sets,
                 const __half* __restrict__ K, const __half* __restrict__ V,
-                const int32_t* __restrict__ idx, int icap, const int32_t* __restrict__ count,
+                const uint32_t* __restrict__ rows, int icap, const int32_t* __restrict__ count,
                 int nsets, float* __restrict__ part, int32_t* __restrict__ done,
                 __half* __restrict__ out, float* __restrict__ lse) {
   __shared__ __align__(16) DecSmem<NH> sm;
@@ -257,7 +346,6 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
       const int64_t lo = max(begin, soff), hi = min(end, soff + scnt);
       int b, hk, hq0;
       set_heads(set, b, hk, hq0);
-      const int len = L.len(b);
       float qf[NH][8];
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
@@ -274,13 +362,12 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
       }
-      const int32_t* ids = idx + (int64_t)set * icap;
+      const uint32_t* srows = rows + (int64_t)set * icap;
       for (int64_t w0 = lo; w0 < hi; w0 += kWin) {
         const int wn = (int)min((int64_t)kWin, hi - w0);
-        __syncthreads();   // previous window's ids and ring are no longer read
+        __syncthreads();   // previous window's rows and ring are no longer read
         for (int i = tid; i < wn; i += kDecThreads) {
-          const int tk = ids[w0 - soff + i];
-          sm.ids[i] = (unsigned)tk < (unsigned)len ? tk : -1;   // ids outside [0, len) are ignored
+          sm.rows[i] = srows[w0 - soff + i];
         }
         __syncthreads();
         const int nst = (wn + kStageTok - 1) / kStageTok;
@@ -291,9 +378,9 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
             for (int x = tid; x < kStageTok * 32; x += kDecThreads) {
               const int j = x >> 5, part_ = x & 31;
               const int pos = st * kStageTok + j;
-              const int tk = pos < wn ? sm.ids[pos] : -1;
-              if (tk >= 0) {
-                const int64_t row = L.row(b, hk, tk);
+              const uint32_t r = pos < wn ? sm.rows[pos] : kNoRow;
+              if (r != kNoRow) {
+                const int64_t row = r;
                 const __half* src = (part_ < 16 ? K : V) + row * kHeadDim + (part_ & 15) * 8;
                 cp_async16(&sm.u.kv[slot][j][part_ >> 4][(part_ & 15) * 8], src);
               }
@@ -314,7 +401,7 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
           for (int jj = 0; jj < 2; ++jj) {
             const int j = 2 * hw + jj;
             const int pos = st * kStageTok + j;
-            ok[jj] = pos < wn && sm.ids[pos] >= 0;
+            ok[jj] = pos < wn && sm.rows[pos] != kNoRow;
             float kf[8];
             h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][j][0][8 * l16])
                             : make_uint4(0u, 0u, 0u, 0u),
@@ -428,7 +515,7 @@ size_t decode_part_floats(int B, int Hq, int Hk) {
 }
 
 cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
-                                 const __half* K, const __half* V, const int32_t* idx, int icap,
+                                 const __half* K, const __half* V, const uint32_t* rows, int icap,
                                  const int32_t* count, float* part, int32_t* done, __half* out,
                                  float* lse, cudaStream_t st, bool pdl) {
   const int G = Hq / L.Hk;
@@ -438,7 +525,7 @@ cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int g
 #define TW_DEC(NN)                                                                           \
   case NN:                                                                                   \
     return launch_k(k_sparse_decode<NN>, dim3(kDecCtas), dim3(kDecThreads), 0, st, pdl, L, q, \
-                    Hq, G, group_sets, K, V, idx, icap, count, nsets, part, done, out, lse);
+                    Hq, G, group_sets, K, V, rows, icap, count, nsets, part, done, out, lse);
     TW_DEC(1) TW_DEC(2) TW_DEC(4) TW_DEC(8)
 #undef TW_DEC
   }

@@ -25,9 +25,11 @@
 // work items (kv unit, 16 candidate pages = 256 candidates: 16 KB of codes +
 // 2 KB of scales + 2 KB of zeros).  A 4-stage shared-memory ring is filled
 // with cp.async by all threads (16-byte chunks of codes, 8-byte rows of
-// scales and zeros) three items ahead, and warp 0 looks up the page ids of the
-// item after that, so the id lookups and the row gathers both stay off the
-// critical path.  Each of the eight warps then takes 32 candidates (two MMA
+// scales and zeros) three items ahead.  A page's rows are located from the
+// candidate list and a list of first physical rows written by the selector
+// (no page-table walk here); warp 0 issues those lookups two items before
+// their gathers and stores them one iteration later, so neither the lookups
+// nor the gathers sit on the critical path.  Each of the eight warps then takes 32 candidates (two MMA
 // tiles) and writes the fp32 logits [unit][cap][G] plus its per-head
 // (max, sum 2^(l - max)).
 #include "tw_common.cuh"
@@ -55,7 +57,7 @@ struct EstPages {
 
 struct EstSmem {
   EstStage st[kEstStages];
-  EstPages pg[kEstStages + 1];
+  EstPages pg[kEstStages + 2];   // items j .. j+S+1 around iteration j
 };
 
 constexpr size_t kEstSmemBytes = sizeof(EstSmem);
@@ -101,28 +103,40 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-// Page lookup of item `it` (lanes 0..15 of one warp): global first row and
-// valid rows of each of its 16 candidate pages.
-__device__ __forceinline__ void est_pages(const Layout& L, const int32_t* cand, int cand_stride,
-                                          const int32_t* ncand, int cmax, int tiles, int it,
-                                          int lane, EstPages& out) {
-  if (lane >= kPagesPerItem) return;
+// Page lookup of one candidate page of item `it`: its page id, the first
+// physical row of the page (from the row list the selector or the resolve
+// kernel wrote), the unit's candidate count and sequence length.  The loads
+// are independent; est_fetch only issues them, est_store consumes them.
+struct EstLook {
+  int page, C, len;
+  uint32_t r0;
+};
+
+__device__ __forceinline__ EstLook est_fetch(const Layout& L, const int32_t* cand, int cand_stride,
+                                             const int32_t* ncand, const uint32_t* row0,
+                                             int cmax, int tiles, int it, int lane) {
+  EstLook k;
   const int u = it / tiles;
-  const int b = u / L.Hk, hk = u % L.Hk;
-  const int len = L.len(b);
-  const int C = min(cand ? ncand[u] * kPage : len, cmax);
+  const int b = u / L.Hk;
   const int lp = (it % tiles) * kPagesPerItem + lane;   // logical candidate page
+  k.len = L.len(b);
+  k.C = cand ? ncand[u] * kPage : k.len;
+  k.C = min(k.C, cmax);
+  k.page = cand ? (lp < cand_stride ? cand[(int64_t)u * cand_stride + lp] : -1) : lp;
+  // without a candidate list (every page a candidate) the row is computed here
+  k.r0 = lp >= L.max_pages ? 0u
+         : row0            ? row0[(int64_t)u * L.max_pages + lp]
+                           : (uint32_t)L.page_row(b, u % L.Hk, lp);
+  k.C = lp * kPage < k.C ? k.C : 0;   // this page is a candidate only if lp * 16 < C
+  return k;
+}
+
+__device__ __forceinline__ void est_store(const EstLook& k, int lane, EstPages& out) {
   int rows = 0;
-  long long row0 = 0;
-  if (lp * kPage < C) {
-    const int page = cand ? (lp < cand_stride ? cand[(int64_t)u * cand_stride + lp] : -1) : lp;
-    if (page >= 0 && page < L.max_pages) {
-      rows = max(0, min(kPage, len - page * kPage));
-      if (rows > 0) row0 = L.page_row(b, hk, page);
-    }
-  }
+  if (k.C > 0 && k.page >= 0 && (int64_t)k.page * kPage < k.len)
+    rows = min(kPage, k.len - k.page * kPage);
   out.rows[lane] = rows;
-  out.row0[lane] = row0;
+  out.row0[lane] = rows > 0 ? (long long)k.r0 : 0ll;
 }
 
 // All threads: gather item `it` (pages already looked up) into a ring stage.
@@ -151,7 +165,8 @@ __global__ void __launch_bounds__(kEstThreads, 2)
 k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __restrict__ codes,
            const __half* __restrict__ scales, const __half* __restrict__ zeros,
            const int32_t* __restrict__ cand, int cand_stride, const int32_t* __restrict__ ncand,
-           int lcap, int cmax, float* __restrict__ logits, float2* __restrict__ stats) {
+           const uint32_t* __restrict__ row0, int lcap, int cmax, float* __restrict__ logits,
+           float2* __restrict__ stats) {
   constexpr int HP = (G + 1) / 2;   // head pairs: one MMA N-block of 8 (head, group) columns each
   extern __shared__ __align__(128) unsigned char est_smem_raw[];
   EstSmem& sm = *reinterpret_cast<EstSmem*>(est_smem_raw);
@@ -163,10 +178,19 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
   if (it0 >= it1) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   griddep_wait();
-  // pipeline prologue: page lookups for items it0 .. it0+S-1, then their gathers
-  if (warp == 0)
-    for (int j = 0; j < kEstStages && it0 + j < it1; ++j)
-      est_pages(L, cand, cand_stride, ncand, cmax, tiles, it0 + j, lane, sm.pg[j]);
+  // pipeline prologue: page lookups of items it0 .. it0+S by all threads at
+  // once, the lookups of item it0+S+1 left in flight in warp 0's registers,
+  // then the gathers of items it0 .. it0+S-2
+  constexpr int kPgRing = kEstStages + 2;
+  if (tid < (kEstStages + 1) * kPagesPerItem) {
+    const int j = tid / kPagesPerItem, lp = tid % kPagesPerItem;
+    if (it0 + j < it1)
+      est_store(est_fetch(L, cand, cand_stride, ncand, row0, cmax, tiles, it0 + j, lp), lp,
+                sm.pg[j]);
+  }
+  EstLook ahead = {};
+  if (warp == 0 && lane < kPagesPerItem && it0 + kEstStages + 1 < it1)
+    ahead = est_fetch(L, cand, cand_stride, ncand, row0, cmax, tiles, it0 + kEstStages + 1, lane);
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < kEstStages - 1; ++j) {
@@ -185,12 +209,17 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
     // pages of item j+S (their ring entries were last read one iteration ago)
     __syncthreads();
     if (it + kEstStages - 1 < it1)
-      est_issue(sm.pg[(j + kEstStages - 1) % (kEstStages + 1)], codes, scales, zeros,
+      est_issue(sm.pg[(j + kEstStages - 1) % kPgRing], codes, scales, zeros,
                 sm.st[(j + kEstStages - 1) % kEstStages]);
     cp_async_commit();
-    if (warp == 0 && it + kEstStages < it1)
-      est_pages(L, cand, cand_stride, ncand, cmax, tiles, it + kEstStages, lane,
-                sm.pg[(j + kEstStages) % (kEstStages + 1)]);
+    // warp 0: store the lookups of item j+S+1 (issued one iteration ago) into
+    // the slot item j-1 used, and issue those of item j+S+2
+    if (warp == 0 && lane < kPagesPerItem) {
+      if (it + kEstStages + 1 < it1) est_store(ahead, lane, sm.pg[(j + kEstStages + 1) % kPgRing]);
+      if (it + kEstStages + 2 < it1)
+        ahead = est_fetch(L, cand, cand_stride, ncand, row0, cmax, tiles, it + kEstStages + 2,
+                          lane);
+    }
     const int u = it / tiles;
     const int b = u / L.Hk, hk = u % L.Hk;
     if (u != staged) {
@@ -220,7 +249,7 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
     }
     cp_async_wait<kEstStages - 1>();
     __syncthreads();
-    const EstPages& pgs = sm.pg[j % (kEstStages + 1)];
+    const EstPages& pgs = sm.pg[j % kPgRing];
     const EstStage& st = sm.st[slot];
     const int cw0 = (it % tiles) * kEstTile + warp * 32;   // this warp's first candidate
     const int Cu = min(cand ? __ldg(ncand + u) * kPage : L.len(b), cmax);
@@ -321,9 +350,9 @@ static cudaError_t est_prepare() {
 
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
                             const __half* scales, const __half* zeros, const int32_t* cand,
-                            int cand_stride, const int32_t* ncand, int lcap, int cmax,
-                            float* logits, float2* stats, cudaStream_t st, int num_sms,
-                            bool pdl) {
+                            int cand_stride, const int32_t* ncand, const uint32_t* row0,
+                            int lcap, int cmax, float* logits, float2* stats, cudaStream_t st,
+                            int num_sms, bool pdl) {
   const int G = Hq / L.Hk;
   const int items = L.B * L.Hk * (lcap / kEstTile);
   const int grid = items < 2 * num_sms ? items : 2 * num_sms;
@@ -333,8 +362,8 @@ cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint
     const cudaError_t e = est_prepare<GG>();                                                \
     if (e != cudaSuccess) return e;                                                         \
     return launch_k(k_estimate<GG>, dim3(grid), dim3(kEstThreads), kEstSmemBytes, st, pdl, \
-                    L, q, Hq, codes, scales, zeros, cand, cand_stride, ncand, lcap, cmax,   \
-                    logits, stats);                                                         \
+                    L, q, Hq, codes, scales, zeros, cand, cand_stride, ncand, row0, lcap,   \
+                    cmax, logits, stats);                                                   \
   }
     TW_EST(1) TW_EST(2) TW_EST(4) TW_EST(8)
 #undef TW_EST

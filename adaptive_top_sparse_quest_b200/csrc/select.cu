@@ -18,8 +18,10 @@
 // k_page_scores is persistent: each CTA owns a contiguous block of
 // (kv unit, 64-page chunk) items and loads item i+1's metadata while scoring
 // item i.  k_page_topk keeps each unit's K_p best pages by a most-significant-
-// digit-first radix select on the ordered score keys (histograms replicated 8
-// ways against same-address contention), then compacts them in page order.
+// digit-first radix select on the ordered score keys (12 bits, then 9 at a
+// time, starting below the bits all of the unit's keys share), then compacts
+// them in page order with one block scan; in the fused decode step it also
+// writes each kept page's first physical row.
 #include "tw_common.cuh"
 #include "tw_kernels.h"
 
@@ -125,134 +127,224 @@ k_page_scores(Layout L, const __half* __restrict__ q, int Hq, const __half* __re
 }
 
 // ---------------------------------------------------------------------------
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkCached = 8;   // keys per thread kept in registers (8192 pages)
-constexpr int kTopkReps = 8;
+constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkCached = 16;  // keys per thread kept in registers (8192 pages)
+constexpr int kTopkBins = 4096;  // first digit: 12 bits (8 per thread), then 9 (1 per thread)
 
-// Exclusive prefix count of a 0/1 flag over the block in thread order; returns
-// the flag's rank and writes the block total to *total.  Uses sh[0..32].
-__device__ __forceinline__ int block_rank(bool flag, int* sh, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, flag);
-  const int in_warp = __popc(bal & ((1u << lane) - 1u));
-  if (lane == 0) sh[warp] = __popc(bal);
+// Inclusive scan over the block, in thread order, of a pair of counts; returns
+// the exclusive prefix and writes the block totals.  Uses sh[0..kTopkWarps].
+__device__ __forceinline__ int2 block_excl_scan2(int2 v, int2* sh, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int2 incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int tx = __shfl_up_sync(0xffffffffu, incl.x, o);
+    const int ty = __shfl_up_sync(0xffffffffu, incl.y, o);
+    if (lane >= o) {
+      incl.x += tx;
+      incl.y += ty;
+    }
+  }
+  if (lane == 31) sh[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int v = lane < nw ? sh[lane] : 0;
-    int incl = v;
+    const int2 x = lane < kTopkWarps ? sh[lane] : make_int2(0, 0);
+    int2 xi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+      const int tx = __shfl_up_sync(0xffffffffu, xi.x, o);
+      const int ty = __shfl_up_sync(0xffffffffu, xi.y, o);
+      if (lane >= o) {
+        xi.x += tx;
+        xi.y += ty;
+      }
     }
-    if (lane < nw) sh[lane] = incl - v;
-    if (lane == 31) sh[32] = incl;
+    if (lane < kTopkWarps) sh[lane] = make_int2(xi.x - x.x, xi.y - x.y);
+    if (lane == 31) sh[kTopkWarps] = xi;
   }
   __syncthreads();
-  const int r = sh[warp] + in_warp;
-  *total = sh[32];
-  __syncthreads();
+  const int2 r = make_int2(sh[warp].x + incl.x - v.x, sh[warp].y + incl.y - v.y);
+  *total = sh[kTopkWarps];
   return r;
 }
 
 // One block per (b, kv head): the K_p largest page scores, ties to the lower
-// page index, written in ascending page order.
-__global__ void __launch_bounds__(kTopkThreads)
+// page index, written in ascending page order (and, when row0 is given, each
+// kept page's first physical row).  Thread t owns the E consecutive pages
+// [t E, t E + E); the first kTopkCached keys stay in registers, later ones are
+// re-read from the score buffer.
+__global__ void __launch_bounds__(kTopkThreads, 2)
 k_page_topk(Layout L, const float* __restrict__ scores, int budget_pages,
-            int32_t* __restrict__ cand, int cand_stride, int32_t* __restrict__ ncand) {
-  __shared__ int hrep[kTopkReps][256];
-  __shared__ int wsum[8];
-  __shared__ int sh_scan[33];
+            int32_t* __restrict__ cand, int cand_stride, int32_t* __restrict__ ncand,
+            uint32_t* __restrict__ row0) {
+  __shared__ __align__(16) int hist[kTopkBins];
+  __shared__ int wsuf[kTopkWarps];
+  __shared__ uint32_t wmin[kTopkWarps], wmax[kTopkWarps];
+  __shared__ int2 sh_scan[kTopkWarps + 1];
   __shared__ int sh_d, sh_above;
   const int u = blockIdx.x;
-  const int b = u / L.Hk;
+  const int b = u / L.Hk, hk = u % L.Hk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  reinterpret_cast<int4*>(hist)[2 * tid] = make_int4(0, 0, 0, 0);
+  reinterpret_cast<int4*>(hist)[2 * tid + 1] = make_int4(0, 0, 0, 0);
   griddep_wait();
   const int P = (L.len(b) + kPage - 1) / kPage;
   const int Kp = min(budget_pages, P);
   int32_t* out = cand + (int64_t)u * cand_stride;
-  const float* sc = scores + (int64_t)u * L.max_pages;
+  uint32_t* orow = row0 ? row0 + (int64_t)u * L.max_pages : nullptr;
+  auto emit = [&](int pos, int pg) {
+    out[pos] = pg;
+    if (orow) orow[pos] = (uint32_t)L.page_row(b, hk, pg);
+  };
   if (Kp >= P) {
-    for (int i = tid; i < P; i += kTopkThreads) out[i] = i;
+    for (int i = tid; i < P; i += kTopkThreads) emit(i, i);
     if (tid == 0) ncand[u] = P;
     griddep_launch();
     return;
   }
+  const float* sc = scores + (int64_t)u * L.max_pages;
+  const int E = (P + kTopkThreads - 1) / kTopkThreads;
+  const int i0 = tid * E;
   uint32_t key[kTopkCached];
+  int ptc[kTopkCached];   // page-table entries of the cached pages (paged layout, row0 wanted)
+  const bool want_pt = orow && L.page_table;
 #pragma unroll
-  for (int j = 0; j < kTopkCached; ++j) {
-    const int i = j * kTopkThreads + tid;
-    key[j] = i < P ? f_key(sc[i]) : 0u;
+  for (int k = 0; k < kTopkCached; ++k) {
+    const bool in = k < E && i0 + k < P;
+    key[k] = in ? f_key(sc[i0 + k]) : 0u;
+    ptc[k] = (want_pt && in) ? L.page_table[(int64_t)b * L.max_pages + i0 + k] : 0;
   }
-  const int chunks = (P + kTopkThreads - 1) / kTopkThreads;
-  auto key_at = [&](int j) -> uint32_t {   // key of page j * kTopkThreads + tid
-    if (j < kTopkCached) {
-      uint32_t r = 0u;
+  // f(k, key, pt) over this thread's valid pages i0 + k in order: the cached
+  // keys with static register indices, then any further ones from memory
+  auto for_keys = [&](auto&& f) {
 #pragma unroll
-      for (int t = 0; t < kTopkCached; ++t)
-        if (t == j) r = key[t];
-      return r;
-    }
-    const int i = j * kTopkThreads + tid;
-    return i < P ? f_key(sc[i]) : 0u;
+    for (int k = 0; k < kTopkCached; ++k)
+      if (k < E && i0 + k < P) f(k, key[k], ptc[k]);
+    for (int k = kTopkCached; k < E; ++k)
+      if (i0 + k < P) f(k, f_key(sc[i0 + k]), 0);
   };
-  uint32_t prefix = 0, pmask = 0;
-  int need = Kp;   // elements matching `prefix` that still belong to the top K_p
-  int* hflat = &hrep[0][0];
-  const int rep = lane & (kTopkReps - 1);
-  for (int round = 0; round < 4; ++round) {
-    const int shift = 24 - 8 * round;
-    for (int i = tid; i < kTopkReps * 256; i += kTopkThreads) hflat[i] = 0;
+  // the keys of one unit's pages share their top bits (scores of similar
+  // magnitude), so the digits start below the common prefix of the block's
+  // smallest and largest key: 12 bits, then 9 at a time
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for_keys([&](int, uint32_t kk, int) {
+    kmin = min(kmin, kk);
+    kmax = max(kmax, kk);
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    wmin[warp] = kmin;
+    wmax[warp] = kmax;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) {
+    kmin = min(kmin, wmin[w]);
+    kmax = max(kmax, wmax[w]);
+  }
+  int nb = 32 - __clz((int)(kmin ^ kmax));   // low bits still to resolve (0: all keys equal)
+  uint32_t pmask = nb >= 32 ? 0u : ~((1u << nb) - 1u);
+  uint32_t prefix = kmin & pmask;
+  int need = Kp;   // keys matching `prefix` that still belong to the top K_p
+  for (int round = 0; nb > 0; ++round) {
+    const int width = min(round == 0 ? 12 : 9, nb);
+    const int shift = nb - width;
+    const uint32_t dm = (1u << width) - 1u;
+    nb = shift;
+    for_keys([&](int, uint32_t kk, int) {
+      if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & dm], 1);
+    });
     __syncthreads();
-    for (int j = 0; j < chunks; ++j) {
-      const int i = j * kTopkThreads + tid;
-      const uint32_t k = key_at(j);
-      if (i < P && (k & pmask) == prefix) atomicAdd(&hrep[rep][(k >> shift) & 255], 1);
+    // this thread's digits: 8 tid .. 8 tid + 7 in the first round, tid after
+    int sl[8];
+    if (round == 0) {
+      const int4 a4 = reinterpret_cast<const int4*>(hist)[2 * tid];
+      const int4 b4 = reinterpret_cast<const int4*>(hist)[2 * tid + 1];
+      sl[7] = b4.w;
+      sl[6] = b4.z + sl[7];
+      sl[5] = b4.y + sl[6];
+      sl[4] = b4.x + sl[5];
+      sl[3] = a4.w + sl[4];
+      sl[2] = a4.z + sl[3];
+      sl[1] = a4.y + sl[2];
+      sl[0] = a4.x + sl[1];
+    } else {
+      sl[0] = hist[tid];
+#pragma unroll
+      for (int k = 1; k < 8; ++k) sl[k] = 0;
     }
+    int incl = sl[0];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += t;
+    }
+    if (lane == 0) wsuf[warp] = incl;
     __syncthreads();
-    // suffix sums over the 256 digits: suf[j] = sum_{d >= j} hist[d]
-    int suf = 0;
-    if (tid < 256) {
+    int after = incl - sl[0];
 #pragma unroll
-      for (int r = 0; r < kTopkReps; ++r) suf += hrep[r][tid];
+    for (int w = 0; w < kTopkWarps; ++w)
+      if (w > warp) after += wsuf[w];
+    // the digit d of the K_p-th largest key: suffix(d) >= need > suffix(d + 1)
+    const int bpt = round == 0 ? 8 : 1;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += t;
+    for (int k = 0; k < 8; ++k) {
+      if (k < bpt) {
+        const int here = sl[k] + after;
+        const int next = (k + 1 < bpt ? sl[k + 1] : 0) + after;
+        if (here >= need && next < need) {
+          sh_d = bpt * tid + k;
+          sh_above = next;
+        }
       }
-      if (lane == 0) wsum[warp] = suf;
     }
-    __syncthreads();
-    if (tid < 256)
-      for (int w = warp + 1; w < 8; ++w) suf += wsum[w];
-    // the digit of the K_p-th largest key is the largest j with suf[j] >= need
-    const int cnt = __syncthreads_count(tid < 256 && suf >= need);
-    const int d = cnt - 1;
-    if (tid == d + 1) sh_above = suf;   // elements strictly above digit d (0 when d = 255)
-    if (tid == 0) sh_d = d;
+    if (round == 0) {
+      reinterpret_cast<int4*>(hist)[2 * tid] = make_int4(0, 0, 0, 0);
+      reinterpret_cast<int4*>(hist)[2 * tid + 1] = make_int4(0, 0, 0, 0);
+    } else {
+      hist[tid] = 0;
+    }
     __syncthreads();
     need -= sh_above;
     prefix |= (uint32_t)sh_d << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
+    pmask |= dm << shift;
   }
   // keep every key above prefix and the `need` lowest-index pages equal to it
-  int ties_before = 0, written = 0;
-  for (int j = 0; j < chunks; ++j) {
-    const int i = j * kTopkThreads + tid;
-    const uint32_t k = key_at(j);
-    const bool gt = i < P && k > prefix;
-    const bool eq = i < P && k == prefix;
-    int eq_total;
-    const int eq_rank = ties_before + block_rank(eq, sh_scan, &eq_total);
-    const bool sel = gt || (eq && eq_rank < need);
-    int sel_total;
-    const int pos = written + block_rank(sel, sh_scan, &sel_total);
-    if (sel) out[pos] = i;
-    ties_before += eq_total;
-    written += sel_total;
-  }
-  if (tid == 0) ncand[u] = written;
+  int n_gt = 0, n_eq = 0;
+  for_keys([&](int, uint32_t kk, int) {
+    n_gt += kk > prefix ? 1 : 0;
+    n_eq += kk == prefix ? 1 : 0;
+  });
+  int2 tot;
+  const int2 ex = block_excl_scan2(make_int2(n_gt, n_eq), sh_scan, &tot);
+  int take = ex.y < need ? min(n_eq, need - ex.y) : 0;
+  int pos = ex.x + min(need, ex.y);
+  for_keys([&](int k, uint32_t kk, int p) {
+    bool sel = kk > prefix;
+    if (!sel && kk == prefix && take > 0) {
+      sel = true;
+      --take;
+    }
+    if (sel) {
+      const int pg = i0 + k;
+      out[pos] = pg;
+      if (orow) {
+        int64_t r;
+        if (want_pt && k < kTopkCached)
+          r = ((int64_t)((unsigned)p < (unsigned)L.pool_pages ? p : 0) * L.Hk + hk) * kPage;
+        else
+          r = L.page_row(b, hk, pg);
+        orow[pos] = (uint32_t)r;
+      }
+      ++pos;
+    }
+  });
+  if (tid == 0) ncand[u] = tot.x + min(need, tot.y);
   griddep_launch();
 }
 
@@ -287,10 +379,10 @@ cudaError_t launch_page_scores(const Layout& L, const __half* q, int Hq, const _
 }
 
 cudaError_t launch_page_topk(const Layout& L, const float* scores, int budget_pages,
-                             int32_t* cand, int cand_stride, int32_t* ncand, cudaStream_t st,
-                             bool pdl) {
+                             int32_t* cand, int cand_stride, int32_t* ncand, uint32_t* row0,
+                             cudaStream_t st, bool pdl) {
   return launch_k(k_page_topk, dim3(L.B * L.Hk), dim3(kTopkThreads), 0, st, pdl, L, scores,
-                  budget_pages, cand, cand_stride, ncand);
+                  budget_pages, cand, cand_stride, ncand, row0);
 }
 
 }  // namespace tw

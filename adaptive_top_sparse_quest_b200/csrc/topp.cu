@@ -13,23 +13,26 @@
 //   w = mean_h 2^(l_h - m_h) / Z_h  (group sets)
 // with logits l in log2 units (the estimate kernel folds log2(e) into its
 // scale) and m, Z merged from that kernel's per-32-candidate statistics.
+//
 // The threshold theta is the largest weight value whose retained mass
 // sum_{w >= theta} w reaches p.  Weights lie in [0, 1], so their fp32 bit
-// patterns order like their values and use 30 bits; theta is found most
-// significant digit first in 4 steps (8 + 8 + 8 + 6 bits) instead of the 30 of
-// a plain bisection.  Each step builds a histogram of masses per digit among
-// the weights that match the digits found so far.  Masses are exact integers
-// (each weight truncated to a multiple of 2^-40), so sums are independent of
-// order; they are accumulated with native 32-bit shared-memory atomics on a low
-// and a high word with an explicit carry.  The histogram is replicated 8 ways
-// (by lane) because the weights of a set share few exponents and the first step
-// would otherwise serialise on a few shared-memory addresses.  Across a cluster the per-CTA histograms are summed
-// through distributed shared memory.  Every weight above theta is kept, plus
-// the lowest-position weights equal to theta needed to reach p; the kept token
-// ids are compacted in ascending order by one block scan (and one exchange of
-// per-CTA totals in a cluster).  Each round costs two block barriers: the
-// replicated histogram is summed, scanned and its digit chosen by one warp
-// while the other warps clear the next round's buffer.
+// patterns order like their values and use 30 bits.  theta is found most
+// significant digit first in 3 steps of 12 + 9 + 9 bits instead of the 30
+// steps of a plain bisection.  Each step builds a histogram of masses per
+// digit over the weights that match the digits found so far; one block-wide
+// suffix scan (each thread owns 8 or 1 consecutive digits) then finds the
+// digit where the retained mass crosses p.  The 12-bit first digit splits each
+// binade of weight values 32 ways, so its shared-memory atomics rarely collide.
+// Masses are exact integers (each weight truncated to a multiple of 2^-40), so
+// sums are independent of order; they use native 32-bit atomics on a low and a
+// high word with an explicit carry.  In a cluster every CTA sums all CTAs'
+// histograms through distributed shared memory and reaches the same digit.
+// Every weight above theta is kept, plus the lowest-position weights equal to
+// theta needed to reach p; the kept token ids are compacted in ascending order
+// by one block scan (and one exchange of per-CTA totals in a cluster).  When
+// asked, the kernel also writes each kept token's physical K/V row (its page's
+// first row, from the selector's row list, plus the offset in the page), so
+// the attention kernel gathers rows without walking the page table.
 #include <cooperative_groups.h>
 
 #include "tw_common.cuh"
@@ -41,7 +44,9 @@ namespace tw {
 
 constexpr int kToppThreads = 512;
 constexpr int kToppWarps = kToppThreads / 32;
-constexpr int kHistReps = 8;
+constexpr int kBins = 4096;                      // first digit: 12 bits
+constexpr int kBinsPerThread = kBins / kToppThreads;
+static_assert(kBinsPerThread == 8, "the first round reads two uint4 of bins per thread");
 constexpr double kMassEps = 1e-12;               // exact ties at p resolve as in real arithmetic
 constexpr float kMassScale = 1099511627776.0f;   // 2^40
 
@@ -49,8 +54,13 @@ __device__ __forceinline__ unsigned long long mass_of(float w) {
   return __float2ull_rz(w * kMassScale);
 }
 
-__device__ __forceinline__ int digit_shift(int round) { return round < 3 ? 22 - 8 * round : 0; }
-__device__ __forceinline__ uint32_t digit_mask(int round) { return round < 3 ? 255u : 63u; }
+// Digits of the 30-bit weight key: bits 29..18, 17..9, 8..0.
+__device__ __forceinline__ int digit_shift(int round) { return round == 0 ? 18 : (round == 1 ? 9 : 0); }
+__device__ __forceinline__ uint32_t digit_mask(int round) { return round == 0 ? 0xFFFu : 0x1FFu; }
+
+__device__ __forceinline__ unsigned long long join64(uint32_t hi, uint32_t lo) {
+  return ((unsigned long long)hi << 32) | lo;
+}
 
 // Block-wide exclusive scan of an unsigned value in thread order; writes the
 // block total to *total.  Uses sh[0..kToppWarps].
@@ -82,25 +92,143 @@ __device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* sh, un
   return r;
 }
 
+// State of the threshold search: the digits fixed so far (prefix under pmask),
+// the mass A of the weights above that prefix range and the target mass T.
+struct Search {
+  uint32_t prefix, pmask;
+  unsigned long long A, T;
+};
+
+// One digit of the search: histogram the masses of the weights inside the
+// current prefix range by the digit (key >> shift) & dm, scan the digits from
+// the top, and fix the digit where the retained mass crosses T.  Each thread
+// owns BPT consecutive digits (BPT * 512 digits in all).  The first step (BPT
+// == 8) also sets T from the total mass, and returns false if that is zero; it
+// is the same in every CTA of a cluster, so all of them leave together.
+// Leaves the histogram zeroed.
+template <int R, int BPT, bool CLUSTER>
+__device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint32_t dm, double p,
+                                           int CS, uint32_t* hlo, uint32_t* hhi,
+                                           unsigned long long* wsuf, int* sh_d,
+                                           unsigned long long* sh_above, Search& s) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if (w[i] >= 0.f) {
+      const uint32_t key = __float_as_uint(w[i]);
+      if ((key & s.pmask) == s.prefix) {
+        // exact 64-bit mass sum from native 32-bit atomics: low word, then the
+        // high word plus the carry out of the low word
+        const unsigned long long F = mass_of(w[i]);
+        const uint32_t dg = (key >> shift) & dm;
+        const uint32_t lo = (uint32_t)F;
+        const uint32_t old = atomicAdd(&hlo[dg], lo);
+        const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
+        if (up) atomicAdd(&hhi[dg], up);
+      }
+    }
+  }
+  if (CLUSTER) cg::this_cluster().sync();
+  else __syncthreads();
+  unsigned long long sl[BPT];   // suffix sums within this thread's digits
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) sl[k] = 0;
+  for (int r = 0; r < CS; ++r) {
+    const uint32_t* lo = hlo;
+    const uint32_t* hi = hhi;
+    if (CLUSTER) {
+      cg::cluster_group cl = cg::this_cluster();
+      lo = cl.map_shared_rank(hlo, r);
+      hi = cl.map_shared_rank(hhi, r);
+    }
+    if (BPT == 8) {
+      const uint4 l0 = reinterpret_cast<const uint4*>(lo)[2 * tid];
+      const uint4 l1 = reinterpret_cast<const uint4*>(lo)[2 * tid + 1];
+      const uint4 u0 = reinterpret_cast<const uint4*>(hi)[2 * tid];
+      const uint4 u1 = reinterpret_cast<const uint4*>(hi)[2 * tid + 1];
+      const uint32_t lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+      const uint32_t uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int k = 0; k < BPT; ++k) sl[k] += join64(uv[k], lv[k]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < BPT; ++k) sl[k] += join64(hi[BPT * tid + k], lo[BPT * tid + k]);
+    }
+  }
+#pragma unroll
+  for (int k = BPT - 2; k >= 0; --k) sl[k] += sl[k + 1];
+  // suffix over this warp's higher lanes, then over the later warps
+  unsigned long long incl = sl[0];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  if (lane == 0) wsuf[warp] = incl;
+  if (CLUSTER) cg::this_cluster().sync();   // also: every peer has read this CTA's bins
+  else __syncthreads();
+  unsigned long long after = incl - sl[0];
+  unsigned long long grand = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kToppWarps; ++w2) {
+    const unsigned long long x = wsuf[w2];
+    grand += x;
+    if (w2 > warp) after += x;
+  }
+  if (BPT == 8) {
+    if (grand == 0) return false;   // no valid candidate
+    const double tf = ceil((p - kMassEps) * (double)grand);
+    unsigned long long T = tf < 1.0 ? 1ull : (unsigned long long)tf;
+    s.T = T > grand ? grand : T;
+  }
+  // the digit d with A + suffix(d) >= T > A + suffix(d + 1); exactly one thread
+  // holds it, since A < T <= A + suffix(0)
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    const unsigned long long here = s.A + sl[k] + after;
+    const unsigned long long next = s.A + (k + 1 < BPT ? sl[k + 1] : 0ull) + after;
+    if (here >= s.T && next < s.T) {
+      *sh_d = BPT * tid + k;
+      *sh_above = next - s.A;
+    }
+  }
+  // clear this thread's own digits (all readers are done) for the next step
+  if (BPT == 8) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(hlo)[2 * tid] = z;
+    reinterpret_cast<uint4*>(hlo)[2 * tid + 1] = z;
+    reinterpret_cast<uint4*>(hhi)[2 * tid] = z;
+    reinterpret_cast<uint4*>(hhi)[2 * tid + 1] = z;
+  } else {
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) hlo[BPT * tid + k] = hhi[BPT * tid + k] = 0u;
+  }
+  __syncthreads();
+  // sh_d, sh_above and wsuf are next written after the next step's first barrier
+  s.A += *sh_above;
+  s.prefix |= (uint32_t)*sh_d << shift;
+  s.pmask |= dm << shift;
+  return true;
+}
 
 // NH: heads averaged into one set (1 for per-head sets, G for group sets).
 template <int NH, int R, bool CLUSTER>
 __global__ void __launch_bounds__(kToppThreads)
 k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand,
-       int cand_stride, const int32_t* __restrict__ ncand, int lcap, int cmax,
-       const float* __restrict__ logits, const float2* __restrict__ stats, double p,
-       int32_t* __restrict__ idx, int icap, int32_t* __restrict__ count,
-       int32_t* __restrict__ done) {
+       int cand_stride, const int32_t* __restrict__ ncand, const uint32_t* __restrict__ row0,
+       int lcap, int cmax, const float* __restrict__ logits, const float2* __restrict__ stats,
+       double p, int32_t* __restrict__ idx, uint32_t* __restrict__ rows, int icap,
+       int32_t* __restrict__ count, int32_t* __restrict__ done) {
   constexpr int NPG = (R + kPage - 1) / kPage;   // candidate pages a thread's R positions span
-  __shared__ uint32_t hlo[2][kHistReps][256], hhi[2][kHistReps][256];   // double-buffered
-  __shared__ unsigned long long hloc[2][256];                           // per-CTA totals (cluster)
-  __shared__ unsigned long long sh_total, sh_above;
+  __shared__ __align__(16) uint32_t hlo[kBins];
+  __shared__ __align__(16) uint32_t hhi[kBins];
+  __shared__ unsigned long long wsuf[kToppWarps];   // per-warp suffix mass of its digits
+  __shared__ unsigned long long sh_above;
   __shared__ int sh_d;
   __shared__ unsigned sh_scan[kToppWarps + 1];
   __shared__ unsigned sh_blk[2];
   __shared__ unsigned sh_pre[4];
-  __shared__ float sh_m[NH], sh_iz[NH];
-  __shared__ float red[kToppWarps][NH];
+  __shared__ float redm[kToppWarps][NH], redz[kToppWarps][NH];
 
   int CS = 1, cr = 0;
   if (CLUSTER) {
@@ -122,17 +250,32 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   }
   const int64_t ukv = (int64_t)b * L.Hk + hk;
   const int cbase = cr * (kToppThreads * R) + tid * R;   // this thread's R consecutive candidates
+  const int spans_cap = lcap / kStatSpan;
+  const float2* st = stats + ukv * spans_cap * G + h0;
+  {   // the first round's histogram starts at zero
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(hlo)[2 * tid] = z;
+    reinterpret_cast<uint4*>(hlo)[2 * tid + 1] = z;
+    reinterpret_cast<uint4*>(hhi)[2 * tid] = z;
+    reinterpret_cast<uint4*>(hhi)[2 * tid + 1] = z;
+  }
   griddep_wait();
-  // Loads that do not depend on the candidate count go out first: the page ids
-  // of this thread's candidates and their logits (masked by the count below).
+  // Every load goes out before any result is needed: the candidate count, the
+  // page ids of this thread's candidates, their logits and the first
+  // statistics records (all masked by the count once it arrives).
+  const int len = L.len(b);
+  const int ncnt = cand ? ncand[ukv] : 0;
   int pgid[NPG];
+  uint32_t pr0[NPG];   // first physical row of each page (for the attention kernel)
 #pragma unroll
   for (int k = 0; k < NPG; ++k) {
     const int pgl = (cbase >> 4) + k;
     pgid[k] = cand ? (pgl < cand_stride ? cand[ukv * cand_stride + pgl] : -1) : pgl;
+    pr0[k] = (!rows || pgl >= L.max_pages) ? 0u
+             : row0                       ? row0[ukv * L.max_pages + pgl]
+                                          : (uint32_t)L.page_row(b, hk, pgl);   // no candidate list
   }
-  // small sets of logits are loaded now, into registers; large ones when used
-  constexpr bool kPre = NH * R <= 64;
+  constexpr bool kPre = NH * R <= 32;   // small sets of logits go to registers now
   float lv[kPre ? R : 1][kPre ? NH : 1];
   if (kPre) {
 #pragma unroll
@@ -142,56 +285,57 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
         lv[kPre ? i : 0][kPre ? h : 0] =
             (cbase + i < lcap) ? logits[(ukv * lcap + cbase + i) * G + h0 + h] : -INFINITY;
   }
-  const int len = L.len(b);
-  const int C = min(cand ? ncand[ukv] * kPage : len, cmax);
+  float2 sv[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h)
+    sv[h] = tid < spans_cap ? st[(int64_t)tid * G + h] : make_float2(-INFINITY, 0.f);
+  const int C = min(cand ? ncnt * kPage : len, cmax);
   const int nspans = (C + kStatSpan - 1) / kStatSpan;
-  const float2* st = stats + ukv * (lcap / kStatSpan) * G + h0;
-  {   // round 0's histogram starts at zero
-    uint32_t* a = &hlo[0][0][0];
-    uint32_t* c = &hhi[0][0][0];
-    for (int i = tid; i < kHistReps * 256; i += kToppThreads) a[i] = c[i] = 0u;
-  }
 
   // 1. merge the statistics records into each head's max and 1 / sum 2^(l - max)
   float mloc[NH];
 #pragma unroll
-  for (int h = 0; h < NH; ++h) mloc[h] = -INFINITY;
-  for (int t = tid; t < nspans; t += kToppThreads)
+  for (int h = 0; h < NH; ++h) mloc[h] = tid < nspans ? sv[h].x : -INFINITY;
+  for (int t = tid + kToppThreads; t < nspans; t += kToppThreads)
 #pragma unroll
     for (int h = 0; h < NH; ++h) mloc[h] = fmaxf(mloc[h], st[(int64_t)t * G + h].x);
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const float m = warp_max(mloc[h]);
-    if (lane == 0) red[warp][h] = m;
+    if (lane == 0) redm[warp][h] = m;
   }
   __syncthreads();
-  if (tid < NH) {
-    float m = -INFINITY;
-    for (int w = 0; w < kToppWarps; ++w) m = fmaxf(m, red[w][tid]);
-    sh_m[tid] = m;
+  float M[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    M[h] = redm[0][h];
+#pragma unroll
+    for (int w2 = 1; w2 < kToppWarps; ++w2) M[h] = fmaxf(M[h], redm[w2][h]);
   }
-  __syncthreads();
   float zloc[NH];
 #pragma unroll
-  for (int h = 0; h < NH; ++h) zloc[h] = 0.f;
-  for (int t = tid; t < nspans; t += kToppThreads)
+  for (int h = 0; h < NH; ++h)
+    zloc[h] = (tid < nspans && sv[h].x != -INFINITY) ? sv[h].y * exp2f(sv[h].x - M[h]) : 0.f;
+  for (int t = tid + kToppThreads; t < nspans; t += kToppThreads)
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const float2 s2 = st[(int64_t)t * G + h];
-      if (s2.x != -INFINITY) zloc[h] += s2.y * exp2f(s2.x - sh_m[h]);
+      if (s2.x != -INFINITY) zloc[h] += s2.y * exp2f(s2.x - M[h]);
     }
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const float z = warp_sum(zloc[h]);
-    if (lane == 0) red[warp][h] = z;
+    if (lane == 0) redz[warp][h] = z;
   }
   __syncthreads();
-  if (tid < NH) {
+  float iz[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
     float z = 0.f;
-    for (int w = 0; w < kToppWarps; ++w) z += red[w][tid];
-    sh_iz[tid] = z > 0.f ? 1.0f / z : 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < kToppWarps; ++w2) z += redz[w2][h];
+    iz[h] = z > 0.f ? 1.0f / z : 0.f;
   }
-  __syncthreads();
 
   // 2. weights (-1 marks an invalid slot)
   float w[R];
@@ -206,7 +350,7 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
         const float l = kPre ? lv[kPre ? i : 0][kPre ? h : 0]
                              : logits[(ukv * lcap + cbase + i) * G + h0 + h];
         ok = ok && (l != -INFINITY);
-        acc += exp2f(l - sh_m[h]) * sh_iz[h];
+        acc += exp2f(l - M[h]) * iz[h];
       }
       if (ok) w[i] = NH == 1 ? acc : acc * (1.0f / NH);
     }
@@ -215,119 +359,19 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   // 3. digit-by-digit search of theta over the cluster
   const bool keep_all = p >= 1.0;
   uint32_t theta = 0;
-  unsigned long long r_need = 0, total = 0;
+  unsigned long long r_need = 0;
   bool have = false;
   if (!keep_all) {
-    uint32_t prefix = 0, pmask = 0;
-    unsigned long long A = 0, T = 0;   // A: mass strictly above the current prefix range
-    const int rep = lane & (kHistReps - 1);
-    for (int round = 0; round < 4; ++round) {
-      const int buf = round & 1;
-      const int shift = digit_shift(round);
-      const uint32_t dm = digit_mask(round);
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        if (w[i] >= 0.f) {
-          const uint32_t key = __float_as_uint(w[i]);
-          if ((key & pmask) == prefix) {
-            // exact 64-bit mass sum from native 32-bit atomics: low word, then
-            // the high word plus the carry out of the low word
-            const unsigned long long F = mass_of(w[i]);
-            const uint32_t dg = (key >> shift) & dm;
-            const uint32_t lo = (uint32_t)F;
-            const uint32_t old = atomicAdd(&hlo[buf][rep][dg], lo);
-            const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
-            if (up) atomicAdd(&hhi[buf][rep][dg], up);
-          }
-        }
-      }
-      {   // the other buffer is not read in this round: clear it for the next one
-        uint32_t* a = &hlo[buf ^ 1][0][0];
-        uint32_t* c = &hhi[buf ^ 1][0][0];
-        for (int i = tid; i < kHistReps * 256; i += kToppThreads) a[i] = c[i] = 0u;
-      }
-      __syncthreads();
-      // warp 0: per-digit mass over the CTA (and cluster), suffix sums, the digit
-      unsigned long long v[8];
-      if (warp == 0) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int j = 8 * lane + k;
-          unsigned long long x = 0;
-#pragma unroll
-          for (int r = 0; r < kHistReps; ++r)
-            x += ((unsigned long long)hhi[buf][r][j] << 32) | hlo[buf][r][j];
-          v[k] = x;
-          if (CLUSTER) hloc[buf][j] = x;
-        }
-      }
-      if (CLUSTER) {
-        cg::cluster_group cl = cg::this_cluster();
-        cl.sync();
-        if (warp == 0) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            unsigned long long x = 0;
-            for (int r = 0; r < CS; ++r) x += cl.map_shared_rank(&hloc[buf][0], r)[8 * lane + k];
-            v[k] = x;
-          }
-        }
-      }
-      if (warp == 0) {
-        unsigned long long sl[8];   // suffix within this lane's 8 digits
-        sl[7] = v[7];
-#pragma unroll
-        for (int k = 6; k >= 0; --k) sl[k] = v[k] + sl[k + 1];
-        unsigned long long incl = sl[0];   // suffix over lanes >= this one
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long t = __shfl_down_sync(0xffffffffu, incl, o);
-          if (lane + o < 32) incl += t;
-        }
-        const unsigned long long after = incl - sl[0];   // mass of digits above this lane's
-        if (round == 0) {
-          total = __shfl_sync(0xffffffffu, incl, 0);
-          const double tf = ceil((p - kMassEps) * (double)total);
-          T = tf < 1.0 ? 1ull : (unsigned long long)tf;
-          if (T > total) T = total;
-        }
-        int cnt = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) cnt += (A + sl[k] + after >= T) ? 1 : 0;
-        cnt = warp_sum(cnt);
-        const int d = cnt - 1;   // largest digit whose suffix mass reaches T
-        const int dn = d + 1;
-        unsigned long long ab = 0;
-        if (dn < 256 && lane == (dn >> 3)) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (k == (dn & 7)) ab = sl[k] + after;
-        }
-        ab = __shfl_sync(0xffffffffu, ab, dn < 256 ? (dn >> 3) : 0);
-        if (lane == 0) {
-          sh_d = d;
-          sh_above = dn < 256 ? ab : 0ull;
-          if (round == 0) sh_total = total;
-        }
-      }
-      __syncthreads();
-      if (round == 0) {
-        total = sh_total;
-        if (total == 0) break;   // no valid candidate (uniform over the cluster)
-        const double tf = ceil((p - kMassEps) * (double)total);
-        T = tf < 1.0 ? 1ull : (unsigned long long)tf;
-        if (T > total) T = total;
-        have = true;
-      }
-      A += sh_above;
-      prefix |= (uint32_t)sh_d << shift;
-      pmask |= dm << shift;
-    }
+    Search s{0u, 0u, 0ull, 0ull};
+    have = digit_step<R, kBinsPerThread, CLUSTER>(w, 18, 0xFFFu, p, CS, hlo, hhi, wsuf, &sh_d,
+                                                 &sh_above, s);
     if (have) {
-      theta = prefix;
+      digit_step<R, 1, CLUSTER>(w, 9, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+      digit_step<R, 1, CLUSTER>(w, 0, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+      theta = s.prefix;
       unsigned long long Ft = mass_of(__uint_as_float(theta));
       if (Ft == 0) Ft = 1;
-      r_need = (T - A + Ft - 1) / Ft;
+      r_need = (s.T - s.A + Ft - 1) / Ft;
     }
   }
 
@@ -383,6 +427,7 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   if (ties_before < r_need) take = (unsigned)min((unsigned long long)n_eq, r_need - ties_before);
   unsigned pos = gt_before + (ex >> 16) + (unsigned)min(r_need, ties_before);
   int32_t* out = idx + (int64_t)set * icap;
+  uint32_t* orow = rows ? rows + (int64_t)set * icap : nullptr;
   unsigned taken = 0;
 #pragma unroll
   for (int i = 0; i < R; ++i) {
@@ -395,7 +440,10 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
     }
     if (sel) {
       const int c = cbase + i;
-      out[pos++] = cand ? pgid[(c >> 4) - (cbase >> 4)] * kPage + (c & 15) : c;
+      const int k = (c >> 4) - (cbase >> 4);
+      out[pos] = cand ? pgid[k] * kPage + (c & 15) : c;
+      if (orow) orow[pos] = pr0[k] + (uint32_t)(c & 15);
+      ++pos;
     }
   }
   if (cr == 0 && tid == 0) {
@@ -427,13 +475,14 @@ int topp_shape(int cmax, int* R, int* CS) {
 template <int NH, int R>
 static cudaError_t launch_topp_t(int sets, int CS, const Layout& L, int Hq, int G, int group_sets,
                                  const int32_t* cand, int cand_stride, const int32_t* ncand,
-                                 int lcap, int cmax, const float* logits, const float2* stats,
-                                 double p, int32_t* idx, int icap, int32_t* count,
-                                 int32_t* done, cudaStream_t st, bool pdl) {
+                                 const uint32_t* row0, int lcap, int cmax, const float* logits,
+                                 const float2* stats, double p, int32_t* idx, uint32_t* rows,
+                                 int icap, int32_t* count, int32_t* done, cudaStream_t st,
+                                 bool pdl) {
   if (CS == 1)
     return launch_k(k_topp<NH, R, false>, dim3(sets), dim3(kToppThreads), 0, st, pdl, L, Hq, G,
-                    group_sets, cand, cand_stride, ncand, lcap, cmax, logits, stats, p, idx, icap,
-                    count, done);
+                    group_sets, cand, cand_stride, ncand, row0, lcap, cmax, logits, stats, p, idx,
+                    rows, icap, count, done);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sets * CS);
   cfg.blockDim = dim3(kToppThreads);
@@ -448,13 +497,15 @@ static cudaError_t launch_topp_t(int sets, int CS, const Layout& L, int Hq, int 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_topp<NH, R, true>, L, Hq, G, group_sets, cand, cand_stride,
-                            ncand, lcap, cmax, logits, stats, p, idx, icap, count, done);
+                            ncand, row0, lcap, cmax, logits, stats, p, idx, rows, icap, count,
+                            done);
 }
 
 cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* cand,
-                        int cand_stride, const int32_t* ncand, int lcap, int cmax,
-                        const float* logits, const float2* stats, double p, int32_t* idx,
-                        int icap, int32_t* count, int32_t* done, cudaStream_t st, bool pdl) {
+                        int cand_stride, const int32_t* ncand, const uint32_t* row0, int lcap,
+                        int cmax, const float* logits, const float2* stats, double p,
+                        int32_t* idx, uint32_t* rows, int icap, int32_t* count, int32_t* done,
+                        cudaStream_t st, bool pdl) {
   const int G = Hq / L.Hk;
   const int NH = group_sets ? G : 1;
   const int sets = group_sets ? L.B * L.Hk : L.B * Hq;
@@ -463,7 +514,8 @@ cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* 
 #define TW_TOPP(NN, RR)                                                                       \
   if (NH == NN && R == RR)                                                                    \
     return launch_topp_t<NN, RR>(sets, CS, L, Hq, G, group_sets, cand, cand_stride, ncand,    \
-                                 lcap, cmax, logits, stats, p, idx, icap, count, done, st, pdl);
+                                 row0, lcap, cmax, logits, stats, p, idx, rows, icap, count,  \
+                                 done, st, pdl);
 #define TW_TOPP_R(NN) TW_TOPP(NN, 4) TW_TOPP(NN, 8) TW_TOPP(NN, 16) TW_TOPP(NN, 32)
   TW_TOPP_R(1) TW_TOPP_R(2) TW_TOPP_R(4) TW_TOPP_R(8)
 #undef TW_TOPP_R

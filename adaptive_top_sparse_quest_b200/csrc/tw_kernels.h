@@ -36,6 +36,7 @@ constexpr int kPartStride = 132;     // floats per split record: m, l, 2 pad, ac
 constexpr int kPartAcc = 4;
 constexpr int kTargetSms = 148;      // B200 SM count used to size decode splits
 constexpr int kMaxSetCandidates = 8 * 512 * 32;   // cluster of 8 x 512 threads x 32 weights
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;           // physical row list: "no token here"
 
 void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __half* scales,
                           __half* zeros, cudaStream_t st, int num_sms);
@@ -43,24 +44,30 @@ void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream
                       int num_sms);
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
                             const __half* scales, const __half* zeros, const int32_t* cand,
-                            int cand_stride, const int32_t* ncand, int lcap, int cmax,
-                            float* logits, float2* stats, cudaStream_t st, int num_sms,
-                            bool pdl);
+                            int cand_stride, const int32_t* ncand, const uint32_t* row0,
+                            int lcap, int cmax, float* logits, float2* stats, cudaStream_t st,
+                            int num_sms, bool pdl);
 int topp_shape(int cmax, int* R, int* CS);
 cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* cand,
-                        int cand_stride, const int32_t* ncand, int lcap, int cmax,
-                        const float* logits, const float2* stats, double p, int32_t* idx,
-                        int icap, int32_t* count, int32_t* done, cudaStream_t st, bool pdl);
+                        int cand_stride, const int32_t* ncand, const uint32_t* row0, int lcap,
+                        int cmax, const float* logits, const float2* stats, double p,
+                        int32_t* idx, uint32_t* rows, int icap, int32_t* count, int32_t* done,
+                        cudaStream_t st, bool pdl);
 constexpr int kDecCtas = 4 * kTargetSms;   // CTAs sharing the concatenated selected tokens
 size_t decode_part_floats(int B, int Hq, int Hk);
 cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int group_sets,
-                                 const __half* K, const __half* V, const int32_t* idx, int icap,
+                                 const __half* K, const __half* V, const uint32_t* rows, int icap,
                                  const int32_t* count, float* part, int32_t* done, __half* out,
                                  float* lse, cudaStream_t st, bool pdl);
 cudaError_t launch_page_scores(const Layout& L, const __half* q, int Hq, const __half* meta,
                                float* scores, cudaStream_t st, int num_sms, bool pdl);
 cudaError_t launch_page_topk(const Layout& L, const float* scores, int budget_pages,
-                             int32_t* cand, int cand_stride, int32_t* ncand, cudaStream_t st,
-                             bool pdl);
+                             int32_t* cand, int cand_stride, int32_t* ncand, uint32_t* row0,
+                             cudaStream_t st, bool pdl);
+cudaError_t launch_resolve_pages(const Layout& L, const int32_t* cand, int cand_stride,
+                                 uint32_t* row0, cudaStream_t st, bool pdl);
+cudaError_t launch_resolve_rows(const Layout& L, int Hq, int group_sets, const int32_t* idx,
+                                int icap, const int32_t* count, uint32_t* rows, cudaStream_t st,
+                                bool pdl);
 
 }  // namespace tw

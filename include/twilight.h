@@ -188,8 +188,9 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
  * Same inputs, outputs and results as tw_topp_prune; the scratch is one fixed
  * array of TW_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library, resident
  * on every GPU that loads it until the process exits.  Shapes whose scratch
- * (logits and softmax statistics: about B * Hk * capacity * G * 4 bytes) does
- * not fit return TW_ERR_CAPACITY before any device work.  The first call on a
+ * (logits and softmax statistics, about B * Hk * capacity * G * 4 bytes, plus
+ * 4 bytes per page of the B * Hk * ceil(N / 16) cache pages) does not fit
+ * return TW_ERR_CAPACITY before any device work.  The first call on a
  * device looks up the array's device address (TW_ERR_CUDA if that fails), so
  * make it before any stream capture.  Every call shares the array: calls that
  * overlap on the GPU race.  Nothing in it needs to start at zero.
