@@ -21,7 +21,8 @@
 // table; kNoRow marks an id outside the sequence), so no page-table load sits
 // in front of a gather.  The rows of a window of the range are staged in
 // shared memory once; the gathered 256-byte K and V rows then stream through a
-// 4-stage cp.async ring of 16 tokens per stage (32 KB in flight per CTA), so
+// 6-stage cp.async ring of 16 tokens per stage (40 KB in flight per CTA, four
+// CTAs per SM: about the whole working set of a 32k-context step at once), so
 // a CTA pays one dependent round trip per window instead of one per batch.
 // Each half-warp takes 2 tokens of a stage; lane l of the half-warp holds
 // channels 8l..8l+7, the scores are reduced with 4 xor-shuffles and the online
@@ -41,7 +42,7 @@ namespace tw {
 constexpr int kDecThreads = 128;
 constexpr int kDecHW = kDecThreads / 16;       // half-warps
 constexpr int kStageTok = 16;                  // tokens per pipeline stage
-constexpr int kStages = 4;
+constexpr int kStages = 6;                     // 5 stages (40 KB) in flight per CTA
 constexpr int kWin = 512;                      // token rows staged per window
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -262,7 +263,8 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
                 const uint32_t* __restrict__ rows, int icap, const int32_t* __restrict__ count,
                 int nsets, float* __restrict__ part, int32_t* __restrict__ done,
                 __half* __restrict__ out, float* __restrict__ lse) {
-  __shared__ __align__(16) DecSmem<NH> sm;
+  extern __shared__ __align__(16) unsigned char dec_smem_raw[];
+  DecSmem<NH>& sm = *reinterpret_cast<DecSmem<NH>*>(dec_smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int hw = tid >> 4, l16 = tid & 15;
   const unsigned hmask = 0xFFFFu << (lane & 16);
@@ -507,6 +509,15 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
   griddep_launch();
 }
 
+template <int NH>
+static cudaError_t dec_prepare() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaErrorNotReady)
+    done = cudaFuncSetAttribute(k_sparse_decode<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(DecSmem<NH>));
+  return done;
+}
+
 size_t decode_part_floats(int B, int Hq, int Hk) {
   const int G = Hq / Hk;
   const size_t grp = (size_t)(kDecCtas + B * Hk) * G * kPartStride;
@@ -523,9 +534,13 @@ cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int g
   const int nsets = group_sets ? L.B * L.Hk : L.B * Hq;
   switch (NH) {
 #define TW_DEC(NN)                                                                           \
-  case NN:                                                                                   \
-    return launch_k(k_sparse_decode<NN>, dim3(kDecCtas), dim3(kDecThreads), 0, st, pdl, L, q, \
-                    Hq, G, group_sets, K, V, rows, icap, count, nsets, part, done, out, lse);
+  case NN: {                                                                                 \
+    const cudaError_t e = dec_prepare<NN>();                                                 \
+    if (e != cudaSuccess) return e;                                                          \
+    return launch_k(k_sparse_decode<NN>, dim3(kDecCtas), dim3(kDecThreads),                  \
+                    sizeof(DecSmem<NN>), st, pdl, L, q, Hq, G, group_sets, K, V, rows, icap, \
+                    count, nsets, part, done, out, lse);                                     \
+  }
     TW_DEC(1) TW_DEC(2) TW_DEC(4) TW_DEC(8)
 #undef TW_DEC
   }

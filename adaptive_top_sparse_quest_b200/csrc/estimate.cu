@@ -30,7 +30,7 @@
 // (no page-table walk here); warp 0 issues those lookups two items before
 // their gathers and stores them one iteration later, so neither the lookups
 // nor the gathers sit on the critical path.  Each of the eight warps then takes 32 candidates (two MMA
-// tiles) and writes the fp32 logits [unit][cap][G] plus its per-head
+// tiles) and writes the fp32 logits [unit][G][cap] plus its per-head
 // (max, sum 2^(l - max)).
 #include "tw_common.cuh"
 #include "tw_kernels.h"
@@ -300,13 +300,14 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
       for (int hp = 0; hp < HP; ++hp) {
         const int he = 2 * hp + (t >> 1);
         const bool hv = he < G;
-        // logits [unit][lcap][G]
+        // logits [unit][G][lcap]: 8 lanes store 8 consecutive candidates of a head
         if (owner && hv) {
+          float* lrow = logits + ((int64_t)u * G + he) * lcap;
 #pragma unroll
           for (int k = 0; k < kEstTiles; ++k) {
             const int c0 = cw0 + k * 16 + gid;
-            if (c0 < Cu) logits[((int64_t)u * lcap + c0) * G + he] = lg[k][hp][0];
-            if (c0 + 8 < Cu) logits[((int64_t)u * lcap + c0 + 8) * G + he] = lg[k][hp][1];
+            if (c0 < Cu) lrow[c0] = lg[k][hp][0];
+            if (c0 + 8 < Cu) lrow[c0 + 8] = lg[k][hp][1];
           }
         }
         // (max, sum 2^(l - max)) over this warp's 32 candidates for head he

@@ -129,7 +129,7 @@ k_page_scores(Layout L, const __half* __restrict__ q, int Hq, const __half* __re
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkCached = 16;  // keys per thread kept in registers (8192 pages)
+constexpr int kTopkMaxCached = 16;   // keys per thread kept in registers (up to 8192 pages)
 constexpr int kTopkBins = 4096;  // first digit: 12 bits (8 per thread), then 9 (1 per thread)
 
 // Inclusive scan over the block, in thread order, of a pair of counts; returns
@@ -172,8 +172,10 @@ __device__ __forceinline__ int2 block_excl_scan2(int2 v, int2* sh, int2* total) 
 // One block per (b, kv head): the K_p largest page scores, ties to the lower
 // page index, written in ascending page order (and, when row0 is given, each
 // kept page's first physical row).  Thread t owns the E consecutive pages
-// [t E, t E + E); the first kTopkCached keys stay in registers, later ones are
-// re-read from the score buffer.
+// [t E, t E + E); the first EC keys stay in registers (EC is chosen from the
+// cache's page count, so the unrolled loops are as long as the work), later
+// ones are re-read from the score buffer.
+template <int EC>
 __global__ void __launch_bounds__(kTopkThreads, 2)
 k_page_topk(Layout L, const float* __restrict__ scores, int budget_pages,
             int32_t* __restrict__ cand, int cand_stride, int32_t* __restrict__ ncand,
@@ -206,11 +208,11 @@ k_page_topk(Layout L, const float* __restrict__ scores, int budget_pages,
   const float* sc = scores + (int64_t)u * L.max_pages;
   const int E = (P + kTopkThreads - 1) / kTopkThreads;
   const int i0 = tid * E;
-  uint32_t key[kTopkCached];
-  int ptc[kTopkCached];   // page-table entries of the cached pages (paged layout, row0 wanted)
+  uint32_t key[EC];
+  int ptc[EC];   // page-table entries of the cached pages (paged layout, row0 wanted)
   const bool want_pt = orow && L.page_table;
 #pragma unroll
-  for (int k = 0; k < kTopkCached; ++k) {
+  for (int k = 0; k < EC; ++k) {
     const bool in = k < E && i0 + k < P;
     key[k] = in ? f_key(sc[i0 + k]) : 0u;
     ptc[k] = (want_pt && in) ? L.page_table[(int64_t)b * L.max_pages + i0 + k] : 0;
@@ -219,9 +221,9 @@ k_page_topk(Layout L, const float* __restrict__ scores, int budget_pages,
   // keys with static register indices, then any further ones from memory
   auto for_keys = [&](auto&& f) {
 #pragma unroll
-    for (int k = 0; k < kTopkCached; ++k)
+    for (int k = 0; k < EC; ++k)
       if (k < E && i0 + k < P) f(k, key[k], ptc[k]);
-    for (int k = kTopkCached; k < E; ++k)
+    for (int k = EC; k < E; ++k)
       if (i0 + k < P) f(k, f_key(sc[i0 + k]), 0);
   };
   // the keys of one unit's pages share their top bits (scores of similar
@@ -335,7 +337,7 @@ k_page_topk(Layout L, const float* __restrict__ scores, int budget_pages,
       out[pos] = pg;
       if (orow) {
         int64_t r;
-        if (want_pt && k < kTopkCached)
+        if (want_pt && k < EC)
           r = ((int64_t)((unsigned)p < (unsigned)L.pool_pages ? p : 0) * L.Hk + hk) * kPage;
         else
           r = L.page_row(b, hk, pg);
@@ -381,8 +383,14 @@ cudaError_t launch_page_scores(const Layout& L, const __half* q, int Hq, const _
 cudaError_t launch_page_topk(const Layout& L, const float* scores, int budget_pages,
                              int32_t* cand, int cand_stride, int32_t* ncand, uint32_t* row0,
                              cudaStream_t st, bool pdl) {
-  return launch_k(k_page_topk, dim3(L.B * L.Hk), dim3(kTopkThreads), 0, st, pdl, L, scores,
-                  budget_pages, cand, cand_stride, ncand, row0);
+  const int e = (L.max_pages + kTopkThreads - 1) / kTopkThreads;
+#define TW_TK(EE)                                                                             \
+  if (e <= EE || EE == kTopkMaxCached)                                                        \
+    return launch_k(k_page_topk<EE>, dim3(L.B * L.Hk), dim3(kTopkThreads), 0, st, pdl, L,     \
+                    scores, budget_pages, cand, cand_stride, ncand, row0);
+  TW_TK(1) TW_TK(2) TW_TK(4) TW_TK(8) TW_TK(16)
+#undef TW_TK
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace tw

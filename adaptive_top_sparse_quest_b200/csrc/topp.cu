@@ -211,6 +211,33 @@ __device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint3
   return true;
 }
 
+// Shared memory of k_topp<NH, R>: the mass histogram (reused after the
+// search to stage the outputs), then, for mid-sized logit runs, a staging
+// area the logits are copied into while the statistics are merged.
+// kMode: 0 = logits to registers at entry, 1 = to shared memory at entry,
+// 2 = loaded once the statistics are known.
+template <int NH, int R>
+struct ToppShape {
+  static constexpr int kMode = NH * R <= 16 ? 0 : (NH * R <= 64 ? 1 : 2);
+  static constexpr size_t kHistBytes =
+      2 * kBins * 4 > kToppThreads * R * 4 ? 2 * kBins * 4 : (size_t)kToppThreads * R * 4;
+  static constexpr size_t kBytes = kHistBytes + (kMode == 1 ? (size_t)kToppThreads * NH * R * 4 : 0);
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (unsigned)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // NH: heads averaged into one set (1 for per-head sets, G for group sets).
 template <int NH, int R, bool CLUSTER>
 __global__ void __launch_bounds__(kToppThreads)
@@ -220,8 +247,12 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
        double p, int32_t* __restrict__ idx, uint32_t* __restrict__ rows, int icap,
        int32_t* __restrict__ count, int32_t* __restrict__ done) {
   constexpr int NPG = (R + kPage - 1) / kPage;   // candidate pages a thread's R positions span
-  __shared__ __align__(16) uint32_t hlo[kBins];
-  __shared__ __align__(16) uint32_t hhi[kBins];
+  using SH = ToppShape<NH, R>;
+  extern __shared__ __align__(16) unsigned char topp_smem_raw[];
+  uint32_t* hlo = reinterpret_cast<uint32_t*>(topp_smem_raw);   // mass histogram, low words
+  uint32_t* hhi = hlo + kBins;                                   // and high words
+  uint32_t* obuf = hlo;   // after the search: this CTA's output, staged for coalesced stores
+  float4* lstage = reinterpret_cast<float4*>(topp_smem_raw + SH::kHistBytes);   // [NH][R/4][512]
   __shared__ unsigned long long wsuf[kToppWarps];   // per-warp suffix mass of its digits
   __shared__ unsigned long long sh_above;
   __shared__ int sh_d;
@@ -275,15 +306,30 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
              : row0                       ? row0[ukv * L.max_pages + pgl]
                                           : (uint32_t)L.page_row(b, hk, pgl);   // no candidate list
   }
-  constexpr bool kPre = NH * R <= 32;   // small sets of logits go to registers now
-  float lv[kPre ? R : 1][kPre ? NH : 1];
-  if (kPre) {
+  // logits [unit][G][lcap]: per head, this thread's R candidates are one
+  // contiguous run of R / 4 float4 (R and lcap are multiples of 4)
+  auto lrun = [&](int h) {
+    return reinterpret_cast<const float4*>(logits + (ukv * G + h0 + h) * lcap + cbase);
+  };
+  const float4 kNone = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  float4 lv[SH::kMode == 0 ? NH : 1][SH::kMode == 0 ? R / 4 : 1];
+  if (SH::kMode == 0) {   // few: straight to registers
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int h = 0; h < NH; ++h)
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
-        lv[kPre ? i : 0][kPre ? h : 0] =
-            (cbase + i < lcap) ? logits[(ukv * lcap + cbase + i) * G + h0 + h] : -INFINITY;
+      for (int j = 0; j < R / 4; ++j)
+        lv[SH::kMode == 0 ? h : 0][SH::kMode == 0 ? j : 0] =
+            cbase + 4 * j < lcap ? lrun(h)[j] : kNone;
+  } else if (SH::kMode == 1) {   // more: to shared memory by cp.async, read after the statistics
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int j = 0; j < R / 4; ++j) {
+        float4* dst = &lstage[(h * (R / 4) + j) * kToppThreads + tid];
+        if (cbase + 4 * j < lcap) cp_async16(dst, lrun(h) + j);
+        else *dst = kNone;
+      }
+    cp_async_commit();
   }
   float2 sv[NH];
 #pragma unroll
@@ -338,23 +384,33 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   }
 
   // 2. weights (-1 marks an invalid slot)
+  if (SH::kMode == 1) {
+    cp_async_wait<0>();   // each thread reads back only its own staged logits
+  }
   float w[R];
 #pragma unroll
-  for (int i = 0; i < R; ++i) {
-    w[i] = -1.0f;
-    if (cbase + i < C) {
-      float acc = 0.f;
-      bool ok = true;
+  for (int i = 0; i < R; ++i) w[i] = 0.f;
+  bool okw[R];
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const float l = kPre ? lv[kPre ? i : 0][kPre ? h : 0]
-                             : logits[(ukv * lcap + cbase + i) * G + h0 + h];
-        ok = ok && (l != -INFINITY);
-        acc += exp2f(l - M[h]) * iz[h];
+  for (int i = 0; i < R; ++i) okw[i] = cbase + i < C;
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+#pragma unroll
+    for (int j = 0; j < R / 4; ++j) {
+      float4 l4;
+      if (SH::kMode == 0) l4 = lv[SH::kMode == 0 ? h : 0][SH::kMode == 0 ? j : 0];
+      else if (SH::kMode == 1) l4 = lstage[(h * (R / 4) + j) * kToppThreads + tid];
+      else l4 = cbase + 4 * j < lcap ? lrun(h)[j] : kNone;
+      const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        okw[4 * j + e] = okw[4 * j + e] && (l[e] != -INFINITY);
+        w[4 * j + e] += exp2f(l[e] - M[h]) * iz[h];
       }
-      if (ok) w[i] = NH == 1 ? acc : acc * (1.0f / NH);
     }
   }
+#pragma unroll
+  for (int i = 0; i < R; ++i) w[i] = okw[i] ? (NH == 1 ? w[i] : w[i] * (1.0f / NH)) : -1.0f;
 
   // 3. digit-by-digit search of theta over the cluster
   const bool keep_all = p >= 1.0;
@@ -425,26 +481,46 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   const unsigned long long ties_before = (unsigned long long)eq_before + (ex & 0xFFFFu);
   unsigned take = 0;
   if (ties_before < r_need) take = (unsigned)min((unsigned long long)n_eq, r_need - ties_before);
-  unsigned pos = gt_before + (ex >> 16) + (unsigned)min(r_need, ties_before);
-  int32_t* out = idx + (int64_t)set * icap;
-  uint32_t* orow = rows ? rows + (int64_t)set * icap : nullptr;
-  unsigned taken = 0;
+  // this CTA's outputs are one contiguous run [first, first + n_out) of the
+  // set's list; they are staged in shared memory and written coalesced
+  const unsigned first = gt_before + (unsigned)min(r_need, (unsigned long long)eq_before);
+  const unsigned eq_blk = blk_total & 0xFFFFu;
+  const unsigned n_out =
+      (blk_total >> 16) +
+      (r_need > eq_before ? (unsigned)min((unsigned long long)eq_blk, r_need - eq_before) : 0u);
+  const unsigned lpos0 = (ex >> 16) + (unsigned)min(r_need, ties_before) -
+                         (unsigned)min(r_need, (unsigned long long)eq_before);
+  unsigned sel_mask = 0;   // bit i: candidate cbase + i is kept
+  {
+    unsigned taken = 0;
 #pragma unroll
-  for (int i = 0; i < R; ++i) {
-    if (w[i] < 0.f) continue;
-    const uint32_t key = __float_as_uint(w[i]);
-    bool sel = keep_all || (have && key > theta);
-    if (!sel && have && key == theta && taken < take) {
-      sel = true;
-      ++taken;
+    for (int i = 0; i < R; ++i) {
+      if (w[i] < 0.f) continue;
+      const uint32_t key = __float_as_uint(w[i]);
+      bool sel = keep_all || (have && key > theta);
+      if (!sel && have && key == theta && taken < take) {
+        sel = true;
+        ++taken;
+      }
+      if (sel) sel_mask |= 1u << i;
     }
-    if (sel) {
-      const int c = cbase + i;
-      const int k = (c >> 4) - (cbase >> 4);
-      out[pos] = cand ? pgid[k] * kPage + (c & 15) : c;
-      if (orow) orow[pos] = pr0[k] + (uint32_t)(c & 15);
-      ++pos;
+  }
+  int32_t* out = idx + (int64_t)set * icap + first;
+  for (int pass = 0; pass < (rows ? 2 : 1); ++pass) {
+    unsigned lp = lpos0;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      if (sel_mask & (1u << i)) {
+        const int c = cbase + i;
+        const int k = (c >> 4) - (cbase >> 4);
+        obuf[lp++] = pass == 0 ? (uint32_t)(cand ? pgid[k] * kPage + (c & 15) : c)
+                               : pr0[k] + (uint32_t)(c & 15);
+      }
     }
+    __syncthreads();
+    uint32_t* dst = pass == 0 ? reinterpret_cast<uint32_t*>(out) : rows + (int64_t)set * icap + first;
+    for (unsigned i = tid; i < n_out; i += kToppThreads) dst[i] = obuf[i];
+    __syncthreads();   // obuf is rewritten by the next pass
   }
   if (cr == 0 && tid == 0) {
     count[set] = (int32_t)(gt_all + (unsigned)min(r_need, (unsigned long long)eq_all));
@@ -479,13 +555,24 @@ static cudaError_t launch_topp_t(int sets, int CS, const Layout& L, int Hq, int 
                                  const float2* stats, double p, int32_t* idx, uint32_t* rows,
                                  int icap, int32_t* count, int32_t* done, cudaStream_t st,
                                  bool pdl) {
+  using SH = ToppShape<NH, R>;
+  static cudaError_t prepared = cudaErrorNotReady;
+  if (prepared == cudaErrorNotReady) {
+    prepared = cudaFuncSetAttribute(k_topp<NH, R, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SH::kBytes);
+    if (prepared == cudaSuccess)
+      prepared = cudaFuncSetAttribute(k_topp<NH, R, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SH::kBytes);
+  }
+  if (prepared != cudaSuccess) return prepared;
   if (CS == 1)
-    return launch_k(k_topp<NH, R, false>, dim3(sets), dim3(kToppThreads), 0, st, pdl, L, Hq, G,
+    return launch_k(k_topp<NH, R, false>, dim3(sets), dim3(kToppThreads), SH::kBytes, st, pdl, L, Hq, G,
                     group_sets, cand, cand_stride, ncand, row0, lcap, cmax, logits, stats, p, idx,
                     rows, icap, count, done);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sets * CS);
   cfg.blockDim = dim3(kToppThreads);
+  cfg.dynamicSmemBytes = SH::kBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
