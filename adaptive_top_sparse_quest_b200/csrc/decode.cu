@@ -9,8 +9,9 @@
 // Work split.  The selected-token counts are only known on the device and
 // differ per set (head or KV group) by an order of magnitude, so a fixed split
 // per set leaves most of the GPU idle.  The selected tokens of all sets are
-// viewed as one concatenated list of S tokens and a fixed grid of kDecCtas
-// CTAs takes equal contiguous ranges: CTA c owns [c*S/n, (c+1)*S/n).  Each CTA
+// viewed as one concatenated list of S tokens and a grid of n CTAs (up to
+// kDecCtas, fewer for a few wide GQA sets; see decode_grid) takes equal
+// contiguous ranges: CTA c owns [c*S/n, (c+1)*S/n).  Each CTA
 // derives the set offsets from the counts.  For every set its range touches,
 // the CTA writes one partial record {m, l, acc[128]} per query head to slot
 // (c + set), unique because (c, set) pairs advance monotonically along the
@@ -86,13 +87,17 @@ __device__ __forceinline__ bool range_has(int64_t c, int64_t S, int n, int64_t o
 }
 
 // Merge layout: 32 lanes with a float4 each cover one head's 128 channels.
-// With fewer than 4 heads the warps also split the records (kMergeRS ways);
-// with 8 heads each thread carries two heads.
+// With fewer than 4 heads the warps also split the records (RS ways); with 8
+// heads each thread carries two heads.  The records' accumulator rows are
+// staged in shared memory (the idle K/V ring) by cp.async, kMergeStageBytes
+// at a time.
+constexpr int kMergeStageBytes = 36 * 1024;
+
 template <int NH>
 struct MergeShape {
   static constexpr int RS = NH >= 4 ? 1 : 4 / NH;    // record split
   static constexpr int HPT = NH > 4 ? NH / 4 : 1;    // heads per thread
-  static constexpr int U = NH >= 4 ? 8 / HPT : 16;   // records per batch of loads
+  static constexpr int CAP = kMergeStageBytes / (NH * kHeadDim * 4);   // records per staged batch
 };
 
 template <int NH>
@@ -105,6 +110,7 @@ struct DecSmem {
       float acc[kDecHW][NH][kHeadDim];
     } comb;
     struct {
+      float4 stage[MergeShape<NH>::CAP][NH][kHeadDim / 4];      // staged accumulator rows
       float f[NH][kDecThreads];                                 // weights of a chunk of records
       float red[kDecThreads / 32][NH];
       float4 acc[MergeShape<NH>::RS][NH][kHeadDim / 4];         // per-split partial sums
@@ -119,8 +125,10 @@ struct DecSmem {
 };
 
 // Fold the records of `set` into out / lse (called by the CTA that completes
-// it).  All heads are folded together; the records were written by other CTAs
-// of this launch, so they are read through L2 only (ld.global.cg).
+// it).  All heads are folded together.  The records were written by other
+// CTAs of this launch, so they are read through L2 only (ld.global.cg and
+// cp.async.cg).  The first batch of accumulator rows is requested before the
+// (m, l) pairs, so a set whose records fit one batch costs one round trip.
 template <int NH>
 __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_t S, int n_ctas,
                           int Hq, int hq0, int b, const float* part, __half* out, float* lse) {
@@ -130,9 +138,21 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
   const int64_t c1 = ((off + cnt) * n_ctas + S - 1) / S - 1;
   const int nrec = (int)(c1 - c0 + 1);
   auto rec_ptr = [&](int r, int h) { return part + ((c0 + r + set) * NH + h) * kPartStride; };
+  auto valid = [&](int r) { return range_has(c0 + r, S, n_ctas, off, cnt); };
+  // stage the accumulator rows of records [r0, r0 + nr); a slot of a record
+  // that was never written (an empty range) is copied too but gets weight 0
+  auto stage = [&](int r0, int nr) {
+    for (int x = t; x < nr * NH * (kHeadDim / 4); x += kDecThreads) {
+      const int r = x / (NH * (kHeadDim / 4)), h = (x / (kHeadDim / 4)) % NH, q4 = x % (kHeadDim / 4);
+      cp_async16(&sm.u.merge.stage[r][h][q4], rec_ptr(r0 + r, h) + kPartAcc + 4 * q4);
+    }
+    cp_async_commit();
+  };
+  __syncthreads();   // the shared union was used by the caller
+  stage(0, min(nrec, MS::CAP));
   // 1. per-head max over the records; the first chunk's (m, l) stay in registers
   float m0[NH], l0[NH], mx[NH];
-  const bool v0 = t < nrec && range_has(c0 + t, S, n_ctas, off, cnt);
+  const bool v0 = t < nrec && valid(t);
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const float2 ml = v0 ? __ldcg(reinterpret_cast<const float2*>(rec_ptr(t, h)))
@@ -142,10 +162,9 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
     mx[h] = ml.x;
   }
   for (int r = t + kDecThreads; r < nrec; r += kDecThreads)
-    if (range_has(c0 + r, S, n_ctas, off, cnt))
+    if (valid(r))
 #pragma unroll
       for (int h = 0; h < NH; ++h) mx[h] = fmaxf(mx[h], __ldcg(rec_ptr(r, h)));
-  __syncthreads();   // the shared union was used by the caller
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     const float v = warp_max(mx[h]);
@@ -159,7 +178,7 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
 #pragma unroll
     for (int w = 1; w < kDecThreads / 32; ++w) M[h] = fmaxf(M[h], sm.u.merge.red[w][h]);
   }
-  // 2. chunks of 128 records: weights 2^(m_r - M), then the weighted rows
+  // 2. chunks of 128 records: weights 2^(m_r - M), then the staged rows
   const int rs = warp / (NH >= 4 ? 4 : NH) % MS::RS;    // this warp's record split
   const int hbase = NH >= 4 ? warp : warp % NH;          // first head of this thread
   float Lp[NH];
@@ -168,8 +187,9 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
   for (int h = 0; h < NH; ++h) Lp[h] = 0.f;
 #pragma unroll
   for (int k = 0; k < MS::HPT; ++k) A[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int r0 = 0; r0 < nrec; r0 += kDecThreads) {
-    const int r = r0 + t;
+  bool staged_first = true;
+  for (int w0 = 0; w0 < nrec; w0 += kDecThreads) {
+    const int r = w0 + t;
     bool vr = v0;
     float mr[NH], lr[NH];
 #pragma unroll
@@ -177,8 +197,8 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
       mr[h] = m0[h];
       lr[h] = l0[h];
     }
-    if (r0 > 0) {
-      vr = r < nrec && range_has(c0 + r, S, n_ctas, off, cnt);
+    if (w0 > 0) {
+      vr = r < nrec && valid(r);
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         const float2 ml = vr ? __ldcg(reinterpret_cast<const float2*>(rec_ptr(r, h)))
@@ -186,40 +206,36 @@ __device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_
         mr[h] = ml.x;
         lr[h] = ml.y;
       }
-      __syncthreads();   // the previous chunk's weights are no longer read
     }
+    __syncthreads();   // the previous chunk's weights are no longer read
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const float f = (vr && mr[h] != -INFINITY) ? exp2f(mr[h] - M[h]) : 0.f;
       Lp[h] += lr[h] * f;
       sm.u.merge.f[h][t] = f;
     }
-    __syncthreads();
-    const int nr = min(kDecThreads, nrec - r0);
-    for (int i0 = rs; i0 < nr; i0 += MS::RS * MS::U) {
-      float fv[MS::U][MS::HPT];
-      float4 x[MS::U][MS::HPT];
-#pragma unroll
-      for (int u = 0; u < MS::U; ++u) {
-        const int i = i0 + u * MS::RS;
+    const int wn = min(kDecThreads, nrec - w0);
+    for (int b0 = w0; b0 < w0 + wn; b0 += MS::CAP) {
+      const int nr = min(MS::CAP, w0 + wn - b0);
+      if (!staged_first) stage(b0, nr);
+      staged_first = false;
+      cp_async_wait<0>();
+      __syncthreads();   // staged rows and weights visible
+      for (int i = rs; i < nr; i += MS::RS) {
 #pragma unroll
         for (int k = 0; k < MS::HPT; ++k) {
           const int h = hbase + 4 * k;
-          fv[u][k] = i < nr ? sm.u.merge.f[h][i] : 0.f;
-          x[u][k] = fv[u][k] != 0.f
-                        ? __ldcg(reinterpret_cast<const float4*>(rec_ptr(r0 + i, h) + kPartAcc) + lane)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float f = sm.u.merge.f[h][b0 - w0 + i];
+          if (f != 0.f) {
+            const float4 x = sm.u.merge.stage[i][h][lane];
+            A[k].x = __fmaf_rn(f, x.x, A[k].x);
+            A[k].y = __fmaf_rn(f, x.y, A[k].y);
+            A[k].z = __fmaf_rn(f, x.z, A[k].z);
+            A[k].w = __fmaf_rn(f, x.w, A[k].w);
+          }
         }
       }
-#pragma unroll
-      for (int u = 0; u < MS::U; ++u)
-#pragma unroll
-        for (int k = 0; k < MS::HPT; ++k) {
-          A[k].x = __fmaf_rn(fv[u][k], x[u][k].x, A[k].x);
-          A[k].y = __fmaf_rn(fv[u][k], x[u][k].y, A[k].y);
-          A[k].z = __fmaf_rn(fv[u][k], x[u][k].z, A[k].z);
-          A[k].w = __fmaf_rn(fv[u][k], x[u][k].w, A[k].w);
-        }
+      __syncthreads();   // the stage is refilled by the next batch
     }
   }
   // 3. totals: sum of l-weights per head, the record splits' partial rows
@@ -509,6 +525,17 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
   griddep_launch();
 }
 
+// Grid of the attention kernel: kDecCtas CTAs share the concatenated selected
+// tokens, but a set's partial records are folded by one CTA, which reads them
+// through L2 at a few tens of GB/s.  So few, wide sets (GQA at batch 1) get
+// fewer CTAs: at most about 128 / NH records of 512 B per head and set (64 KB),
+// never fewer than two CTAs per SM.
+static int decode_grid(int nsets, int NH) {
+  const long long want = (long long)nsets * (128 / NH);
+  const int lo = 2 * kTargetSms;
+  return want < lo ? lo : (want > kDecCtas ? kDecCtas : (int)want);
+}
+
 template <int NH>
 static cudaError_t dec_prepare() {
   static cudaError_t done = cudaErrorNotReady;
@@ -537,7 +564,7 @@ cudaError_t launch_sparse_decode(const Layout& L, const __half* q, int Hq, int g
   case NN: {                                                                                 \
     const cudaError_t e = dec_prepare<NN>();                                                 \
     if (e != cudaSuccess) return e;                                                          \
-    return launch_k(k_sparse_decode<NN>, dim3(kDecCtas), dim3(kDecThreads),                  \
+    return launch_k(k_sparse_decode<NN>, dim3(decode_grid(nsets, NN)), dim3(kDecThreads),    \
                     sizeof(DecSmem<NN>), st, pdl, L, q, Hq, G, group_sets, K, V, rows, icap, \
                     count, nsets, part, done, out, lse);                                     \
   }
