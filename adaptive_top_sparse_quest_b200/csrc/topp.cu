@@ -211,6 +211,124 @@ __device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint3
   return true;
 }
 
+// Cluster form of digit_step: CTA r of the cluster sums slice r of the digits
+// ([r NB / CS, (r + 1) NB / CS)) over every CTA's histogram through
+// distributed shared memory (a reduce-scatter, so each histogram word crosses
+// the cluster once), the slice totals are exchanged, and the one thread whose
+// digit holds the crossing writes it into every CTA's shared memory.  Three
+// cluster barriers per step; leaves this CTA's histogram zeroed.
+template <int R, int NB>
+__device__ __forceinline__ bool digit_step_cluster(const float (&w)[R], int shift, uint32_t dm,
+                                                   double p, int CS, int cr, uint32_t* hlo,
+                                                   uint32_t* hhi, unsigned long long* wsuf,
+                                                   unsigned long long* slice_tot, int* sh_d,
+                                                   unsigned long long* sh_above, Search& s) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if (w[i] >= 0.f) {
+      const uint32_t key = __float_as_uint(w[i]);
+      if ((key & s.pmask) == s.prefix) {
+        const unsigned long long F = mass_of(w[i]);
+        const uint32_t dg = (key >> shift) & dm;
+        const uint32_t lo = (uint32_t)F;
+        const uint32_t old = atomicAdd(&hlo[dg], lo);
+        const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
+        if (up) atomicAdd(&hhi[dg], up);
+      }
+    }
+  }
+  cl.sync();   // every CTA's histogram is complete
+  const int SB = NB / CS;                                       // digits per slice
+  const int bpt = SB > kToppThreads ? SB / kToppThreads : 1;    // digits per thread (<= 8)
+  const int first = cr * SB + tid * bpt;                        // this thread's first digit
+  const bool holder = tid * bpt < SB;
+  unsigned long long sl[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) sl[k] = 0;
+  if (holder) {
+    // every peer's words are requested before any is added, so the remote
+    // loads overlap instead of costing one round trip per peer
+    for (int k0 = 0; k0 < bpt; k0 += 2) {
+      uint32_t lv[8][2], hv[8][2];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          lv[r][k] = hv[r][k] = 0u;
+          if (r < CS && k0 + k < bpt) {
+            lv[r][k] = cl.map_shared_rank(hlo, r)[first + k0 + k];
+            hv[r][k] = cl.map_shared_rank(hhi, r)[first + k0 + k];
+          }
+        }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (k >= k0 && k < k0 + 2)
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+            sl[k] += ((unsigned long long)hv[r][k - k0] << 32) | lv[r][k - k0];
+    }
+  }
+#pragma unroll
+  for (int k = 6; k >= 0; --k)
+    if (k + 1 < bpt) sl[k] += sl[k + 1];
+  unsigned long long incl = sl[0];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  if (lane == 0) wsuf[warp] = incl;
+  __syncthreads();
+  unsigned long long after = incl - sl[0];   // within the slice, digits above this thread's
+  unsigned long long slice = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kToppWarps; ++w2) {
+    const unsigned long long x = wsuf[w2];
+    slice += x;
+    if (w2 > warp) after += x;
+  }
+  if (tid == 0) *slice_tot = slice;
+  cl.sync();   // slice totals published; nobody reads this CTA's histogram any more
+  for (int i = tid; i < NB; i += kToppThreads) hlo[i] = hhi[i] = 0u;
+  unsigned long long tots[8];   // every slice's mass, requested together
+#pragma unroll
+  for (int r = 0; r < 8; ++r) tots[r] = r < CS ? *cl.map_shared_rank(slice_tot, r) : 0ull;
+  unsigned long long total = 0, higher = 0;   // all slices; slices of larger digits
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    total += tots[r];
+    if (r > cr) higher += tots[r];
+  }
+  if (NB == kBins) {   // first step: the target mass (the same in every CTA)
+    if (total == 0) return false;
+    const double tf = ceil((p - kMassEps) * (double)total);
+    unsigned long long T = tf < 1.0 ? 1ull : (unsigned long long)tf;
+    s.T = T > total ? total : T;
+  }
+  if (holder) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k < bpt) {
+        const unsigned long long here = s.A + higher + sl[k] + after;
+        const unsigned long long next =
+            s.A + higher + (k + 1 < bpt ? sl[k + 1] : 0ull) + after;
+        if (here >= s.T && next < s.T)
+          for (int r = 0; r < CS; ++r) {
+            *cl.map_shared_rank(sh_d, r) = first + k;
+            *cl.map_shared_rank(sh_above, r) = next - s.A;
+          }
+      }
+    }
+  }
+  cl.sync();   // the digit is in every CTA's shared memory
+  s.A += *sh_above;
+  s.prefix |= (uint32_t)*sh_d << shift;
+  s.pmask |= dm << shift;
+  return true;
+}
+
 // Shared memory of k_topp<NH, R>: the mass histogram (reused after the
 // search to stage the outputs), then, for mid-sized logit runs, a staging
 // area the logits are copied into while the statistics are merged.
@@ -260,6 +378,9 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   __shared__ unsigned sh_blk[2];
   __shared__ unsigned sh_pre[4];
   __shared__ float redm[kToppWarps][NH], redz[kToppWarps][NH];
+  __shared__ unsigned long long slice_tot;       // cluster: this CTA's digit-slice mass
+  __shared__ float2 mz_own[NH];                  // cluster: this CTA's (max, sum) per head
+  __shared__ float2 mz_all[8][NH];               // cluster: every CTA's (max, sum) per head
 
   int CS = 1, cr = 0;
   if (CLUSTER) {
@@ -331,23 +452,22 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
       }
     cp_async_commit();
   }
+  // statistics records of this CTA's candidates: one 32-candidate span per
+  // thread (a CTA holds at most 512 * 32 candidates = 512 spans)
+  const int sp = cr * (kToppThreads * R / kStatSpan) + tid;
   float2 sv[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h)
-    sv[h] = tid < spans_cap ? st[(int64_t)tid * G + h] : make_float2(-INFINITY, 0.f);
+    sv[h] = (tid < kToppThreads * R / kStatSpan && sp < spans_cap) ? st[(int64_t)sp * G + h]
+                                                                    : make_float2(-INFINITY, 0.f);
   const int C = min(cand ? ncnt * kPage : len, cmax);
   const int nspans = (C + kStatSpan - 1) / kStatSpan;
+  const bool mine = tid < kToppThreads * R / kStatSpan && sp < nspans;
 
   // 1. merge the statistics records into each head's max and 1 / sum 2^(l - max)
-  float mloc[NH];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) mloc[h] = tid < nspans ? sv[h].x : -INFINITY;
-  for (int t = tid + kToppThreads; t < nspans; t += kToppThreads)
-#pragma unroll
-    for (int h = 0; h < NH; ++h) mloc[h] = fmaxf(mloc[h], st[(int64_t)t * G + h].x);
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    const float m = warp_max(mloc[h]);
+    const float m = warp_max(mine ? sv[h].x : -INFINITY);
     if (lane == 0) redm[warp][h] = m;
   }
   __syncthreads();
@@ -358,30 +478,40 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
 #pragma unroll
     for (int w2 = 1; w2 < kToppWarps; ++w2) M[h] = fmaxf(M[h], redm[w2][h]);
   }
-  float zloc[NH];
-#pragma unroll
-  for (int h = 0; h < NH; ++h)
-    zloc[h] = (tid < nspans && sv[h].x != -INFINITY) ? sv[h].y * exp2f(sv[h].x - M[h]) : 0.f;
-  for (int t = tid + kToppThreads; t < nspans; t += kToppThreads)
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      const float2 s2 = st[(int64_t)t * G + h];
-      if (s2.x != -INFINITY) zloc[h] += s2.y * exp2f(s2.x - M[h]);
-    }
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    const float z = warp_sum(zloc[h]);
+    const float z =
+        warp_sum((mine && sv[h].x != -INFINITY) ? sv[h].y * exp2f(sv[h].x - M[h]) : 0.f);
     if (lane == 0) redz[warp][h] = z;
   }
   __syncthreads();
-  float iz[NH];
+  float Z[NH];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    float z = 0.f;
+    Z[h] = 0.f;
 #pragma unroll
-    for (int w2 = 0; w2 < kToppWarps; ++w2) z += redz[w2][h];
-    iz[h] = z > 0.f ? 1.0f / z : 0.f;
+    for (int w2 = 0; w2 < kToppWarps; ++w2) Z[h] += redz[w2][h];
   }
+  if (CLUSTER) {   // combine the CTAs' (max, sum) pairs
+    cg::cluster_group cl = cg::this_cluster();
+    if (tid < NH) mz_own[tid] = make_float2(M[tid], Z[tid]);
+    cl.sync();
+    if (tid < CS * NH) mz_all[tid / NH][tid % NH] = *cl.map_shared_rank(&mz_own[tid % NH], tid / NH);
+    cl.sync();   // also: no CTA reads mz_own again
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float m = -INFINITY;
+      for (int r = 0; r < CS; ++r) m = fmaxf(m, mz_all[r][h].x);
+      float z = 0.f;
+      for (int r = 0; r < CS; ++r)
+        if (mz_all[r][h].x != -INFINITY) z += mz_all[r][h].y * exp2f(mz_all[r][h].x - m);
+      M[h] = m;
+      Z[h] = z;
+    }
+  }
+  float iz[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) iz[h] = Z[h] > 0.f ? 1.0f / Z[h] : 0.f;
 
   // 2. weights (-1 marks an invalid slot)
   if (SH::kMode == 1) {
@@ -419,11 +549,24 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
   bool have = false;
   if (!keep_all) {
     Search s{0u, 0u, 0ull, 0ull};
-    have = digit_step<R, kBinsPerThread, CLUSTER>(w, 18, 0xFFFu, p, CS, hlo, hhi, wsuf, &sh_d,
-                                                 &sh_above, s);
+    if (CLUSTER) {
+      have = digit_step_cluster<R, kBins>(w, 18, 0xFFFu, p, CS, cr, hlo, hhi, wsuf, &slice_tot,
+                                          &sh_d, &sh_above, s);
+      if (have) {
+        digit_step_cluster<R, 512>(w, 9, 0x1FFu, p, CS, cr, hlo, hhi, wsuf, &slice_tot, &sh_d,
+                                   &sh_above, s);
+        digit_step_cluster<R, 512>(w, 0, 0x1FFu, p, CS, cr, hlo, hhi, wsuf, &slice_tot, &sh_d,
+                                   &sh_above, s);
+      }
+    } else {
+      have = digit_step<R, kBinsPerThread, false>(w, 18, 0xFFFu, p, CS, hlo, hhi, wsuf, &sh_d,
+                                                  &sh_above, s);
+      if (have) {
+        digit_step<R, 1, false>(w, 9, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+        digit_step<R, 1, false>(w, 0, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+      }
+    }
     if (have) {
-      digit_step<R, 1, CLUSTER>(w, 9, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
-      digit_step<R, 1, CLUSTER>(w, 0, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
       theta = s.prefix;
       unsigned long long Ft = mass_of(__uint_as_float(theta));
       if (Ft == 0) Ft = 1;
@@ -531,21 +674,29 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
 }
 
 // ---------------------------------------------------------------------------
-int topp_shape(int cmax, int* R, int* CS) {
+int topp_shape(int cmax, int sets, int* R, int* CS) {
   if (cmax <= kToppThreads * 16) {
     *CS = 1;
     *R = cmax <= kToppThreads * 4 ? 4 : (cmax <= kToppThreads * 8 ? 8 : 16);
     return 0;
   }
+  // clusters of 2, 4 or 8 CTAs (a power of two splits the digits into equal
+  // slices for the reduce-scatter) of one CTA per SM: 16 weights per thread,
+  // or 32 when that keeps every cluster of the launch resident at once
+  int best_r = 0, best_cs = 0;
   for (int r = 16; r <= 32; r *= 2) {
-    const int cs = (cmax + kToppThreads * r - 1) / (kToppThreads * r);
-    if (cs <= 8) {
-      *R = r;
-      *CS = cs;
-      return 0;
+    int cs = (cmax + kToppThreads * r - 1) / (kToppThreads * r);
+    cs = cs <= 2 ? 2 : (cs <= 4 ? 4 : (cs <= 8 ? 8 : 16));
+    if (cs > 8) continue;
+    if (best_r == 0 || ((long long)sets * best_cs > kTargetSms && (long long)sets * cs <= kTargetSms)) {
+      best_r = r;
+      best_cs = cs;
     }
   }
-  return -1;
+  if (best_r == 0) return -1;
+  *R = best_r;
+  *CS = best_cs;
+  return 0;
 }
 
 template <int NH, int R>
@@ -597,7 +748,7 @@ cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* 
   const int NH = group_sets ? G : 1;
   const int sets = group_sets ? L.B * L.Hk : L.B * Hq;
   int R = 0, CS = 0;
-  if (topp_shape(cmax, &R, &CS) != 0) return cudaErrorInvalidValue;
+  if (topp_shape(cmax, sets, &R, &CS) != 0) return cudaErrorInvalidValue;
 #define TW_TOPP(NN, RR)                                                                       \
   if (NH == NN && R == RR)                                                                    \
     return launch_topp_t<NN, RR>(sets, CS, L, Hq, G, group_sets, cand, cand_stride, ncand,    \

@@ -47,7 +47,7 @@ cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint
                             int cand_stride, const int32_t* ncand, const uint32_t* row0,
                             int lcap, int cmax, float* logits, float2* stats, cudaStream_t st,
                             int num_sms, bool pdl);
-int topp_shape(int cmax, int* R, int* CS);
+int topp_shape(int cmax, int sets, int* R, int* CS);
 cudaError_t launch_topp(const Layout& L, int Hq, int group_sets, const int32_t* cand,
                         int cand_stride, const int32_t* ncand, const uint32_t* row0, int lcap,
                         int cmax, const float* logits, const float2* stats, double p,

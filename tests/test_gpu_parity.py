@@ -86,6 +86,9 @@ SMALL = [
     dict(seed=5, B=1, Hq=8, Hk=1, N=2049, paged=False, budget=None, p=0.7, gm=1),
     dict(seed=6, B=4, Hq=4, Hk=2, N=333, paged=True, budget=48, p=0.95, gm=1),
     dict(seed=7, B=2, Hq=4, Hk=2, N=5000, paged=False, budget=4096, p=0.99, gm=1),
+    # more than 8192 candidates per set: top-p over clusters of 2 and 4 CTAs
+    dict(seed=8, B=1, Hq=4, Hk=2, N=12000, paged=False, budget=None, p=0.85, gm=1),
+    dict(seed=9, B=1, Hq=2, Hk=2, N=30000, paged=True, budget=None, p=0.9, gm=0),
 ]
 
 
