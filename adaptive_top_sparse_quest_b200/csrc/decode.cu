@@ -130,15 +130,16 @@ struct DecSmem {
 // cp.async.cg).  The first batch of accumulator rows is requested before the
 // (m, l) pairs, so a set whose records fit one batch costs one round trip.
 template <int NH>
-__device__ void merge_set(DecSmem<NH>& sm, int set, int64_t off, int cnt, int64_t S, int n_ctas,
-                          int Hq, int hq0, int b, const float* part, __half* out, float* lse) {
+__device__ void merge_set(DecSmem<NH>& sm, int set, int64_t c0, int nspan, bool conc, int64_t off,
+                          int cnt, int64_t S, int n_ctas, int Hq, int hq0, int b,
+                          const float* part, __half* out, float* lse) {
   using MS = MergeShape<NH>;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int64_t c0 = ((off + 1) * n_ctas + S - 1) / S - 1;
-  const int64_t c1 = ((off + cnt) * n_ctas + S - 1) / S - 1;
-  const int nrec = (int)(c1 - c0 + 1);
+  // the set's records sit in the slots of CTAs c0 .. c0 + nrec - 1; with the
+  // concatenated split some of those CTAs may have had an empty range
+  const int nrec = conc ? (int)(((off + cnt) * n_ctas + S - 1) / S - 1 - c0 + 1) : nspan;
   auto rec_ptr = [&](int r, int h) { return part + ((c0 + r + set) * NH + h) * kPartStride; };
-  auto valid = [&](int r) { return range_has(c0 + r, S, n_ctas, off, cnt); };
+  auto valid = [&](int r) { return !conc || range_has(c0 + r, S, n_ctas, off, cnt); };
   // stage the accumulator rows of records [r0, r0 + nr); a slot of a record
   // that was never written (an empty range) is copied too but gets weight 0
   auto stage = [&](int r0, int nr) {
@@ -314,13 +315,224 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
       }
     }
   }
+  const float qscale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+
+  // Attention over tokens [lo, hi) of `set` (offsets within the set's list
+  // plus soff), writing this CTA's record to slot (c + set); the set has nrec
+  // records starting at CTA c0 (conc: some of those CTAs may have empty ranges).
+  auto process = [&](int set, int64_t soff, int64_t lo, int64_t hi, int64_t c0, int nrec,
+                     bool conc) {
+    const int scnt = max(0, min(count[set], icap));
+    int b, hk, hq0;
+    set_heads(set, b, hk, hq0);
+    float qf[NH][8];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const uint4 r = *reinterpret_cast<const uint4*>(q + ((int64_t)b * Hq + hq0 + h) * kHeadDim + 8 * l16);
+      h8_to_f8(r, qf[h]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) qf[h][j] *= qscale;
+    }
+    float m[NH], l[NH], acc[NH][8];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
+    }
+    const uint32_t* srows = rows + (int64_t)set * icap;
+    for (int64_t w0 = lo; w0 < hi; w0 += kWin) {
+      const int wn = (int)min((int64_t)kWin, hi - w0);
+      __syncthreads();   // previous window's rows and ring are no longer read
+      for (int i = tid; i < wn; i += kDecThreads) {
+        sm.rows[i] = srows[w0 - soff + i];
+      }
+      __syncthreads();
+      const int nst = (wn + kStageTok - 1) / kStageTok;
+      auto issue = [&](int st) {
+        if (st < nst) {
+          const int slot = st % kStages;
+#pragma unroll
+          for (int x = tid; x < kStageTok * 32; x += kDecThreads) {
+            const int j = x >> 5, part_ = x & 31;
+            const int pos = st * kStageTok + j;
+            const uint32_t r = pos < wn ? sm.rows[pos] : kNoRow;
+            if (r != kNoRow) {
+              const int64_t row = r;
+              const __half* src = (part_ < 16 ? K : V) + row * kHeadDim + (part_ & 15) * 8;
+              cp_async16(&sm.u.kv[slot][j][part_ >> 4][(part_ & 15) * 8], src);
+            }
+          }
+        }
+        cp_async_commit();
+      };
+#pragma unroll
+      for (int st = 0; st < kStages - 1; ++st) issue(st);
+      for (int st = 0; st < nst; ++st) {
+        issue(st + kStages - 1);
+        cp_async_wait<kStages - 1>();
+        __syncthreads();
+        const int slot = st % kStages;
+        float sc[NH][2];
+        bool ok[2];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * hw + jj;
+          const int pos = st * kStageTok + j;
+          ok[jj] = pos < wn && sm.rows[pos] != kNoRow;
+          float kf[8];
+          h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][j][0][8 * l16])
+                          : make_uint4(0u, 0u, 0u, 0u),
+                   kf);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            float s0 = qf[h][0] * kf[0];
+#pragma unroll
+            for (int dd = 1; dd < 8; ++dd) s0 = __fmaf_rn(qf[h][dd], kf[dd], s0);
+            sc[h][jj] = s0;
+          }
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            sc[h][0] += __shfl_xor_sync(hmask, sc[h][0], o, 16);
+            sc[h][1] += __shfl_xor_sync(hmask, sc[h][1], o, 16);
+          }
+        if (ok[0] || ok[1]) {   // uniform across the half-warp
+          float vf[2][8];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj)
+            h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][2 * hw + jj][1][8 * l16])
+                            : make_uint4(0u, 0u, 0u, 0u),
+                     vf[jj]);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            float mb = m[h];
+            if (ok[0]) mb = fmaxf(mb, sc[h][0]);
+            if (ok[1]) mb = fmaxf(mb, sc[h][1]);
+            const float corr = exp2f(m[h] - mb);
+            const float p0 = ok[0] ? exp2f(sc[h][0] - mb) : 0.f;
+            const float p1 = ok[1] ? exp2f(sc[h][1] - mb) : 0.f;
+            l[h] = l[h] * corr + (p0 + p1);
+#pragma unroll
+            for (int dd = 0; dd < 8; ++dd)
+              acc[h][dd] = __fmaf_rn(p1, vf[1][dd], __fmaf_rn(p0, vf[0][dd], acc[h][dd] * corr));
+            m[h] = mb;
+          }
+        }
+        __syncthreads();   // this slot is refilled by a later issue()
+      }
+      cp_async_wait<0>();
+    }
+    // fold the 8 half-warps and write this CTA's record for the set
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      if (l16 == 0) {
+        sm.u.comb.m[hw][h] = m[h];
+        sm.u.comb.l[hw][h] = l[h];
+      }
+      *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16]) =
+          make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+      *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16 + 4]) =
+          make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+    }
+    __syncthreads();
+    float* rec = part + ((int64_t)(c + set) * NH) * kPartStride;
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kDecHW; ++w) M = fmaxf(M, sm.u.comb.m[w][h]);
+      float Ls = 0.f, A = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecHW; ++w) {
+        const float f = sm.u.comb.m[w][h] == -INFINITY ? 0.f : exp2f(sm.u.comb.m[w][h] - M);
+        Ls += sm.u.comb.l[w][h] * f;
+        A += sm.u.comb.acc[w][h][tid] * f;
+      }
+      rec[h * kPartStride + kPartAcc + tid] = A;
+      if (tid == 0) {
+        rec[h * kPartStride] = M;
+        rec[h * kPartStride + 1] = Ls;
+      }
+    }
+    // publish the record; the CTA that completes the set merges it
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int prev = atomicAdd(&done[set], 1);
+      sm.last = (prev == nrec - 1);
+    }
+    __syncthreads();
+    if (sm.last) {
+      __threadfence();
+      merge_set<NH>(sm, set, c0, nrec, conc, soff, scnt, S, n, Hq, hq0, b, part, out, lse);
+      if (tid == 0) done[set] = 0;   // ready for the next call
+    }
+  };
+
+  if ((long long)nsets * 8 <= n) {
+    // Few sets: every set gets whole CTAs, so no CTA's range straddles two
+    // sets (a straddling CTA pays a second row staging and ring ramp-up, and
+    // the set's merge waits for it).  A set with cnt tokens gets
+    // 1 + floor(cnt * (n - E) / S) CTAs, E the number of non-empty sets, so the
+    // shares add up to at most n and no CTA holds more than about S / (n - E).
+    int64_t ne = 0;
+    for (int s = tid; s < nsets; s += kDecThreads) ne += count[s] > 0 && icap > 0 ? 1 : 0;
+    const int64_t E = block_sum_i64(ne, sm.red64);
+    const int64_t np = n - E;
+    if (tid == 0) sm.nlist = -1;
+    int64_t before = 0;   // CTAs given to the sets of earlier chunks
+    for (int base = 0; base < nsets; base += kDecThreads) {
+      const int s = base + tid;
+      const int cnt = s < nsets ? max(0, min(count[s], icap)) : 0;
+      const int ns = cnt > 0 ? 1 + (int)((int64_t)cnt * np / S) : 0;
+      int incl = ns;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      __syncthreads();
+      if (lane == 31) sm.wcnt[warp] = incl;
+      __syncthreads();
+      int wbefore = 0, chunk = 0;
+#pragma unroll
+      for (int i = 0; i < kDecThreads / 32; ++i) {
+        const int v = (int)sm.wcnt[i];
+        if (i < warp) wbefore += v;
+        chunk += v;
+      }
+      const int64_t start = before + wbefore + incl - ns;
+      if (ns > 0 && c >= start && c < start + ns) {
+        sm.nlist = s;
+        sm.list_off[0] = start;
+        sm.list_set[0] = ns;
+      }
+      before += chunk;
+    }
+    __syncthreads();
+    const int set = sm.nlist;
+    if (set >= 0) {
+      const int64_t start = sm.list_off[0];
+      const int ns = sm.list_set[0];
+      const int cnt = max(0, min(count[set], icap));
+      const int64_t j = c - start;
+      process(set, 0, j * cnt / ns, (j + 1) * cnt / ns, start, ns, false);
+    }
+    griddep_launch();
+    return;
+  }
+
+  // Many sets: CTA c takes [c*S/n, (c+1)*S/n) of the concatenated list.
   const int64_t begin = (int64_t)c * S / n, end = (int64_t)(c + 1) * S / n;
   if (begin >= end) {
     griddep_launch();
     return;
   }
-  const float qscale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
-
   int64_t running = 0;
   for (int base = 0; base < nsets && running < end; base += kDecThreads) {
     // offsets of this chunk of sets, and the sets that overlap [begin, end)
@@ -361,164 +573,16 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
       const int set = sm.list_set[li];
       const int64_t soff = sm.list_off[li];
       const int scnt = max(0, min(count[set], icap));
-      const int64_t lo = max(begin, soff), hi = min(end, soff + scnt);
-      int b, hk, hq0;
-      set_heads(set, b, hk, hq0);
-      float qf[NH][8];
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const uint4 r = *reinterpret_cast<const uint4*>(q + ((int64_t)b * Hq + hq0 + h) * kHeadDim + 8 * l16);
-        h8_to_f8(r, qf[h]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) qf[h][j] *= qscale;
+      // the records of the set: CTAs c0..c1, some possibly with empty ranges
+      const int64_t c0 = ((soff + 1) * n + S - 1) / S - 1;
+      const int64_t c1 = ((soff + scnt) * n + S - 1) / S - 1;
+      int nrec = 0;
+      if (S >= n) {
+        nrec = (int)(c1 - c0 + 1);
+      } else {
+        for (int64_t cc = c0; cc <= c1; ++cc) nrec += range_has(cc, S, n, soff, scnt) ? 1 : 0;
       }
-      float m[NH], l[NH], acc[NH][8];
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        m[h] = -INFINITY;
-        l[h] = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[h][j] = 0.f;
-      }
-      const uint32_t* srows = rows + (int64_t)set * icap;
-      for (int64_t w0 = lo; w0 < hi; w0 += kWin) {
-        const int wn = (int)min((int64_t)kWin, hi - w0);
-        __syncthreads();   // previous window's rows and ring are no longer read
-        for (int i = tid; i < wn; i += kDecThreads) {
-          sm.rows[i] = srows[w0 - soff + i];
-        }
-        __syncthreads();
-        const int nst = (wn + kStageTok - 1) / kStageTok;
-        auto issue = [&](int st) {
-          if (st < nst) {
-            const int slot = st % kStages;
-#pragma unroll
-            for (int x = tid; x < kStageTok * 32; x += kDecThreads) {
-              const int j = x >> 5, part_ = x & 31;
-              const int pos = st * kStageTok + j;
-              const uint32_t r = pos < wn ? sm.rows[pos] : kNoRow;
-              if (r != kNoRow) {
-                const int64_t row = r;
-                const __half* src = (part_ < 16 ? K : V) + row * kHeadDim + (part_ & 15) * 8;
-                cp_async16(&sm.u.kv[slot][j][part_ >> 4][(part_ & 15) * 8], src);
-              }
-            }
-          }
-          cp_async_commit();
-        };
-#pragma unroll
-        for (int st = 0; st < kStages - 1; ++st) issue(st);
-        for (int st = 0; st < nst; ++st) {
-          issue(st + kStages - 1);
-          cp_async_wait<kStages - 1>();
-          __syncthreads();
-          const int slot = st % kStages;
-          float sc[NH][2];
-          bool ok[2];
-#pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int j = 2 * hw + jj;
-            const int pos = st * kStageTok + j;
-            ok[jj] = pos < wn && sm.rows[pos] != kNoRow;
-            float kf[8];
-            h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][j][0][8 * l16])
-                            : make_uint4(0u, 0u, 0u, 0u),
-                     kf);
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              float s0 = qf[h][0] * kf[0];
-#pragma unroll
-              for (int dd = 1; dd < 8; ++dd) s0 = __fmaf_rn(qf[h][dd], kf[dd], s0);
-              sc[h][jj] = s0;
-            }
-          }
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              sc[h][0] += __shfl_xor_sync(hmask, sc[h][0], o, 16);
-              sc[h][1] += __shfl_xor_sync(hmask, sc[h][1], o, 16);
-            }
-          if (ok[0] || ok[1]) {   // uniform across the half-warp
-            float vf[2][8];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
-              h8_to_f8(ok[jj] ? *reinterpret_cast<const uint4*>(&sm.u.kv[slot][2 * hw + jj][1][8 * l16])
-                              : make_uint4(0u, 0u, 0u, 0u),
-                       vf[jj]);
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              float mb = m[h];
-              if (ok[0]) mb = fmaxf(mb, sc[h][0]);
-              if (ok[1]) mb = fmaxf(mb, sc[h][1]);
-              const float corr = exp2f(m[h] - mb);
-              const float p0 = ok[0] ? exp2f(sc[h][0] - mb) : 0.f;
-              const float p1 = ok[1] ? exp2f(sc[h][1] - mb) : 0.f;
-              l[h] = l[h] * corr + (p0 + p1);
-#pragma unroll
-              for (int dd = 0; dd < 8; ++dd)
-                acc[h][dd] = __fmaf_rn(p1, vf[1][dd], __fmaf_rn(p0, vf[0][dd], acc[h][dd] * corr));
-              m[h] = mb;
-            }
-          }
-          __syncthreads();   // this slot is refilled by a later issue()
-        }
-        cp_async_wait<0>();
-      }
-      // fold the 8 half-warps and write this CTA's record for the set
-      __syncthreads();
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        if (l16 == 0) {
-          sm.u.comb.m[hw][h] = m[h];
-          sm.u.comb.l[hw][h] = l[h];
-        }
-        *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16]) =
-            make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-        *reinterpret_cast<float4*>(&sm.u.comb.acc[hw][h][8 * l16 + 4]) =
-            make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
-      }
-      __syncthreads();
-      float* rec = part + ((int64_t)(c + set) * NH) * kPartStride;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kDecHW; ++w) M = fmaxf(M, sm.u.comb.m[w][h]);
-        float Ls = 0.f, A = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecHW; ++w) {
-          const float f = sm.u.comb.m[w][h] == -INFINITY ? 0.f : exp2f(sm.u.comb.m[w][h] - M);
-          Ls += sm.u.comb.l[w][h] * f;
-          A += sm.u.comb.acc[w][h][tid] * f;
-        }
-        rec[h * kPartStride + kPartAcc + tid] = A;
-        if (tid == 0) {
-          rec[h * kPartStride] = M;
-          rec[h * kPartStride + 1] = Ls;
-        }
-      }
-      // publish the record; the CTA that completes the set merges it
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) {
-        const int64_t c0 = ((soff + 1) * n + S - 1) / S - 1;
-        const int64_t c1 = ((soff + scnt) * n + S - 1) / S - 1;
-        int nrec = 0;
-        if (S >= n) {
-          nrec = (int)(c1 - c0 + 1);
-        } else {
-          for (int64_t cc = c0; cc <= c1; ++cc) nrec += range_has(cc, S, n, soff, scnt) ? 1 : 0;
-        }
-        const int prev = atomicAdd(&done[set], 1);
-        sm.last = (prev == nrec - 1);
-      }
-      __syncthreads();
-      if (sm.last) {
-        __threadfence();
-        merge_set<NH>(sm, set, soff, scnt, S, n, Hq, hq0, b, part, out, lse);
-        if (tid == 0) done[set] = 0;   // ready for the next call
-      }
+      process(set, soff, max(begin, soff), min(end, soff + scnt), c0, nrec, true);
     }
     __syncthreads();
   }
