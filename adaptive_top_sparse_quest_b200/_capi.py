@@ -40,7 +40,7 @@ class TwStep(ctypes.Structure):
         ("zeros", c_vp), ("meta", c_vp), ("budget_tokens", c_i32), ("p", ctypes.c_double),
         ("group_mode", c_i32), ("cand_pages", c_vp), ("cand_stride", c_i32), ("ncand", c_vp),
         ("idx", c_vp), ("capacity", c_i32), ("count", c_vp), ("out", c_vp), ("lse", c_vp),
-        ("ws", c_vp), ("ws_bytes", c_size),
+        ("ws", c_vp), ("ws_bytes", c_size), ("append_keys", c_i32),
     ]
 
 
@@ -50,6 +50,7 @@ _SIGS = {
     "tw_version": (ctypes.c_int, []),
     "tw_quantize_keys": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_vp, c_vp, c_vp]),
     "tw_page_meta": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_vp]),
+    "tw_append_keys": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_vp, c_vp, c_vp, c_vp]),
     "tw_workspace_size": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_i32,
                                          ctypes.POINTER(c_size)]),
     "tw_select_pages": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_i32, c_vp,

@@ -149,6 +149,17 @@ def page_meta(kv: KVCache, out: Optional[torch.Tensor] = None, stream=None) -> t
     return out
 
 
+def append_keys(kv: KVCache, keys: Int4Keys, meta: Optional[torch.Tensor] = None,
+                stream=None) -> None:
+    """tw_append_keys: quantise the newest token (position seq_lens[b] - 1) of
+    every sequence into `keys` and fold it into `meta` (if given).  The caller
+    writes that token's K / V rows and raises seq_lens first."""
+    lib = _capi.load()
+    s = kv.struct()
+    check(lib.tw_append_keys(ctypes.byref(s), _ptr(keys.codes), _ptr(keys.scales),
+                             _ptr(keys.zeros), _ptr(meta), _stream(stream)), "tw_append_keys")
+
+
 def workspace_bytes(B: int, Hq: int, Hk: int, N: int, capacity: int) -> int:
     lib = _capi.load()
     n = ctypes.c_size_t(0)
@@ -235,12 +246,15 @@ class DecodeStep:
     """Pre-allocated buffers for repeated tw_decode_step calls on one shape.
 
     budget_tokens None (or <= 0) means base = full attention (every token is a
-    candidate); otherwise Quest keeps budget_tokens // 16 pages first."""
+    candidate); otherwise Quest keeps budget_tokens // 16 pages first.
+    append_keys: each call first folds the newest token of every sequence into
+    the int4 cache and the page metadata (tw_append_keys inside the step)."""
 
     def __init__(self, kv: KVCache, keys: Int4Keys, meta: Optional[torch.Tensor], Hq: int,
                  budget_tokens: Optional[int], p: float, group_mode: int = 0,
-                 with_lse: bool = True):
+                 with_lse: bool = True, append_keys: bool = False):
         self.kv, self.keys, self.meta = kv, keys, meta
+        self.append = bool(append_keys)
         self.Hq = Hq
         self.budget = int(budget_tokens) if budget_tokens and budget_tokens > 0 else 0
         self.p = float(p)
@@ -283,6 +297,7 @@ class DecodeStep:
         s.idx, s.capacity, s.count = _ptr(self.idx), self.capacity, _ptr(self.count)
         s.out, s.lse = _ptr(self.out), _ptr(self.lse)
         s.ws, s.ws_bytes = _ptr(self.ws), self.ws.numel()
+        s.append_keys = 1 if self.append else 0
         self._q, self._s = q, s
         return s
 

@@ -226,6 +226,16 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   Marker mk{events, n_events, st};
   cudaError_t e;
   if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  if (s->append_keys) {   // the newest token of every sequence joins the int4 cache and metadata
+    e = tw::launch_append_keys(L, reinterpret_cast<const __half*>(s->kv.k),
+                               const_cast<uint8_t*>(s->codes),
+                               reinterpret_cast<__half*>(const_cast<uint16_t*>(s->scales)),
+                               reinterpret_cast<__half*>(const_cast<uint16_t*>(s->zeros)),
+                               use_select ? reinterpret_cast<__half*>(const_cast<uint16_t*>(s->meta))
+                                          : nullptr,
+                               st, sms, pdl);
+    if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  }
   float* scores = reinterpret_cast<float*>(wsp(s->ws, plan.scores_off));
   // physical rows: the selector writes the candidate pages' first rows, the
   // top-p kernel the kept tokens' rows (without selection the estimate and
@@ -306,6 +316,25 @@ int tw_page_meta(const tw_kv* kv, uint16_t* meta, void* stream) {
   TW_TRY(device_check(&sms));
   tw::launch_page_meta(L, reinterpret_cast<const __half*>(kv->k), reinterpret_cast<__half*>(meta),
                        static_cast<cudaStream_t>(stream), sms);
+  return check_launch();
+}
+
+int tw_append_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                   uint16_t* meta, void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, true, false, &L));
+  if (!codes != !scales || !codes != !zeros) return TW_ERR_INVALID_ARG;
+  if ((codes && (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(zeros, 16))) ||
+      (meta && !aligned(meta, 16)))
+    return TW_ERR_INVALID_ARG;
+  if ((int64_t)L.B * L.N == 0 || (!codes && !meta)) return TW_OK;
+  int sms = 0;
+  TW_TRY(device_check(&sms));
+  const cudaError_t e = tw::launch_append_keys(
+      L, reinterpret_cast<const __half*>(kv->k), codes, reinterpret_cast<__half*>(scales),
+      reinterpret_cast<__half*>(zeros), reinterpret_cast<__half*>(meta),
+      static_cast<cudaStream_t>(stream), sms, false);
+  if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 
@@ -413,7 +442,7 @@ int tw_decode_step(const tw_step* step, void* stream) {
 
 int tw_decode_step_num_kernels(const tw_step* step) {
   if (!step) return -TW_ERR_INVALID_ARG;
-  return step->budget_tokens > 0 ? 5 : 3;
+  return (step->budget_tokens > 0 ? 5 : 3) + (step->append_keys ? 1 : 0);
 }
 
 const char* tw_decode_step_kernel_name(const tw_step* step, int32_t i) {
@@ -421,6 +450,10 @@ const char* tw_decode_step_kernel_name(const tw_step* step, int32_t i) {
                                        "sparse_decode"};
   static const char* no_select[3] = {"estimate", "topp", "sparse_decode"};
   if (!step) return nullptr;
+  if (step->append_keys) {
+    if (i == 0) return "append_keys";
+    --i;
+  }
   if (step->budget_tokens > 0) return (i >= 0 && i < 5) ? with_select[i] : nullptr;
   return (i >= 0 && i < 3) ? no_select[i] : nullptr;
 }

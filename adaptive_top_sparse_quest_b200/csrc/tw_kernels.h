@@ -42,6 +42,9 @@ void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __ha
                           __half* zeros, cudaStream_t st, int num_sms);
 void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream_t st,
                       int num_sms);
+cudaError_t launch_append_keys(const Layout& L, const __half* K, uint8_t* codes, __half* scales,
+                               __half* zeros, __half* meta, cudaStream_t st, int num_sms,
+                               bool pdl);
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
                             const __half* scales, const __half* zeros, const int32_t* cand,
                             int cand_stride, const int32_t* ncand, const uint32_t* row0,

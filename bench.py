@@ -294,7 +294,8 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    from adaptive_top_sparse_quest_b200 import DecodeStep, KVCache, _capi, page_meta, quantize_keys
+    from adaptive_top_sparse_quest_b200 import (DecodeStep, KVCache, _capi, append_keys, page_meta,
+                                                quantize_keys)
     from adaptive_top_sparse_quest_b200 import build as _b
     _b.build()
     _capi.load()
@@ -323,6 +324,17 @@ def main():
     ev[2].record()
     torch.cuda.synchronize()
     build_ms = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]))
+    # incremental append of each sequence's newest token (idempotent at fixed
+    # lengths, so it can be repeated): mean of 20 calls after 3 warm-up calls
+    for _ in range(3):
+        append_keys(kv0, keys0, meta0)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record()
+    for _ in range(20):
+        append_keys(kv0, keys0, meta0)
+    eb.record()
+    torch.cuda.synchronize()
+    append_us = ea.elapsed_time(eb) * 1e3 / 20
 
     steps = []
     for r in range(R):
@@ -470,7 +482,8 @@ def main():
                      "traffic": traffic, "algorithmic_bytes": kb[dom]},
         "cache_build": {
             "quantize_keys_gbs": toks_total * (256 + 80) / (build_ms[0] * 1e-3) / 1e9,
-            "page_meta_gbs": (toks_total * 256 + pages_total * 512) / (build_ms[1] * 1e-3) / 1e9},
+            "page_meta_gbs": (toks_total * 256 + pages_total * 512) / (build_ms[1] * 1e-3) / 1e9,
+            "append_keys_us": append_us},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": q.numel() * q.element_size(),
                 "d2h_bytes_per_step": steps[0].out.numel() * steps[0].out.element_size()},
         "gpu_launches": args.steps * nk,

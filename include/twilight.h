@@ -120,6 +120,23 @@ int tw_quantize_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t
 int tw_page_meta(const tw_kv* kv, uint16_t* meta, void* stream);
 
 /*
+ * Incremental decode append: after the caller has written the newest token's
+ * K (and V) row at position t = seq_lens[b] - 1 of every sequence b and KV
+ * head (and raised seq_lens), quantise that key row into codes / scales /
+ * zeros exactly as tw_quantize_keys does, and fold it into the metadata of its
+ * page (a page whose first row is t holds only t).  The int4 cache supplies
+ * the weight estimate for every cached token (atlas.scime.ai summary,
+ * "Approach"); keeping it current one token per step is this library's
+ * reading of how a decoder maintains it.  If codes / meta were current for the
+ * lengths minus one, the result equals tw_quantize_keys + tw_page_meta for
+ * the new lengths bit for bit.  Sequences with seq_lens[b] == 0 are skipped.
+ * codes, scales and zeros are all NULL or all set (16-byte aligned); meta may
+ * be NULL (metadata not maintained).
+ */
+int tw_append_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                   uint16_t* meta, void* stream);
+
+/*
  * Workspace bytes needed by tw_select_pages / tw_topp_prune / tw_sparse_decode
  * and tw_decode_step for these sizes (the maximum over the calls).
  * capacity: the idx row length that will be passed (>= candidates per set).
@@ -202,9 +219,11 @@ int tw_topp_prune_noalloc(const uint16_t* q, int32_t num_q_heads, const tw_kv* k
                           double p, int32_t group_mode, int32_t* idx, int32_t capacity,
                           int32_t* count, void* stream);
 
-/* One decode step: tw_select_pages (skipped when budget_tokens <= 0, every token
- * is then a candidate) -> tw_topp_prune -> tw_sparse_decode, enqueued back to
- * back on one stream with no host synchronisation. */
+/* One decode step: [tw_append_keys when append_keys != 0] -> tw_select_pages
+ * (skipped when budget_tokens <= 0, every token is then a candidate) ->
+ * tw_topp_prune -> tw_sparse_decode, enqueued back to back on one stream with
+ * no host synchronisation.  With append_keys set, codes / scales / zeros (and
+ * meta when budget_tokens > 0) must be writable: the step updates them first. */
 typedef struct tw_step {
   const uint16_t* q;          /* [B][Hq][128] */
   int32_t num_q_heads;        /* Hq */
@@ -226,6 +245,7 @@ typedef struct tw_step {
   float* lse;                 /* [B][Hq] or NULL */
   void* ws;
   size_t ws_bytes;
+  int32_t append_keys;        /* nonzero: run tw_append_keys on the cache first */
 } tw_step;
 
 int tw_decode_step(const tw_step* step, void* stream);
