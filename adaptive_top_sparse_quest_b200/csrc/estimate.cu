@@ -310,28 +310,26 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
             if (c0 + 8 < Cu) lrow[c0 + 8] = lg[k][hp][1];
           }
         }
-        // (max, sum 2^(l - max)) over this warp's 32 candidates for head he
+        // (max, sum 2^(l - max)) over this warp's 32 candidates for head he:
+        // the max over the 8 lanes (gid) that share t first, then one exp2
+        // per logit against it, then the sum over the same lanes
         float m = -INFINITY;
         if (owner && hv) {
 #pragma unroll
           for (int k = 0; k < kEstTiles; ++k) m = fmaxf(m, fmaxf(lg[k][hp][0], lg[k][hp][1]));
         }
-        float z = 0.f;
-        if (m != -INFINITY) {
 #pragma unroll
-          for (int k = 0; k < kEstTiles; ++k) {
-            if (lg[k][hp][0] != -INFINITY) z += exp2f(lg[k][hp][0] - m);
-            if (lg[k][hp][1] != -INFINITY) z += exp2f(lg[k][hp][1] - m);
+        for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float z = 0.f;
+        if (owner && hv && m != -INFINITY) {
+#pragma unroll
+          for (int k = 0; k < kEstTiles; ++k) {   // exp2(-inf - m) = 0 for masked slots
+            z += exp2f(lg[k][hp][0] - m);
+            z += exp2f(lg[k][hp][1] - m);
           }
         }
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {   // fold the 8 lanes (gid) that share t
-          const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-          const float zo = __shfl_xor_sync(0xffffffffu, z, o);
-          const float mn = fmaxf(m, mo);
-          z = (m == -INFINITY ? 0.f : z * exp2f(m - mn)) + (mo == -INFINITY ? 0.f : zo * exp2f(mo - mn));
-          m = mn;
-        }
+        for (int o = 4; o < 32; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
         if (gid == 0 && owner && hv)
           stats[((int64_t)u * nspan + cw0 / kStatSpan) * G + he] = make_float2(m, z);
       }
