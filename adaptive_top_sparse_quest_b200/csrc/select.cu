@@ -17,7 +17,8 @@
 //
 // k_page_scores is persistent: each CTA owns a contiguous block of
 // (kv unit, 64-page chunk) items and loads item i+1's metadata while scoring
-// item i.  k_page_topk keeps each unit's K_p best pages by a most-significant-
+// item i (k_page_scores_paged does the same over the paged pool's record
+// order, all KV heads of a page at once).  k_page_topk keeps each unit's K_p best pages by a most-significant-
 // digit-first radix select on the ordered score keys (12 bits, then 9 at a
 // time, starting below the bits all of the unit's keys share), then compacts
 // them in page order with one block scan; in the fused decode step it also
@@ -122,6 +123,107 @@ k_page_scores(Layout L, const __half* __restrict__ q, int Hq, const __half* __re
       A.mn[k] = B.mn[k];
       A.mx[k] = B.mx[k];
     }
+  }
+  griddep_launch();
+}
+
+// Paged layout: a pool page stores the metadata records of all KV heads side by
+// side, so an item here is (sequence, ppi pages, a block of hb <= 64 KV heads)
+// with ppi * hb <= 64 records, read as whole runs of hb * 512 B instead of one
+// scattered 512 B record per page.  Record r of an item is page r / hb, head
+// r % hb of the block; a thread's four records (r = half-warp + 16 k) are the
+// same in every item, so their offsets are computed once.  The query rows vary
+// by record and come through the read-only cache.
+struct PagedGeo {
+  int hb, ppi, nhb, chunks;
+};
+
+__device__ __forceinline__ void score_issue_paged(const Layout& L, const __half* meta,
+                                                  const PagedGeo& g, int it, const int (&rp)[4],
+                                                  const int (&rh)[4], int l16, MetaLoad& d,
+                                                  int& b, int& pg0, int& hk0, int& P) {
+  b = it / (g.chunks * g.nhb);
+  const int rest = it % (g.chunks * g.nhb);
+  pg0 = (rest / g.nhb) * g.ppi;
+  hk0 = (rest % g.nhb) * g.hb;
+  P = (L.len(b) + kPage - 1) / kPage;
+#pragma unroll
+  for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
+    d.mn[k] = make_uint4(0u, 0u, 0u, 0u);
+    d.mx[k] = make_uint4(0u, 0u, 0u, 0u);
+    const int pg = pg0 + rp[k], hk = hk0 + rh[k];
+    if (rp[k] < g.ppi && hk < L.Hk && pg < P) {
+      const __half* m = meta + L.meta_index(b, hk, pg) * (2 * kHeadDim) + l16 * 8;
+      d.mn[k] = ld_stream16(m);
+      d.mx[k] = ld_stream16(m + kHeadDim);
+    }
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kScoreThreads)
+k_page_scores_paged(Layout L, const __half* __restrict__ q, int Hq,
+                    const __half* __restrict__ meta, float* __restrict__ scores, PagedGeo g) {
+  const int items = L.B * g.chunks * g.nhb;
+  const int per = (items + gridDim.x - 1) / gridDim.x;
+  const int it0 = blockIdx.x * per, it1 = min(items, it0 + per);
+  if (it0 >= it1) return;
+  const int lane = threadIdx.x & 31, l16 = lane & 15;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const int hw = threadIdx.x >> 4;
+  int rp[kScorePagesPerHalfWarp], rh[kScorePagesPerHalfWarp];
+#pragma unroll
+  for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
+    const int r = hw + 16 * k;
+    rp[k] = r / g.hb;
+    rh[k] = r % g.hb;
+  }
+  griddep_wait();
+  MetaLoad A, B;
+  int bA, pgA, hkA, PA, bB = 0, pgB = 0, hkB = 0, PB = 0;
+  score_issue_paged(L, meta, g, it0, rp, rh, l16, A, bA, pgA, hkA, PA);
+  for (int it = it0; it < it1; ++it) {
+    if (it + 1 < it1) score_issue_paged(L, meta, g, it + 1, rp, rh, l16, B, bB, pgB, hkB, PB);
+#pragma unroll
+    for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
+      const int pg = pgA + rp[k], hk = hkA + rh[k];
+      if (!(rp[k] < g.ppi && hk < L.Hk && pg < PA)) continue;   // uniform across the half-warp
+      const uint32_t wn[4] = {A.mn[k].x, A.mn[k].y, A.mn[k].z, A.mn[k].w};
+      const uint32_t wx[4] = {A.mx[k].x, A.mx[k].y, A.mx[k].z, A.mx[k].w};
+      float mnv[8], mxv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        mnv[j] = h_lo_hi(wn[j >> 1], j & 1);
+        mxv[j] = h_lo_hi(wx[j >> 1], j & 1);
+      }
+      float total = 0.0f;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4*>(
+            q + ((int64_t)bA * Hq + hk * G + gg) * kHeadDim + l16 * 8));
+        const uint32_t wq[4] = {r.x, r.y, r.z, r.w};
+        float qv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qv[j] = h_lo_hi(wq[j >> 1], j & 1);
+        float s = fmaxf(__fmul_rn(qv[0], mnv[0]), __fmul_rn(qv[0], mxv[0]));
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+          s = __fadd_rn(s, fmaxf(__fmul_rn(qv[j], mnv[j]), __fmul_rn(qv[j], mxv[j])));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(hmask, s, o, 16));
+        total = (gg == 0) ? s : __fadd_rn(total, s);
+      }
+      if (l16 == 0) scores[((int64_t)bA * L.Hk + hk) * L.max_pages + pg] = total;
+    }
+#pragma unroll
+    for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
+      A.mn[k] = B.mn[k];
+      A.mx[k] = B.mx[k];
+    }
+    bA = bB;
+    pgA = pgB;
+    hkA = hkB;
+    PA = PB;
   }
   griddep_launch();
 }
@@ -363,9 +465,43 @@ static int score_grid(int num_sms) {
   return num_sms * per_sm;
 }
 
+template <int G>
+static int score_grid_paged(int num_sms) {
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_page_scores_paged<G>, kScoreThreads,
+                                                      0) != cudaSuccess || n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  return num_sms * per_sm;
+}
+
 cudaError_t launch_page_scores(const Layout& L, const __half* q, int Hq, const __half* meta,
                                float* scores, cudaStream_t st, int num_sms, bool pdl) {
   const int G = Hq / L.Hk;
+  if (L.page_table) {
+    PagedGeo g;
+    g.hb = L.Hk < kScorePagesPerItem ? L.Hk : kScorePagesPerItem;
+    g.ppi = kScorePagesPerItem / g.hb;
+    g.nhb = (L.Hk + g.hb - 1) / g.hb;
+    g.chunks = (L.max_pages + g.ppi - 1) / g.ppi;
+    const long long items64 = (long long)L.B * g.chunks * g.nhb;
+    if (items64 > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const int items = (int)items64;
+    switch (G) {
+#define TW_SCP(GG)                                                                          \
+  case GG: {                                                                                \
+    const int grid = items < score_grid_paged<GG>(num_sms) ? items : score_grid_paged<GG>(num_sms); \
+    return launch_k(k_page_scores_paged<GG>, dim3(grid), dim3(kScoreThreads), 0, st, pdl, L, q, \
+                    Hq, meta, scores, g);                                                   \
+  }
+      TW_SCP(1) TW_SCP(2) TW_SCP(4) TW_SCP(8)
+#undef TW_SCP
+    }
+    return cudaErrorInvalidValue;
+  }
   const int items = L.B * L.Hk * ((L.max_pages + kScorePagesPerItem - 1) / kScorePagesPerItem);
   switch (G) {
 #define TW_SC(GG)                                                                           \
