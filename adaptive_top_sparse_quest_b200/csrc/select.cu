@@ -138,22 +138,42 @@ struct PagedGeo {
   int hb, ppi, nhb, chunks;
 };
 
-__device__ __forceinline__ void score_issue_paged(const Layout& L, const __half* meta,
-                                                  const PagedGeo& g, int it, const int (&rp)[4],
-                                                  const int (&rh)[4], int l16, MetaLoad& d,
-                                                  int& b, int& pg0, int& hk0, int& P) {
-  b = it / (g.chunks * g.nhb);
+struct PagedItem {
+  int b, pg0, hk0, P;
+};
+
+__device__ __forceinline__ PagedItem paged_item(const Layout& L, const PagedGeo& g, int it) {
+  PagedItem x;
+  x.b = it / (g.chunks * g.nhb);
   const int rest = it % (g.chunks * g.nhb);
-  pg0 = (rest / g.nhb) * g.ppi;
-  hk0 = (rest % g.nhb) * g.hb;
-  P = (L.len(b) + kPage - 1) / kPage;
+  x.pg0 = (rest / g.nhb) * g.ppi;
+  x.hk0 = (rest % g.nhb) * g.hb;
+  x.P = (L.len(x.b) + kPage - 1) / kPage;
+  return x;
+}
+
+// Pool pages of this thread's four records of an item (loads issued, not waited for).
+__device__ __forceinline__ void paged_pt(const Layout& L, const PagedGeo& g, const PagedItem& x,
+                                         const int (&rp)[4], int (&pt)[4]) {
+#pragma unroll
+  for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
+    const int pg = x.pg0 + rp[k];
+    pt[k] = (rp[k] < g.ppi && pg < x.P) ? L.page_table[(int64_t)x.b * L.max_pages + pg] : 0;
+  }
+}
+
+__device__ __forceinline__ void score_issue_paged(const Layout& L, const __half* meta,
+                                                  const PagedGeo& g, const PagedItem& x,
+                                                  const int (&rp)[4], const int (&rh)[4],
+                                                  const int (&pt)[4], int l16, MetaLoad& d) {
 #pragma unroll
   for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
     d.mn[k] = make_uint4(0u, 0u, 0u, 0u);
     d.mx[k] = make_uint4(0u, 0u, 0u, 0u);
-    const int pg = pg0 + rp[k], hk = hk0 + rh[k];
-    if (rp[k] < g.ppi && hk < L.Hk && pg < P) {
-      const __half* m = meta + L.meta_index(b, hk, pg) * (2 * kHeadDim) + l16 * 8;
+    const int pg = x.pg0 + rp[k], hk = x.hk0 + rh[k];
+    if (rp[k] < g.ppi && hk < L.Hk && pg < x.P) {
+      const int64_t rec = (int64_t)((unsigned)pt[k] < (unsigned)L.pool_pages ? pt[k] : 0) * L.Hk + hk;
+      const __half* m = meta + rec * (2 * kHeadDim) + l16 * 8;
       d.mn[k] = ld_stream16(m);
       d.mx[k] = ld_stream16(m + kHeadDim);
     }
@@ -179,11 +199,30 @@ k_page_scores_paged(Layout L, const __half* __restrict__ q, int Hq,
     rh[k] = r % g.hb;
   }
   griddep_wait();
+  // items it, it+1 and it+2 are in flight as (records in A), (page-table
+  // entries in ptn, records issued into B this iteration), (entries loading)
   MetaLoad A, B;
-  int bA, pgA, hkA, PA, bB = 0, pgB = 0, hkB = 0, PB = 0;
-  score_issue_paged(L, meta, g, it0, rp, rh, l16, A, bA, pgA, hkA, PA);
+  int pt0[4], ptn[4];
+  PagedItem xa = paged_item(L, g, it0), xb = xa;
+  paged_pt(L, g, xa, rp, pt0);
+  score_issue_paged(L, meta, g, xa, rp, rh, pt0, l16, A);
+  if (it0 + 1 < it1) {
+    xb = paged_item(L, g, it0 + 1);
+    paged_pt(L, g, xb, rp, ptn);
+  }
+  int bA = xa.b, pgA = xa.pg0, hkA = xa.hk0, PA = xa.P;
   for (int it = it0; it < it1; ++it) {
-    if (it + 1 < it1) score_issue_paged(L, meta, g, it + 1, rp, rh, l16, B, bB, pgB, hkB, PB);
+    if (it + 1 < it1) {
+      score_issue_paged(L, meta, g, xb, rp, rh, ptn, l16, B);
+      if (it + 2 < it1) {   // the entries are consumed one iteration later
+        const PagedItem xc = paged_item(L, g, it + 2);
+        paged_pt(L, g, xc, rp, ptn);
+        xa = xb;
+        xb = xc;
+      } else {
+        xa = xb;
+      }
+    }
 #pragma unroll
     for (int k = 0; k < kScorePagesPerHalfWarp; ++k) {
       const int pg = pgA + rp[k], hk = hkA + rh[k];
@@ -220,10 +259,10 @@ k_page_scores_paged(Layout L, const __half* __restrict__ q, int Hq,
       A.mn[k] = B.mn[k];
       A.mx[k] = B.mx[k];
     }
-    bA = bB;
-    pgA = pgB;
-    hkA = hkB;
-    PA = PB;
+    bA = xa.b;
+    pgA = xa.pg0;
+    hkA = xa.hk0;
+    PA = xa.P;
   }
   griddep_launch();
 }
