@@ -602,11 +602,11 @@ static int decode_grid(int nsets, int NH) {
 
 template <int NH>
 static cudaError_t dec_prepare() {
-  static cudaError_t done = cudaErrorNotReady;
-  if (done == cudaErrorNotReady)
-    done = cudaFuncSetAttribute(k_sparse_decode<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static std::atomic<int> done[kMaxDevices];
+  return once_per_device(done, [] {
+    return cudaFuncSetAttribute(k_sparse_decode<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)sizeof(DecSmem<NH>));
-  return done;
+  });
 }
 
 size_t decode_part_floats(int B, int Hq, int Hk) {

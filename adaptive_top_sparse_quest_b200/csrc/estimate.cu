@@ -340,11 +340,11 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
 
 template <int G>
 static cudaError_t est_prepare() {
-  static cudaError_t done = cudaErrorNotReady;
-  if (done == cudaErrorNotReady)
-    done = cudaFuncSetAttribute(k_estimate<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static std::atomic<int> done[kMaxDevices];
+  return once_per_device(done, [] {
+    return cudaFuncSetAttribute(k_estimate<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kEstSmemBytes);
-  return done;
+  });
 }
 
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,

@@ -707,14 +707,16 @@ static cudaError_t launch_topp_t(int sets, int CS, const Layout& L, int Hq, int 
                                  int icap, int32_t* count, int32_t* done, cudaStream_t st,
                                  bool pdl) {
   using SH = ToppShape<NH, R>;
-  static cudaError_t prepared = cudaErrorNotReady;
-  if (prepared == cudaErrorNotReady) {
-    prepared = cudaFuncSetAttribute(k_topp<NH, R, false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SH::kBytes);
-    if (prepared == cudaSuccess)
-      prepared = cudaFuncSetAttribute(k_topp<NH, R, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SH::kBytes);
-  }
+  static std::atomic<int> attr_set[kMaxDevices];
+  const cudaError_t prepared = once_per_device(attr_set, [] {
+    cudaError_t e = cudaFuncSetAttribute(k_topp<NH, R, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SH::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_topp<NH, R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SH::kBytes);
+    return e;
+  });
   if (prepared != cudaSuccess) return prepared;
   if (CS == 1)
     return launch_k(k_topp<NH, R, false>, dim3(sets), dim3(kToppThreads), SH::kBytes, st, pdl, L, Hq, G,

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "tw_common.cuh"
@@ -28,6 +29,22 @@ cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
+// Kernel attributes such as the dynamic shared-memory limit are per device:
+// run `set` once on each device the process launches on (a repeated call from
+// a racing thread only sets the same value again).
+constexpr int kMaxDevices = 64;
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<int> (&done)[kMaxDevices], F&& set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return set();
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
 }
 
 constexpr int kEstTile = 256;        // candidates per estimate work item

@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="llama2_mha",
-                    choices=["llama2_mha", "llama3_gqa", "batched_paged", "tiny"])
+                    choices=["llama2_mha", "llama3_gqa", "batched_paged", "sweep", "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
