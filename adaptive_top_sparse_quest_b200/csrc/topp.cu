@@ -99,16 +99,15 @@ struct Search {
   unsigned long long A, T;
 };
 
-// One digit of the search: histogram the masses of the weights inside the
-// current prefix range by the digit (key >> shift) & dm, scan the digits from
-// the top, and fix the digit where the retained mass crosses T.  Each thread
-// owns BPT consecutive digits (BPT * 512 digits in all).  The first step (BPT
-// == 8) also sets T from the total mass, and returns false if that is zero; it
-// is the same in every CTA of a cluster, so all of them leave together.
-// Leaves the histogram zeroed.
-template <int R, int BPT, bool CLUSTER>
+// One digit of the search within one CTA: histogram the masses of the weights
+// inside the current prefix range by the digit (key >> shift) & dm, scan the
+// digits from the top, and fix the digit where the retained mass crosses T.
+// Each thread owns BPT consecutive digits (BPT * 512 digits in all).  The
+// first step (BPT == 8) also sets T from the total mass, and returns false if
+// that is zero.  Leaves the histogram zeroed.
+template <int R, int BPT>
 __device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint32_t dm, double p,
-                                           int CS, uint32_t* hlo, uint32_t* hhi,
+                                           uint32_t* hlo, uint32_t* hhi,
                                            unsigned long long* wsuf, int* sh_d,
                                            unsigned long long* sh_above, Search& s) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -128,32 +127,20 @@ __device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint3
       }
     }
   }
-  if (CLUSTER) cg::this_cluster().sync();
-  else __syncthreads();
+  __syncthreads();
   unsigned long long sl[BPT];   // suffix sums within this thread's digits
+  if (BPT == 8) {
+    const uint4 l0 = reinterpret_cast<const uint4*>(hlo)[2 * tid];
+    const uint4 l1 = reinterpret_cast<const uint4*>(hlo)[2 * tid + 1];
+    const uint4 u0 = reinterpret_cast<const uint4*>(hhi)[2 * tid];
+    const uint4 u1 = reinterpret_cast<const uint4*>(hhi)[2 * tid + 1];
+    const uint32_t lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    const uint32_t uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-  for (int k = 0; k < BPT; ++k) sl[k] = 0;
-  for (int r = 0; r < CS; ++r) {
-    const uint32_t* lo = hlo;
-    const uint32_t* hi = hhi;
-    if (CLUSTER) {
-      cg::cluster_group cl = cg::this_cluster();
-      lo = cl.map_shared_rank(hlo, r);
-      hi = cl.map_shared_rank(hhi, r);
-    }
-    if (BPT == 8) {
-      const uint4 l0 = reinterpret_cast<const uint4*>(lo)[2 * tid];
-      const uint4 l1 = reinterpret_cast<const uint4*>(lo)[2 * tid + 1];
-      const uint4 u0 = reinterpret_cast<const uint4*>(hi)[2 * tid];
-      const uint4 u1 = reinterpret_cast<const uint4*>(hi)[2 * tid + 1];
-      const uint32_t lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-      const uint32_t uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    for (int k = 0; k < BPT; ++k) sl[k] = join64(uv[k], lv[k]);
+  } else {
 #pragma unroll
-      for (int k = 0; k < BPT; ++k) sl[k] += join64(uv[k], lv[k]);
-    } else {
-#pragma unroll
-      for (int k = 0; k < BPT; ++k) sl[k] += join64(hi[BPT * tid + k], lo[BPT * tid + k]);
-    }
+    for (int k = 0; k < BPT; ++k) sl[k] = join64(hhi[BPT * tid + k], hlo[BPT * tid + k]);
   }
 #pragma unroll
   for (int k = BPT - 2; k >= 0; --k) sl[k] += sl[k + 1];
@@ -165,8 +152,7 @@ __device__ __forceinline__ bool digit_step(const float (&w)[R], int shift, uint3
     if (lane + o < 32) incl += t;
   }
   if (lane == 0) wsuf[warp] = incl;
-  if (CLUSTER) cg::this_cluster().sync();   // also: every peer has read this CTA's bins
-  else __syncthreads();
+  __syncthreads();
   unsigned long long after = incl - sl[0];
   unsigned long long grand = 0;
 #pragma unroll
@@ -559,11 +545,10 @@ k_topp(Layout L, int Hq, int G, int group_sets, const int32_t* __restrict__ cand
                                    &sh_above, s);
       }
     } else {
-      have = digit_step<R, kBinsPerThread, false>(w, 18, 0xFFFu, p, CS, hlo, hhi, wsuf, &sh_d,
-                                                  &sh_above, s);
+      have = digit_step<R, kBinsPerThread>(w, 18, 0xFFFu, p, hlo, hhi, wsuf, &sh_d, &sh_above, s);
       if (have) {
-        digit_step<R, 1, false>(w, 9, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
-        digit_step<R, 1, false>(w, 0, 0x1FFu, p, CS, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+        digit_step<R, 1>(w, 9, 0x1FFu, p, hlo, hhi, wsuf, &sh_d, &sh_above, s);
+        digit_step<R, 1>(w, 0, 0x1FFu, p, hlo, hhi, wsuf, &sh_d, &sh_above, s);
       }
     }
     if (have) {
