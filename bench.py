@@ -443,11 +443,10 @@ def main():
     dom_us = kernel_us[dom]
     achieved = kb[dom] / (dom_us * 1e-6) / 1e9
     traffic = None
-    try:
+    try:   # ncu DRAM bytes per launch, valid only for the sources they were taken on
         tr = json.load(open(TRAFFIC_PATH))
-        if tr.get("src_hash") == src_hash() and tr.get("workload") == w.name and \
-                tr.get("kernel") == dom:
-            traffic = tr.get("dram_bytes_per_launch")
+        if tr.get("src_hash") == src_hash() and tr.get("workload") == w.name:
+            traffic = tr.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
     except Exception:
         pass
     clocks = sampler.summary(t_start - 0.05, t_load_end + 0.05) if sampler else None
