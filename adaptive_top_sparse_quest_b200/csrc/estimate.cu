@@ -51,7 +51,7 @@ struct EstStage {
 
 // Where the 16 pages of an item live: first global row and valid rows (0 = none).
 struct EstPages {
-  long long row0[kPagesPerItem];
+  uint32_t row0[kPagesPerItem];   // physical rows fit 32 bits (checked on the host)
   int rows[kPagesPerItem];
 };
 
@@ -136,7 +136,7 @@ __device__ __forceinline__ void est_store(const EstLook& k, int lane, EstPages& 
   if (k.C > 0 && k.page >= 0 && (int64_t)k.page * kPage < k.len)
     rows = min(kPage, k.len - k.page * kPage);
   out.rows[lane] = rows;
-  out.row0[lane] = rows > 0 ? (long long)k.r0 : 0ll;
+  out.row0[lane] = rows > 0 ? k.r0 : 0u;
 }
 
 // All threads: gather item `it` (pages already looked up) into a ring stage.
@@ -149,13 +149,14 @@ __device__ __forceinline__ void est_issue(const EstPages& pg, const uint8_t* cod
     const int x = tid + k * kEstThreads;
     const int c = x >> 2, part = x & 3, p = c >> 4, r = c & 15;
     if (r < pg.rows[p])
-      cp_async16(&st.codes[c][16 * part], codes + (pg.row0[p] + r) * (kHeadDim / 2) + 16 * part);
+      cp_async16(&st.codes[c][16 * part],
+                 codes + (size_t)(pg.row0[p] + r) * (kHeadDim / 2) + 16 * part);
   }
   {   // scales and zeros: one 8-byte row each per thread
     const int c = tid, p = c >> 4, r = c & 15;
     if (r < pg.rows[p]) {
-      cp_async8(&st.scales[c][0], scales + (pg.row0[p] + r) * kGroups);
-      cp_async8(&st.zeros[c][0], zeros + (pg.row0[p] + r) * kGroups);
+      cp_async8(&st.scales[c][0], scales + (size_t)(pg.row0[p] + r) * kGroups);
+      cp_async8(&st.zeros[c][0], zeros + (size_t)(pg.row0[p] + r) * kGroups);
     }
   }
 }
@@ -203,6 +204,9 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
   uint32_t bfr[HP][8][2];                // B fragments: column gid = (head 2hp + gid/4, group gid%4)
   float Qv[HP][2];                       // Q[h][g0], Q[h][g0+1] for the lane's epilogue head
   int staged = -1;
+  int u = it0 / tiles, tile = it0 % tiles;   // item it = (unit u, candidate tile)
+  int b = u / L.Hk, hk = u % L.Hk;
+  int Cu = 0;                                // candidates of unit u
   for (int it = it0; it < it1; ++it) {
     const int j = it - it0, slot = j % kEstStages;
     // refill: gather item j+S-1 into the slot item j-1 used, and look up the
@@ -220,9 +224,16 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
         ahead = est_fetch(L, cand, cand_stride, ncand, row0, cmax, tiles, it + kEstStages + 2,
                           lane);
     }
-    const int u = it / tiles;
-    const int b = u / L.Hk, hk = u % L.Hk;
+    if (it > it0 && ++tile == tiles) {
+      tile = 0;
+      ++u;
+      if (++hk == L.Hk) {
+        hk = 0;
+        ++b;
+      }
+    }
     if (u != staged) {
+      Cu = min(cand ? __ldg(ncand + u) * kPage : L.len(b), cmax);
 #pragma unroll
       for (int hp = 0; hp < HP; ++hp) {
         const int hb = 2 * hp + (gid >> 2);   // head of B column gid
@@ -251,8 +262,7 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
     __syncthreads();
     const EstPages& pgs = sm.pg[j % kPgRing];
     const EstStage& st = sm.st[slot];
-    const int cw0 = (it % tiles) * kEstTile + warp * 32;   // this warp's first candidate
-    const int Cu = min(cand ? __ldg(ncand + u) * kPage : L.len(b), cmax);
+    const int cw0 = tile * kEstTile + warp * 32;   // this warp's first candidate
     float lg[kEstTiles][HP][2];
 #pragma unroll
     for (int k = 0; k < kEstTiles; ++k) {
