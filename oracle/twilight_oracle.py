@@ -48,6 +48,10 @@ notes of this repository):
      arithmetic does instead of by the last bit of a rounded sum.
   R7 sparse attention over the selected fp16 K/V rows, softmax scale
      1/sqrt(128); out = 0 and lse = -inf for an empty selection.
+  R8 the 2-bit key cache of the quantisation ablation (4-bit preferred to
+     2-bit for stable cumulative weights, table of measured effects) is R1
+     with 3 in place of 15: scale = fp16_rn((max - min) / 3), codes 0..3,
+     four per byte, channel 4i + j in bits 2j, 2j + 1 of byte i.
 """
 from __future__ import annotations
 
@@ -67,8 +71,10 @@ __all__ = [
     "dequantize_keys", "page_meta", "quest_page_scores", "select_pages", "candidate_tokens",
     "estimate_logits", "softmax_weights", "group_weights", "topp_select", "sparse_attention",
     "SeqInputs", "sequence_rows", "oracle_unit", "oracle_decode", "int4_cache_bytes_per_token",
-    "kv_cache_bytes_per_token",
+    "key_cache_bytes_per_token", "kv_cache_bytes_per_token", "KEY_BITS", "retained_mass",
 ]
+
+KEY_BITS = (4, 2)   # key-cache widths: 4-bit (R1) and the ablation's 2-bit (R8)
 
 
 # ----------------------------------------------------------------------------- R2
@@ -93,51 +99,67 @@ def fp16_max(x: np.ndarray, axis: int) -> np.ndarray:
     return np.take_along_axis(np.asarray(x, np.float16), i, axis=axis).squeeze(axis)
 
 
-# ----------------------------------------------------------------------------- R1
-def quantize_keys(k: np.ndarray):
-    """4-bit per-token asymmetric key quantisation, group 32 (reading R1).
+# ----------------------------------------------------------------------------- R1, R8
+def _levels(bits: int) -> int:
+    if bits not in KEY_BITS:
+        raise ValueError(f"key cache width must be one of {KEY_BITS}, got {bits}")
+    return (1 << bits) - 1
+
+
+def quantize_keys(k: np.ndarray, bits: int = 4):
+    """Per-token asymmetric key quantisation, group 32 (reading R1; R8 for 2 bits).
 
     The 4-bit key cache used to estimate attention weights: atlas.scime.ai
-    summary, "Approach" and the quantisation ablation row of its table.
+    summary, "Approach"; the 2-bit width is the one its quantisation ablation
+    row compares against (table of measured effects).
 
-    k: fp16 [..., 128].  Returns codes uint8 [..., 64] (channel 2i in the low
-    nibble of byte i, 2i+1 in the high nibble), scales fp16 [..., 4] and zeros
-    fp16 [..., 4].  Per group of 32 channels, in IEEE fp32 round-to-nearest:
+    k: fp16 [..., 128].  Returns codes uint8 [..., 128 * bits / 8], scales fp16
+    [..., 4] and zeros fp16 [..., 4].  With n = 2^bits - 1 (15 or 3), per group
+    of 32 channels, in IEEE fp32 round-to-nearest:
         mn, mx = exact fp16 min / max of the group
-        scale  = fp16_rn( (f32(mx) - f32(mn)) / 15 )
-        code   = clamp( rint_even( (f32(x) - f32(mn)) / f32(scale) ), 0, 15 )
+        scale  = fp16_rn( (f32(mx) - f32(mn)) / n )
+        code   = clamp( rint_even( (f32(x) - f32(mn)) / f32(scale) ), 0, n )
                  (0 when scale == 0)
         zero   = mn
+    Packing: 8 / bits codes per byte, channel (8 / bits) * i + j in bits
+    bits * j .. bits * j + bits - 1 of byte i (4-bit: even channel in the low
+    nibble).
     """
+    n = _levels(bits)
     k = np.asarray(k, dtype=np.float16)
     lead = k.shape[:-1]
     x = k.reshape(lead + (NGROUPS, GROUP))
     mn = fp16_min(x, axis=-1)                                    # [..., 4] fp16
     mx = fp16_max(x, axis=-1)
     d = mx.astype(np.float32) - mn.astype(np.float32)            # fp32 RN
-    scale = (d / np.float32(15.0)).astype(np.float16)            # fp32 RN, then fp16 RN
+    scale = (d / np.float32(n)).astype(np.float16)               # fp32 RN, then fp16 RN
     num = x.astype(np.float32) - mn.astype(np.float32)[..., None]
     sc = scale.astype(np.float32)[..., None]
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = num / sc                                         # fp32 RN
-    code = np.where(sc == 0, np.float32(0), np.clip(np.rint(ratio), 0, 15)).astype(np.uint8)
+    code = np.where(sc == 0, np.float32(0), np.clip(np.rint(ratio), 0, n)).astype(np.uint8)
     code = code.reshape(lead + (HEAD_DIM,))
-    packed = (code[..., 0::2] | (code[..., 1::2] << 4)).astype(np.uint8)
+    per = 8 // bits
+    packed = np.zeros(lead + (HEAD_DIM // per,), dtype=np.uint8)
+    for j in range(per):
+        packed |= (code[..., j::per] << (bits * j)).astype(np.uint8)
     return packed, scale, mn.copy()
 
 
-def unpack_codes(codes: np.ndarray) -> np.ndarray:
-    """uint8 [..., 64] -> int codes [..., 128] (even channel = low nibble)."""
+def unpack_codes(codes: np.ndarray, bits: int = 4) -> np.ndarray:
+    """uint8 [..., 128 * bits / 8] -> int codes [..., 128] (the packing of quantize_keys)."""
+    n = _levels(bits)
+    per = 8 // bits
     codes = np.asarray(codes, dtype=np.uint8)
     out = np.empty(codes.shape[:-1] + (HEAD_DIM,), dtype=np.int64)
-    out[..., 0::2] = codes & 0x0F
-    out[..., 1::2] = codes >> 4
+    for j in range(per):
+        out[..., j::per] = (codes >> (bits * j)) & n
     return out
 
 
-def dequantize_keys(codes, scales, zeros) -> np.ndarray:
+def dequantize_keys(codes, scales, zeros, bits: int = 4) -> np.ndarray:
     """k_hat = zero_g + scale_g * code, in fp64 from the stored fp16 scale and zero."""
-    c = unpack_codes(codes).astype(np.float64)
+    c = unpack_codes(codes, bits).astype(np.float64)
     lead = c.shape[:-1]
     c = c.reshape(lead + (NGROUPS, GROUP))
     s = np.asarray(scales, np.float16).astype(np.float64)[..., None]
@@ -145,10 +167,17 @@ def dequantize_keys(codes, scales, zeros) -> np.ndarray:
     return (z + s * c).reshape(lead + (HEAD_DIM,))
 
 
+def key_cache_bytes_per_token(bits: int = 4, with_scale_zero: bool = True) -> int:
+    """Bytes of the quantised key cache per token per KV head: 128 * bits / 8 B
+    of codes, plus an fp16 scale and an fp16 zero for each of the 4 groups."""
+    _levels(bits)
+    return HEAD_DIM * bits // 8 + (2 * 2 * NGROUPS if with_scale_zero else 0)
+
+
 def int4_cache_bytes_per_token(with_scale_zero: bool = True) -> int:
     """Bytes of the 4-bit key cache per token per KV head: 64 B of codes, plus an
     fp16 scale and an fp16 zero for each of the 4 groups."""
-    return HEAD_DIM // 2 + (2 * 2 * NGROUPS if with_scale_zero else 0)
+    return key_cache_bytes_per_token(4, with_scale_zero)
 
 
 def kv_cache_bytes_per_token() -> int:
@@ -229,12 +258,12 @@ def candidate_tokens(pages: Optional[np.ndarray], length: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- R5, R6
-def estimate_logits(q_group: np.ndarray, codes, scales, zeros) -> np.ndarray:
-    """Estimated attention logits from the 4-bit key cache, fp64:
+def estimate_logits(q_group: np.ndarray, codes, scales, zeros, bits: int = 4) -> np.ndarray:
+    """Estimated attention logits from the quantised key cache, fp64:
         l[i, h] = (q_h . k_hat_i) / sqrt(128),  k_hat = zero + scale * code.
-    (atlas.scime.ai summary, "Approach": weights estimated from INT4 keys.)
-    Returns [C][G]."""
-    khat = dequantize_keys(codes, scales, zeros)                 # [C][128] fp64
+    (atlas.scime.ai summary, "Approach": weights estimated from INT4 keys;
+    `bits` = 2 for the ablation's 2-bit cache.)  Returns [C][G]."""
+    khat = dequantize_keys(codes, scales, zeros, bits)           # [C][128] fp64
     q = np.asarray(q_group, np.float16).astype(np.float64)       # [G][128]
     return (khat @ q.T) / math.sqrt(HEAD_DIM)
 
@@ -299,6 +328,20 @@ def sparse_attention(q: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray):
     return (e @ v_rows) / L, float(m + math.log(L))
 
 
+def retained_mass(q: np.ndarray, k_rows: np.ndarray, selected: np.ndarray) -> float:
+    """Exact attention mass that a selection keeps: the sum over the selected
+    rows of the fp64 softmax of q . k / sqrt(128) over all the given rows (the
+    candidate set).  The cumulative attention weight whose stability the
+    quantisation ablation measures (atlas.scime.ai summary, table of measured
+    effects).  An empty candidate set keeps mass 0."""
+    k_rows = np.asarray(k_rows, np.float16).astype(np.float64)
+    if k_rows.shape[0] == 0:
+        return 0.0
+    s = (k_rows @ np.asarray(q, np.float16).astype(np.float64)) / math.sqrt(HEAD_DIM)
+    e = np.exp(s - s.max())
+    return float(e[np.asarray(selected, np.int64)].sum() / e.sum())
+
+
 # ----------------------------------------------------------------------------- layout
 class SeqInputs:
     """numpy views of one decode-layer input, in either layout.
@@ -333,20 +376,22 @@ def sequence_rows(arr: np.ndarray, page_table, b: int, h: int, length: int) -> n
 
 
 def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: float,
-                group_mode: int, sel_override: Optional[dict] = None) -> dict:
+                group_mode: int, sel_override: Optional[dict] = None,
+                key_bits: int = 4) -> dict:
     """Every result of the decode path for one (sequence, KV head).
 
-    Returns a dict with the int4 cache, page meta, page scores, candidate pages
-    and tokens, fp64 logits, per-set weights / selections / thresholds, and the
-    attention output of each query head of the group.  `sel_override` maps a
-    query head to the selected token list to attend over (used to check the
-    attention stage on another implementation's selection)."""
+    Returns a dict with the quantised key cache (`key_bits` wide), page meta,
+    page scores, candidate pages and tokens, fp64 logits, per-set weights /
+    selections / thresholds, and the attention output of each query head of the
+    group.  `sel_override` maps a query head to the selected token list to
+    attend over (used to check the attention stage on another implementation's
+    selection)."""
     L = int(x.seq_lens[b])
     G = x.Hq // x.Hk
     heads = list(range(hk * G, (hk + 1) * G))
     k_seq = sequence_rows(x.k, x.page_table, b, hk, L)
     v_seq = sequence_rows(x.v, x.page_table, b, hk, L)
-    codes, scales, zeros = quantize_keys(k_seq)
+    codes, scales, zeros = quantize_keys(k_seq, key_bits)
     meta = page_meta(k_seq, L)
     qg = x.q[b, heads]
     res = {"len": L, "codes": codes, "scales": scales, "zeros": zeros, "meta": meta}
@@ -357,7 +402,7 @@ def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: 
         pages = select_pages(scores, budget_tokens)
     toks = candidate_tokens(pages, L)
     res.update(scores=scores, pages=pages, cand_tokens=toks)
-    logits = estimate_logits(qg, codes[toks], scales[toks], zeros[toks])   # [C][G]
+    logits = estimate_logits(qg, codes[toks], scales[toks], zeros[toks], key_bits)   # [C][G]
     res["logits"] = logits
     sets = {}
     if group_mode and G > 1:
@@ -386,8 +431,9 @@ def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: 
 
 
 def oracle_decode(x: SeqInputs, budget_tokens: Optional[int], p: float, group_mode: int,
-                  units=None) -> dict:
+                  units=None, key_bits: int = 4) -> dict:
     """oracle_unit over the given (b, hk) units (default: all)."""
     if units is None:
         units = [(b, h) for b in range(x.B) for h in range(x.Hk)]
-    return {u: oracle_unit(x, u[0], u[1], budget_tokens, p, group_mode) for u in units}
+    return {u: oracle_unit(x, u[0], u[1], budget_tokens, p, group_mode, key_bits=key_bits)
+            for u in units}
