@@ -30,7 +30,7 @@ class TwKv(ctypes.Structure):
         ("k", c_vp), ("v", c_vp), ("batch", c_i32), ("num_kv_heads", c_i32),
         ("max_seq_len", c_i32), ("seq_lens", c_vp), ("page_table", c_vp),
         ("max_pages_per_seq", c_i32), ("num_pool_pages", c_i32), ("page_size", c_i32),
-        ("head_dim", c_i32),
+        ("head_dim", c_i32), ("key_bits", c_i32),
     ]
 
 

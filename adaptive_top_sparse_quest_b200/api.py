@@ -7,8 +7,9 @@ CUDA kernels of libtwilight.so.
 
 Method: "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning"
 (arXiv 2502.02770): Quest page pre-selection, top-p pruning of the candidates'
-attention weights estimated from a 4-bit key cache, exact sparse attention over
-the survivors.
+attention weights estimated from a 4-bit key cache (or the 2-bit cache of its
+quantisation ablation, KVCache.key_bits = 2), exact sparse attention over the
+survivors.
 """
 from __future__ import annotations
 
@@ -43,14 +44,19 @@ def _need(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+KEY_BITS = (4, 2)
+
+
 @dataclasses.dataclass
 class KVCache:
     """fp16 K/V in the contiguous [B][Hk][N][128] layout, or a paged pool
-    [pages][Hk][16][128] with page_table [B][max_pages]."""
+    [pages][Hk][16][128] with page_table [B][max_pages].  key_bits is the width
+    of the quantised key cache that goes with it (4, or 2)."""
     k: torch.Tensor
     v: Optional[torch.Tensor]
     seq_lens: torch.Tensor
     page_table: Optional[torch.Tensor] = None
+    key_bits: int = 4
 
     def __post_init__(self):
         _need(self.k, torch.float16, "k")
@@ -67,6 +73,13 @@ class KVCache:
                 raise ValueError("paged k must be [pages][Hk][16][128]")
         elif self.k.dim() != 4:
             raise ValueError("contiguous k must be [B][Hk][N][128]")
+        if self.key_bits not in KEY_BITS:
+            raise ValueError(f"key_bits must be one of {KEY_BITS}")
+
+    @property
+    def code_bytes(self) -> int:
+        """Bytes of codes per token row: 128 * key_bits / 8."""
+        return HEAD_DIM * self.key_bits // 8
 
     @property
     def paged(self) -> bool:
@@ -101,6 +114,7 @@ class KVCache:
         s.num_pool_pages = int(self.k.shape[0]) if self.paged else 0
         s.page_size = PAGE
         s.head_dim = HEAD_DIM
+        s.key_bits = self.key_bits
         return s
 
     def row_shape(self, last: int):
@@ -115,24 +129,33 @@ class KVCache:
         return (self.B, self.Hk, self.max_pages, 2, HEAD_DIM)
 
     @classmethod
-    def from_workload(cls, w) -> "KVCache":
-        return cls(w.k, w.v, w.seq_lens, w.page_table)
+    def from_workload(cls, w, key_bits: int = 4) -> "KVCache":
+        return cls(w.k, w.v, w.seq_lens, w.page_table, key_bits)
 
 
 @dataclasses.dataclass
 class Int4Keys:
-    codes: torch.Tensor    # uint8  [..][64]
+    """The quantised key cache (4-bit, or 2-bit when its KVCache says so)."""
+    codes: torch.Tensor    # uint8  [..][128 * key_bits / 8]
     scales: torch.Tensor   # fp16   [..][4]
     zeros: torch.Tensor    # fp16   [..][4]
 
 
+def _check_keys(kv: KVCache, keys: Int4Keys) -> None:
+    if tuple(keys.codes.shape) != kv.row_shape(kv.code_bytes):
+        raise ValueError(f"codes must be {kv.row_shape(kv.code_bytes)} for "
+                         f"{kv.key_bits}-bit keys, got {tuple(keys.codes.shape)}")
+
+
 def quantize_keys(kv: KVCache, out: Optional[Int4Keys] = None, stream=None) -> Int4Keys:
-    """4-bit per-token asymmetric key cache (group 32): tw_quantize_keys."""
+    """Per-token asymmetric key cache (group 32, kv.key_bits wide): tw_quantize_keys."""
     lib = _capi.load()
     if out is None:
-        out = Int4Keys(torch.zeros(kv.row_shape(64), dtype=torch.uint8, device=kv.k.device),
-                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=kv.k.device),
-                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=kv.k.device))
+        dev = kv.k.device
+        out = Int4Keys(torch.zeros(kv.row_shape(kv.code_bytes), dtype=torch.uint8, device=dev),
+                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=dev),
+                       torch.zeros(kv.row_shape(4), dtype=torch.float16, device=dev))
+    _check_keys(kv, out)
     s = kv.struct()
     check(lib.tw_quantize_keys(ctypes.byref(s), _ptr(out.codes), _ptr(out.scales),
                                _ptr(out.zeros), _stream(stream)), "tw_quantize_keys")
@@ -155,6 +178,7 @@ def append_keys(kv: KVCache, keys: Int4Keys, meta: Optional[torch.Tensor] = None
     every sequence into `keys` and fold it into `meta` (if given).  The caller
     writes that token's K / V rows and raises seq_lens first."""
     lib = _capi.load()
+    _check_keys(kv, keys)
     s = kv.struct()
     check(lib.tw_append_keys(ctypes.byref(s), _ptr(keys.codes), _ptr(keys.scales),
                              _ptr(keys.zeros), _ptr(meta), _stream(stream)), "tw_append_keys")
@@ -204,6 +228,7 @@ def topp_prune(q: torch.Tensor, kv: KVCache, keys: Int4Keys, cand: Optional[torc
     """Twilight top-p pruning of the candidates: tw_topp_prune -> (idx, count)."""
     lib = _capi.load()
     _need(q, torch.float16, "q")
+    _check_keys(kv, keys)
     Hq = int(q.shape[1])
     stride = int(cand.shape[-1]) if cand is not None else 0
     if capacity is None:
@@ -253,6 +278,7 @@ class DecodeStep:
     def __init__(self, kv: KVCache, keys: Int4Keys, meta: Optional[torch.Tensor], Hq: int,
                  budget_tokens: Optional[int], p: float, group_mode: int = 0,
                  with_lse: bool = True, append_keys: bool = False):
+        _check_keys(kv, keys)
         self.kv, self.keys, self.meta = kv, keys, meta
         self.append = bool(append_keys)
         self.Hq = Hq
@@ -324,12 +350,12 @@ class DecodeStep:
               "tw_decode_step_profiled")
 
 
-def prepare(w, device=None):
-    """Move a workload to the GPU and build its int4 key cache and page metadata
-    with the library.  Returns (kv, keys, meta, q)."""
+def prepare(w, device=None, key_bits: int = 4):
+    """Move a workload to the GPU and build its quantised key cache (key_bits
+    wide) and page metadata with the library.  Returns (kv, keys, meta, q)."""
     if device is not None:
         w = w.to(device)
-    kv = KVCache.from_workload(w)
+    kv = KVCache.from_workload(w, key_bits)
     keys = quantize_keys(kv)
     meta = page_meta(kv)
     return kv, keys, meta, w.q

@@ -1,11 +1,13 @@
-// Cache-build kernels (prefill time, once per token): the 4-bit key cache and
-// the Quest page metadata.
+// Cache-build kernels (prefill time, once per token): the quantised key cache
+// and the Quest page metadata.
 //
-// 4-bit key cache: Twilight estimates attention weights from INT4 keys
+// Key cache: Twilight estimates attention weights from INT4 keys
 // (atlas.scime.ai summary of "Twilight: Adaptive Attention Sparsity with
-// Hierarchical Top-p Pruning", "Approach"; 4-bit preferred to 2-bit in its
-// table of measured effects).  Quest page metadata: per-page channel-wise key
-// min / max, the layout Quest's page selection works on ("Surprising findings").
+// Hierarchical Top-p Pruning", "Approach"); the 2-bit width its quantisation
+// ablation compares against (table of measured effects) is built by the same
+// kernels with 3 levels instead of 15.  Quest page metadata: per-page
+// channel-wise key min / max, the layout Quest's page selection works on
+// ("Surprising findings").
 //
 // Both kernels stream K once with 16-byte loads; one half-warp owns one token
 // row (or one page), lane l owns channels 8l..8l+7, so a group of 32 channels
@@ -18,13 +20,19 @@
 namespace tw {
 
 // Quantise one token row held by a half-warp (lane l16 holds channels
-// 8 l16 .. 8 l16 + 7 in `raw`) and store its codes, scales and zeros at `row`.
-// Every value is a fixed sequence of IEEE round-to-nearest operations, so it
-// is bit-exact with the CPU definition.
+// 8 l16 .. 8 l16 + 7 in `raw`) to BITS-bit codes (levels 0 .. 2^BITS - 1) and
+// store its codes, scales and zeros at `row`.  Every value is a fixed sequence
+// of IEEE round-to-nearest operations, so it is bit-exact with the CPU
+// definition.  Code j of the lane sits at bits BITS * j of its 4 (BITS = 4) or
+// 2 (BITS = 2) bytes: channel c at bits BITS * (c % (8 / BITS)) of byte
+// c / (8 / BITS).
+template <int BITS>
 __device__ __forceinline__ void quantize_row(const uint4 raw, int64_t row, int lane,
                                              unsigned hmask, uint8_t* __restrict__ codes,
                                              __half* __restrict__ scales,
                                              __half* __restrict__ zeros) {
+  static_assert(BITS == 4 || BITS == 2, "key-cache width");
+  constexpr int kLevels = (1 << BITS) - 1;
   const int l16 = lane & 15;
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   int kmin = 0x7FFFFFFF, kmax = -0x7FFFFFFF - 1;
@@ -43,7 +51,7 @@ __device__ __forceinline__ void quantize_row(const uint4 raw, int64_t row, int l
   const uint32_t mx_bits = h_from_key(kmax);
   const float mnf = __half2float(__ushort_as_half((unsigned short)mn_bits));
   const float mxf = __half2float(__ushort_as_half((unsigned short)mx_bits));
-  const float s32 = __fdiv_rn(__fsub_rn(mxf, mnf), 15.0f);
+  const float s32 = __fdiv_rn(__fsub_rn(mxf, mnf), (float)kLevels);
   const __half sc = __float2half_rn(s32);
   const float scf = __half2float(sc);
   uint32_t packed = 0;
@@ -54,11 +62,14 @@ __device__ __forceinline__ void quantize_row(const uint4 raw, int64_t row, int l
     int c = 0;
     if (scf != 0.0f) {
       c = __float2int_rn(__fdiv_rn(__fsub_rn(x, mnf), scf));
-      c = min(max(c, 0), 15);
+      c = min(max(c, 0), kLevels);
     }
-    packed |= (uint32_t)c << (4 * j);
+    packed |= (uint32_t)c << (BITS * j);
   }
-  *reinterpret_cast<uint32_t*>(codes + row * (kHeadDim / 2) + l16 * 4) = packed;
+  if (BITS == 4)
+    *reinterpret_cast<uint32_t*>(codes + row * (kHeadDim / 2) + l16 * 4) = packed;
+  else
+    *reinterpret_cast<uint16_t*>(codes + row * (kHeadDim / 4) + l16 * 2) = (uint16_t)packed;
   // gather the 4 groups' scale / zero to lane 0 of the half-warp: one 8-byte store each
   const uint32_t sc_bits = __half_as_ushort(sc);
   const int base = lane & 16;
@@ -76,6 +87,7 @@ __device__ __forceinline__ void quantize_row(const uint4 raw, int64_t row, int l
   }
 }
 
+template <int BITS>
 __global__ void __launch_bounds__(256)
 k_quantize_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ codes,
                 __half* __restrict__ scales, __half* __restrict__ zeros) {
@@ -92,8 +104,8 @@ k_quantize_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ co
     const int b = (int)(bh / L.Hk);
     if (t >= L.len(b)) continue;  // uniform across the half-warp
     const int64_t row = L.row(b, h, t);
-    quantize_row(ld_stream16(K + row * kHeadDim + l16 * 8), row, lane, hmask, codes, scales,
-                 zeros);
+    quantize_row<BITS>(ld_stream16(K + row * kHeadDim + l16 * 8), row, lane, hmask, codes,
+                       scales, zeros);
   }
 }
 
@@ -103,6 +115,7 @@ k_quantize_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ co
 // current for the lengths minus one, the result equals a rebuild for the new
 // lengths bit for bit: quantisation is per row, and exact fp16 min / max of
 // a page's valid rows may be taken one row at a time.
+template <int BITS>
 __global__ void __launch_bounds__(256)
 k_append_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ codes,
               __half* __restrict__ scales, __half* __restrict__ zeros, __half* __restrict__ meta) {
@@ -120,7 +133,7 @@ k_append_keys(Layout L, const __half* __restrict__ K, uint8_t* __restrict__ code
     if (t < 0) continue;  // uniform across the half-warp
     const int64_t row = L.row(b, h, t);
     const uint4 raw = *reinterpret_cast<const uint4*>(K + row * kHeadDim + l16 * 8);
-    if (codes) quantize_row(raw, row, lane, hmask, codes, scales, zeros);
+    if (codes) quantize_row<BITS>(raw, row, lane, hmask, codes, scales, zeros);
     if (meta) {
       __half* dst = meta + L.meta_index(b, h, t / kPage) * (2 * kHeadDim) + l16 * 8;
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -210,7 +223,10 @@ void launch_quantize_keys(const Layout& L, const __half* K, uint8_t* codes, __ha
   const int64_t want = (rows + 15) / 16;
   const int64_t cap_blocks = (int64_t)num_sms * 8;
   const int blocks = (int)(want < 1 ? 1 : (want < cap_blocks ? want : cap_blocks));
-  k_quantize_keys<<<blocks, 256, 0, st>>>(L, K, codes, scales, zeros);
+  if (L.kbits == 2)
+    k_quantize_keys<2><<<blocks, 256, 0, st>>>(L, K, codes, scales, zeros);
+  else
+    k_quantize_keys<4><<<blocks, 256, 0, st>>>(L, K, codes, scales, zeros);
 }
 
 cudaError_t launch_append_keys(const Layout& L, const __half* K, uint8_t* codes, __half* scales,
@@ -220,8 +236,8 @@ cudaError_t launch_append_keys(const Layout& L, const __half* K, uint8_t* codes,
   const int64_t want = (units + 15) / 16;
   const int64_t cap_blocks = (int64_t)num_sms * 8;
   const int blocks = (int)(want < 1 ? 1 : (want < cap_blocks ? want : cap_blocks));
-  return launch_k(k_append_keys, dim3(blocks), dim3(256), 0, st, pdl, L, K, codes, scales, zeros,
-                  meta);
+  return launch_k(L.kbits == 2 ? k_append_keys<2> : k_append_keys<4>, dim3(blocks), dim3(256), 0,
+                  st, pdl, L, K, codes, scales, zeros, meta);
 }
 
 void launch_page_meta(const Layout& L, const __half* K, __half* meta, cudaStream_t st,

@@ -51,6 +51,7 @@ int check_kv(const tw_kv* kv, bool need_k, bool need_v, tw::Layout* L) {
   if (!kv) return TW_ERR_INVALID_ARG;
   if (kv->head_dim != tw::kHeadDim || kv->page_size != tw::kPage) return TW_ERR_UNSUPPORTED;
   if (kv->batch < 0 || kv->num_kv_heads < 1 || kv->max_seq_len < 0) return TW_ERR_INVALID_ARG;
+  if (kv->key_bits != 0 && kv->key_bits != 4 && kv->key_bits != 2) return TW_ERR_UNSUPPORTED;
   if (need_k && (!kv->k || !aligned(kv->k, 16))) return TW_ERR_INVALID_ARG;
   if (need_v && (!kv->v || !aligned(kv->v, 16))) return TW_ERR_INVALID_ARG;
   if (kv->seq_lens && !aligned(kv->seq_lens, 4)) return TW_ERR_INVALID_ARG;
@@ -70,6 +71,7 @@ int check_kv(const tw_kv* kv, bool need_k, bool need_v, tw::Layout* L) {
   L->page_table = kv->page_table;
   L->max_pages = kv->page_table ? kv->max_pages_per_seq : (kv->max_seq_len + tw::kPage - 1) / tw::kPage;
   L->pool_pages = kv->page_table ? kv->num_pool_pages : 0;
+  L->kbits = kv->key_bits == 2 ? 2 : 4;
   return TW_OK;
 }
 
@@ -289,7 +291,7 @@ const char* tw_status_string(int status) {
 
 int tw_last_cuda_error(void) { return g_last_cuda; }
 
-int tw_version(void) { return 100; }
+int tw_version(void) { return 101; }
 
 int tw_quantize_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
                      void* stream) {

@@ -1,29 +1,32 @@
-// Twilight weight estimation from the 4-bit key cache, with fused softmax
+// Twilight weight estimation from the quantised key cache, with fused softmax
 // statistics ("Twilight: Adaptive Attention Sparsity with Hierarchical Top-p
 // Pruning", atlas.scime.ai summary, "Approach": the candidates' attention
-// weights are estimated from INT4 keys before top-p pruning).
+// weights are estimated from INT4 keys before top-p pruning; the 2-bit cache
+// of its quantisation ablation, table of measured effects, runs through the
+// same kernel).
 //
-// For candidate i, query head h and 32-channel group g with scale s, zero z:
-//   k_hat = z + s * c = (z + 8 s) + s * (c - 8),  c in 0..15
-//   l[i,h] = sum_g ( s_ig * D[i,h,g] + (z_ig + 8 s_ig) * Q[h,g] ) / sqrt(128)
-//   D[i,h,g] = sum_{j in g} (c_ij - 8) * q_hj,   Q[h,g] = sum_{j in g} q_hj
+// For candidate i, query head h and 32-channel group g with scale s, zero z,
+// codes c in 0..n (n = 15 at 4 bits, 3 at 2 bits) and centre o = 8 or 2:
+//   k_hat = z + s * c = (z + o s) + s * (c - o)
+//   l[i,h] = sum_g ( s_ig * D[i,h,g] + (z_ig + o s_ig) * Q[h,g] ) / sqrt(128)
+//   D[i,h,g] = sum_{j in g} (c_ij - o) * q_hj,   Q[h,g] = sum_{j in g} q_hj
 // The D terms are a small dense contraction, run on the tensor cores with
-// mma.sync m16n8k16 (fp16 operands, fp32 accumulation): (c - 8) and the fp16
+// mma.sync m16n8k16 (fp16 operands, fp32 accumulation): (c - o) and the fp16
 // queries are exact in fp16 and their products exact in fp32.  M = 16
 // candidates, N = 8 columns = (head, group) pairs of two heads, K = 16
 // channels per step; column (h, g) keeps only group g's channels of q_h, so
 // after 8 K-steps every column holds one D[*,h,g] and the per-group scales are
 // applied in the fp32 epilogue, where one xor-shuffle adds the lane pair that
 // holds the other two groups.  The K order is permuted so that lane (gid, t)
-// feeds exactly the 16 B of codes of candidates gid and gid+8, group t, it
-// reads: each code pair becomes a half2 A-fragment with one shift, one LOP3
-// (nibbles -> 0x6400|c, i.e. 1024 + c) and one half2 subtract of 1032.
-// Logits are kept in log2 units (log2(e) folded into the 1/sqrt(128) factor),
-// so the statistics and the top-p kernel use exp2.
+// feeds exactly the codes of candidates gid and gid+8, group t, it reads
+// (16 B at 4 bits, 8 B at 2 bits): each code pair becomes a half2 A-fragment
+// with one shift, one LOP3 (codes -> 0x6400|c, i.e. 1024 + c) and one half2
+// subtract of 1024 + o.  Logits are kept in log2 units (log2(e) folded into
+// the 1/sqrt(128) factor), so the statistics and the top-p kernel use exp2.
 //
 // Data path.  Persistent CTAs (two per SM) each own a contiguous block of
-// work items (kv unit, 16 candidate pages = 256 candidates: 16 KB of codes +
-// 2 KB of scales + 2 KB of zeros).  A 4-stage shared-memory ring is filled
+// work items (kv unit, 16 candidate pages = 256 candidates: 16 KB of codes at
+// 4 bits or 8 KB at 2 bits, + 2 KB of scales + 2 KB of zeros).  A 4-stage shared-memory ring is filled
 // with cp.async by all threads (16-byte chunks of codes, 8-byte rows of
 // scales and zeros) three items ahead.  A page's rows are located from the
 // candidate list and a list of first physical rows written by the selector
@@ -43,8 +46,28 @@ constexpr int kEstTiles = 2;                             // MMA tiles of 16 cand
 constexpr int kPagesPerItem = kEstTile / kPage;          // 16
 constexpr float kL2Scale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
 
+// Key-cache width: bytes of codes per row, the centre o subtracted from the
+// codes, and the channel that feeds MMA k-slot pair j (0: k = 2t, 2t+1; 1:
+// k = 2t+8, 2t+9), element hi of the pair, at K-step s, as an offset in the
+// lane's group.  4 bits: the word s / 2 of the lane's 16 B holds channels
+// 8 (s / 2) + 0..7, and nib_pair takes nibbles (e, e + 4).  2 bits: the word
+// s / 4 of the lane's 8 B holds channels 16 (s / 4) + 0..15, and crumb_pair
+// takes crumbs (m, m + 8).
+template <int BITS>
+struct KeyWidth {
+  static_assert(BITS == 4 || BITS == 2, "key-cache width");
+  static constexpr int kRowBytes = kHeadDim * BITS / 8;
+  static constexpr int kLaneBytes = kGroup * BITS / 8;   // one group of one candidate
+  static constexpr float kCentre = BITS == 4 ? 8.f : 2.f;
+  __device__ static constexpr int chan(int s, int j, int hi) {
+    return BITS == 4 ? 8 * (s >> 1) + 2 * (s & 1) + j + 4 * hi
+                     : 16 * (s >> 2) + 2 * (s & 3) + j + 8 * hi;
+  }
+};
+
+template <int BITS>
 struct EstStage {
-  uint8_t codes[kEstTile][kHeadDim / 2];
+  uint8_t codes[kEstTile][KeyWidth<BITS>::kRowBytes];
   __half scales[kEstTile][kGroups];
   __half zeros[kEstTile][kGroups];
 };
@@ -55,12 +78,11 @@ struct EstPages {
   int rows[kPagesPerItem];
 };
 
+template <int BITS>
 struct EstSmem {
-  EstStage st[kEstStages];
+  EstStage<BITS> st[kEstStages];
   EstPages pg[kEstStages + 2];   // items j .. j+S+1 around iteration j
 };
-
-constexpr size_t kEstSmemBytes = sizeof(EstSmem);
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -97,6 +119,22 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t W, int e) {
   uint32_t r;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64086408u));   // minus 1032
   return r;
+}
+
+// 2-bit codes m and m+8 of W as the half2 (c_m - 2, c_{m+8} - 2), exact.
+__device__ __forceinline__ uint32_t crumb_pair(uint32_t W, int m) {
+  uint32_t x = ((W >> (2 * m)) & 0x00030003u) | 0x64006400u;   // (1024 + c) as fp16
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64026402u));   // minus 1026
+  return r;
+}
+
+// A-fragment half2 of k-slot pair j at K-step s from the lane's codes of one
+// candidate (4 words at 4 bits, 2 at 2 bits): channels chan(s, j, 0 / 1).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_pair(const uint32_t* W, int s, int j) {
+  if (BITS == 4) return nib_pair(W[s >> 1], 2 * (s & 1) + j);
+  return crumb_pair(W[s >> 2], 2 * (s & 3) + j);
 }
 
 __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
@@ -140,17 +178,20 @@ __device__ __forceinline__ void est_store(const EstLook& k, int lane, EstPages& 
 }
 
 // All threads: gather item `it` (pages already looked up) into a ring stage.
+template <int BITS>
 __device__ __forceinline__ void est_issue(const EstPages& pg, const uint8_t* codes,
                                           const __half* scales, const __half* zeros,
-                                          EstStage& st) {
+                                          EstStage<BITS>& st) {
+  constexpr int kRowBytes = KeyWidth<BITS>::kRowBytes;
+  constexpr int kChunks = kRowBytes / 16;   // 16-byte chunks per row: 4 or 2
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {   // codes: 1024 chunks of 16 B
+  for (int k = 0; k < kChunks; ++k) {   // codes: 256 rows x kChunks chunks of 16 B
     const int x = tid + k * kEstThreads;
-    const int c = x >> 2, part = x & 3, p = c >> 4, r = c & 15;
+    const int c = x / kChunks, part = x % kChunks, p = c >> 4, r = c & 15;
     if (r < pg.rows[p])
       cp_async16(&st.codes[c][16 * part],
-                 codes + (size_t)(pg.row0[p] + r) * (kHeadDim / 2) + 16 * part);
+                 codes + (size_t)(pg.row0[p] + r) * kRowBytes + 16 * part);
   }
   {   // scales and zeros: one 8-byte row each per thread
     const int c = tid, p = c >> 4, r = c & 15;
@@ -161,7 +202,7 @@ __device__ __forceinline__ void est_issue(const EstPages& pg, const uint8_t* cod
   }
 }
 
-template <int G>
+template <int G, int BITS>
 __global__ void __launch_bounds__(kEstThreads, 2)
 k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __restrict__ codes,
            const __half* __restrict__ scales, const __half* __restrict__ zeros,
@@ -169,8 +210,9 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
            const uint32_t* __restrict__ row0, int lcap, int cmax, float* __restrict__ logits,
            float2* __restrict__ stats) {
   constexpr int HP = (G + 1) / 2;   // head pairs: one MMA N-block of 8 (head, group) columns each
+  using KW = KeyWidth<BITS>;
   extern __shared__ __align__(128) unsigned char est_smem_raw[];
-  EstSmem& sm = *reinterpret_cast<EstSmem*>(est_smem_raw);
+  EstSmem<BITS>& sm = *reinterpret_cast<EstSmem<BITS>*>(est_smem_raw);
   const int tiles = lcap / kEstTile;
   const int items = L.B * L.Hk * tiles;
   const int per = (items + gridDim.x - 1) / gridDim.x;
@@ -240,11 +282,13 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
         const bool on = ((gid & 3) == t) && hb < G;
         const __half* qb = q + ((int64_t)b * Hq + hk * G + min(hb, G - 1)) * kHeadDim;
         const __half z = __float2half_rn(0.f);
+        const __half* qg = qb + kGroup * t;   // group t of the column's head
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
-          const int e = (s & 1) * 2, base = 32 * t + 8 * (s >> 1);
-          bfr[hp][s][0] = pack_h2(on ? qb[base + e] : z, on ? qb[base + e + 4] : z);
-          bfr[hp][s][1] = pack_h2(on ? qb[base + e + 1] : z, on ? qb[base + e + 5] : z);
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj)
+            bfr[hp][s][jj] = pack_h2(on ? qg[KW::chan(s, jj, 0)] : z,
+                                     on ? qg[KW::chan(s, jj, 1)] : z);
         }
         const int he = 2 * hp + (t >> 1);     // head of this lane's epilogue columns
         const __half* qe = q + ((int64_t)b * Hq + hk * G + min(he, G - 1)) * kHeadDim;
@@ -261,25 +305,33 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
     cp_async_wait<kEstStages - 1>();
     __syncthreads();
     const EstPages& pgs = sm.pg[j % kPgRing];
-    const EstStage& st = sm.st[slot];
+    const EstStage<BITS>& st = sm.st[slot];
     const int cw0 = tile * kEstTile + warp * 32;   // this warp's first candidate
     float lg[kEstTiles][HP][2];
 #pragma unroll
     for (int k = 0; k < kEstTiles; ++k) {
       const int ca = warp * 32 + k * 16 + gid, cb = ca + 8;   // candidates (rows gid, gid+8)
-      const uint4 wa = *reinterpret_cast<const uint4*>(&st.codes[ca][16 * t]);
-      const uint4 wb = *reinterpret_cast<const uint4*>(&st.codes[cb][16 * t]);
+      uint32_t WA[4], WB[4];
+      if (BITS == 4) {
+        const uint4 wa = *reinterpret_cast<const uint4*>(&st.codes[ca][KW::kLaneBytes * t]);
+        const uint4 wb = *reinterpret_cast<const uint4*>(&st.codes[cb][KW::kLaneBytes * t]);
+        WA[0] = wa.x, WA[1] = wa.y, WA[2] = wa.z, WA[3] = wa.w;
+        WB[0] = wb.x, WB[1] = wb.y, WB[2] = wb.z, WB[3] = wb.w;
+      } else {
+        const uint2 wa = *reinterpret_cast<const uint2*>(&st.codes[ca][KW::kLaneBytes * t]);
+        const uint2 wb = *reinterpret_cast<const uint2*>(&st.codes[cb][KW::kLaneBytes * t]);
+        WA[0] = wa.x, WA[1] = wa.y, WA[2] = WA[3] = 0u;
+        WB[0] = wb.x, WB[1] = wb.y, WB[2] = WB[3] = 0u;
+      }
       const bool va = (ca & 15) < pgs.rows[ca >> 4];
       const bool vb = (cb & 15) < pgs.rows[cb >> 4];
       float acc[HP][4];
 #pragma unroll
       for (int hp = 0; hp < HP; ++hp) acc[hp][0] = acc[hp][1] = acc[hp][2] = acc[hp][3] = 0.f;
-      const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const int e = (s & 1) * 2;
-        const uint32_t a[4] = {nib_pair(WA[s >> 1], e), nib_pair(WB[s >> 1], e),
-                               nib_pair(WA[s >> 1], e + 1), nib_pair(WB[s >> 1], e + 1)};
+        const uint32_t a[4] = {code_pair<BITS>(WA, s, 0), code_pair<BITS>(WB, s, 0),
+                               code_pair<BITS>(WA, s, 1), code_pair<BITS>(WB, s, 1)};
 #pragma unroll
         for (int hp = 0; hp < HP; ++hp) mma16816(acc[hp], a, bfr[hp][s][0], bfr[hp][s][1]);
       }
@@ -290,8 +342,10 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
       const __half2 zb = *reinterpret_cast<const __half2*>(&st.zeros[cb][g0]);
       const float2 fsa = __half22float2(sa), fza = __half22float2(za);
       const float2 fsb = __half22float2(sb), fzb = __half22float2(zb);
-      const float zza0 = __fmaf_rn(8.f, fsa.x, fza.x), zza1 = __fmaf_rn(8.f, fsa.y, fza.y);
-      const float zzb0 = __fmaf_rn(8.f, fsb.x, fzb.x), zzb1 = __fmaf_rn(8.f, fsb.y, fzb.y);
+      const float zza0 = __fmaf_rn(KW::kCentre, fsa.x, fza.x);
+      const float zza1 = __fmaf_rn(KW::kCentre, fsa.y, fza.y);
+      const float zzb0 = __fmaf_rn(KW::kCentre, fsb.x, fzb.x);
+      const float zzb1 = __fmaf_rn(KW::kCentre, fsb.y, fzb.y);
 #pragma unroll
       for (int hp = 0; hp < HP; ++hp) {
         float pa = __fmaf_rn(fsa.x, acc[hp][0], zza0 * Qv[hp][0]);
@@ -348,13 +402,26 @@ k_estimate(Layout L, const __half* __restrict__ q, int Hq, const uint8_t* __rest
   griddep_launch();
 }
 
-template <int G>
+template <int G, int BITS>
 static cudaError_t est_prepare() {
   static std::atomic<int> done[kMaxDevices];
   return once_per_device(done, [] {
-    return cudaFuncSetAttribute(k_estimate<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kEstSmemBytes);
+    return cudaFuncSetAttribute(k_estimate<G, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(EstSmem<BITS>));
   });
+}
+
+template <int G, int BITS>
+static cudaError_t est_launch(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
+                              const __half* scales, const __half* zeros, const int32_t* cand,
+                              int cand_stride, const int32_t* ncand, const uint32_t* row0,
+                              int lcap, int cmax, float* logits, float2* stats, cudaStream_t st,
+                              int grid, bool pdl) {
+  const cudaError_t e = est_prepare<G, BITS>();
+  if (e != cudaSuccess) return e;
+  return launch_k(k_estimate<G, BITS>, dim3(grid), dim3(kEstThreads), sizeof(EstSmem<BITS>), st,
+                  pdl, L, q, Hq, codes, scales, zeros, cand, cand_stride, ncand, row0, lcap, cmax,
+                  logits, stats);
 }
 
 cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint8_t* codes,
@@ -365,15 +432,13 @@ cudaError_t launch_estimate(const Layout& L, const __half* q, int Hq, const uint
   const int G = Hq / L.Hk;
   const int items = L.B * L.Hk * (lcap / kEstTile);
   const int grid = items < 2 * num_sms ? items : 2 * num_sms;
+  const bool two = L.kbits == 2;
   switch (G) {
-#define TW_EST(GG)                                                                          \
-  case GG: {                                                                                \
-    const cudaError_t e = est_prepare<GG>();                                                \
-    if (e != cudaSuccess) return e;                                                         \
-    return launch_k(k_estimate<GG>, dim3(grid), dim3(kEstThreads), kEstSmemBytes, st, pdl, \
-                    L, q, Hq, codes, scales, zeros, cand, cand_stride, ncand, row0, lcap,   \
-                    cmax, logits, stats);                                                   \
-  }
+#define TW_EST(GG)                                                                               \
+  case GG:                                                                                       \
+    return (two ? est_launch<GG, 2> : est_launch<GG, 4>)(L, q, Hq, codes, scales, zeros, cand,  \
+                                                         cand_stride, ncand, row0, lcap, cmax,  \
+                                                         logits, stats, st, grid, pdl);
     TW_EST(1) TW_EST(2) TW_EST(4) TW_EST(8)
 #undef TW_EST
   }

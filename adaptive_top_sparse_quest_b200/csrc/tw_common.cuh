@@ -14,13 +14,15 @@ constexpr int kGroup = 32;
 constexpr int kGroups = kHeadDim / kGroup;
 
 // Row addressing of one (sequence, KV head) in either layout.  A "row" is one
-// token of one KV head: 128 fp16 of K or V, 64 B of codes, 4 scales, 4 zeros.
+// token of one KV head: 128 fp16 of K or V, 128 * kbits / 8 B of codes (64 B
+// at 4 bits, 32 B at 2 bits), 4 scales, 4 zeros.
 struct Layout {
   int32_t B, Hk, N;                 // N = max_seq_len
   const int32_t* seq_lens;          // [B] or null
   const int32_t* page_table;        // [B][max_pages] or null
   int32_t max_pages;                // ceil(N / 16)
   int32_t pool_pages;               // paged: pages in the pool
+  int32_t kbits;                    // key-cache width: 4 or 2 (host-side dispatch only)
 
   // Valid length of sequence b, clamped to [0, N] so that a bad length can
   // never address outside the cache.

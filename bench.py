@@ -2,13 +2,15 @@
 """Benchmark of one Twilight decode step per layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+                    [--key-bits 4|2]
 
 A step is one pass of the whole hot path over one decode layer: Quest page
 scores + top-K_p pages -> int4 weight estimate + top-p threshold + index
 compaction -> split-K sparse attention + log-sum-exp merge (the KV cache, its
 4-bit key companion and the page metadata are built beforehand, as at
 prefill).  The default workload is the Llama-2-7B-shaped MHA layer: batch 1, 32
-heads, context 32768, Quest budget 8192 tokens, p = 0.85.
+heads, context 32768, Quest budget 8192 tokens, p = 0.85.  --key-bits 2 runs
+the same step on the 2-bit key cache of the paper's quantisation ablation.
 
 The timed region replays the step over R independent copies of the cache in
 rotation, so the bytes touched between two visits of a copy exceed the 126 MB
@@ -55,6 +57,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--copies", type=int, default=0,
                     help="rotating cache copies (0: enough to exceed L2 several times)")
+    ap.add_argument("--key-bits", type=int, default=4, choices=[4, 2],
+                    help="width of the quantised key cache used for the weight estimate")
     return ap.parse_args()
 
 
@@ -63,10 +67,11 @@ def make_workload(name, device):
     return W.CONFIGS[name](device=device)
 
 
-def workload_config(w, copies=None, copy_bytes=None):
+def workload_config(w, copies=None, copy_bytes=None, key_bits=4):
     c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hk,
          "context": w.N, "paged": w.paged, "budget_tokens": w.budget_tokens, "p": w.p,
-         "group_mode": w.group_mode, "head_dim": 128, "page_size": 16, "int4_group": 32}
+         "group_mode": w.group_mode, "head_dim": 128, "page_size": 16, "key_bits": key_bits,
+         "key_group": 32}
     if copies:
         c["l2"] = (f"inputs larger than L2: {copies} rotating cache copies, "
                    f"{copy_bytes / 1e9:.2f} GB each")
@@ -169,11 +174,12 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def cpu_step_sample(w_cpu, seconds: float, max_units=None):
-    """Time the oracle's decode step (page scores, top-K_p, int4 estimate, top-p,
-    sparse attention) on (b, kv head) units of the workload until `seconds` of
-    CPU work; the int4 cache and page metadata are built first, untimed, as at
-    prefill.  Returns (us per full step, units timed, total units, threads)."""
+def cpu_step_sample(w_cpu, seconds: float, max_units=None, key_bits=4):
+    """Time the oracle's decode step (page scores, top-K_p, quantised-key
+    estimate, top-p, sparse attention) on (b, kv head) units of the workload
+    until `seconds` of CPU work; the key cache and page metadata are built
+    first, untimed, as at prefill.  Returns (us per full step, units timed,
+    total units, threads)."""
     try:
         from threadpoolctl import threadpool_limits
         limiter = threadpool_limits(limits=1)
@@ -195,7 +201,7 @@ def cpu_step_sample(w_cpu, seconds: float, max_units=None):
         L = int(x.seq_lens[b])
         k_seq = O.sequence_rows(x.k, x.page_table, b, hk, L)
         v_seq = O.sequence_rows(x.v, x.page_table, b, hk, L)
-        codes, scales, zeros = O.quantize_keys(k_seq)
+        codes, scales, zeros = O.quantize_keys(k_seq, key_bits)
         meta = O.page_meta(k_seq, L) if w_cpu.budget_tokens else None
         qg = x.q[b, hk * G:(hk + 1) * G]
         t0 = time.perf_counter()
@@ -203,7 +209,7 @@ def cpu_step_sample(w_cpu, seconds: float, max_units=None):
         if w_cpu.budget_tokens:
             pages = O.select_pages(O.quest_page_scores(qg, meta), w_cpu.budget_tokens)
         toks = O.candidate_tokens(pages, L)
-        lg = O.estimate_logits(qg, codes[toks], scales[toks], zeros[toks])
+        lg = O.estimate_logits(qg, codes[toks], scales[toks], zeros[toks], key_bits)
         if w_cpu.group_mode and G > 1:
             sel = O.topp_select(O.group_weights(lg), w_cpu.p)[0]
             sels = [sel] * G
@@ -229,7 +235,7 @@ def run_reference(args):
     w = make_workload(args.config, "cpu")
     per = []
     for i in range(args.warmup + args.steps):
-        us, n, tot, cores = cpu_step_sample(w, 0.0, max_units=1)
+        us, n, tot, cores = cpu_step_sample(w, 0.0, max_units=1, key_bits=args.key_bits)
         if i >= args.warmup:
             per.append(us)
     value = statistics.mean(per)
@@ -238,7 +244,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": value / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, key_bits=args.key_bits),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"each step: 1 random (sequence, KV head) unit of {tot}, "
                                    "scaled by the unit count"},
@@ -249,10 +255,12 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def algorithmic_bytes(w, step):
+def algorithmic_bytes(w, step, key_bits=4):
     """Bytes the step must move (per kernel): page metadata scanned (512 B per
-    page per KV head), int4 candidate keys (80 B per candidate token per KV
-    head) and fp16 K+V rows of the selected tokens (512 B per token per set)."""
+    page per KV head), quantised candidate keys (128 * key_bits / 8 B of codes
+    + 16 B of scales and zeros per candidate token per KV head: 80 B at 4 bits,
+    48 B at 2 bits) and fp16 K+V rows of the selected tokens (512 B per token
+    per set)."""
     import torch
     lens = w.seq_lens.to(torch.int64).cpu()
     pages = (lens + 15) // 16
@@ -271,7 +279,7 @@ def algorithmic_bytes(w, step):
                 cand_tokens += n
     else:
         cand_tokens = int(lens.sum()) * w.Hk
-    int4_b = cand_tokens * 80
+    int4_b = cand_tokens * (128 * key_bits // 8 + 16)
     kept = step.count.to(torch.int64).cpu()
     kv_b = int(kept.sum()) * 512
     return {"page_scores": meta_b, "estimate": int4_b, "sparse_decode": kv_b}, cand_tokens, kept
@@ -301,7 +309,7 @@ def main():
     _capi.load()
 
     w = make_workload(args.config, dev)
-    kv0 = KVCache.from_workload(w)
+    kv0 = KVCache.from_workload(w, args.key_bits)
     keys0 = quantize_keys(kv0)
     meta0 = page_meta(kv0)
     torch.cuda.synchronize()
@@ -342,7 +350,7 @@ def main():
             kv, keys, meta = kv0, keys0, meta0
         else:
             kv = KVCache(w.k.clone(), w.v.clone(), w.seq_lens.clone(),
-                         None if w.page_table is None else w.page_table.clone())
+                         None if w.page_table is None else w.page_table.clone(), args.key_bits)
             keys = type(keys0)(keys0.codes.clone(), keys0.scales.clone(), keys0.zeros.clone())
             meta = meta0.clone()
         steps.append(DecodeStep(kv, keys, meta, w.Hq, w.budget_tokens, w.p, w.group_mode))
@@ -429,12 +437,23 @@ def main():
 
     if sampler:
         sampler.stop()
+    # exact attention mass each query head's selection keeps, through the
+    # library alone: exp(lse over the selection - lse over every candidate),
+    # the second lse from the same step run with p = 1 (outside the timed region)
+    steps[0](q)
+    lse_p = steps[0].lse.double().clone()
+    full = DecodeStep(steps[0].kv, steps[0].keys, steps[0].meta, w.Hq, w.budget_tokens, 1.0,
+                      w.group_mode)
+    full(q)
+    torch.cuda.synchronize()
+    retained = torch.exp(lse_p - full.lse.double()).flatten().cpu()
+    del full
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return 0
 
-    kb, cand_tokens, kept = algorithmic_bytes(w, steps[0])
+    kb, cand_tokens, kept = algorithmic_bytes(w, steps[0], args.key_bits)
     toks_total = int(w.seq_lens.to(torch.int64).sum()) * w.Hk
     pages_total = int(((w.seq_lens.to(torch.int64) + 15) // 16).sum()) * w.Hk
     total_b = sum(kb.values())
@@ -454,7 +473,8 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         w_cpu = w.to("cpu")
-        cpu_us, n_units, tot_units, cores = cpu_step_sample(w_cpu, args.cpu_seconds)
+        cpu_us, n_units, tot_units, cores = cpu_step_sample(w_cpu, args.cpu_seconds,
+                                                            key_bits=args.key_bits)
         cpu = {"value": cpu_us, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n_units} of {tot_units} (sequence, KV head) units of the same "
                          f"workload, single-threaded numpy, scaled to the full step"}
@@ -466,7 +486,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, R, copy_bytes),
+        "config": workload_config(w, R, copy_bytes, args.key_bits),
         "hbm_gbs": total_b / (us_per_step * 1e-6) / 1e9,
         "hbm_frac_of_measured": total_b / (us_per_step * 1e-6) / 1e9 / peak,
         "bytes_per_step": total_b,
@@ -475,6 +495,10 @@ def main():
                         "max": int(kept.max()), "sets": sets,
                         "candidates_per_set": cands_per_set},
         "pruned_frac": 1.0 - float(kept.double().mean()) / max(1.0, cands_per_set),
+        "retained_mass": {"p": w.p, "mean": float(retained.mean()),
+                          "std": float(retained.std()) if retained.numel() > 1 else 0.0,
+                          "min": float(retained.min()), "max": float(retained.max()),
+                          "heads": retained.numel()},
         "kernel_us": kernel_us,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,

@@ -8,7 +8,9 @@
  * top-p (nucleus) thresholding over the candidates' attention weights, which
  * are estimated from a 4-bit key cache, prunes them further; exact attention
  * then runs over the survivors only (atlas.scime.ai summary, "Approach";
- * group-wise budgets under GQA: "Limitations").
+ * group-wise budgets under GQA: "Limitations").  A 2-bit key cache, the width
+ * the quantisation ablation compares 4-bit against (table of measured
+ * effects), is selected with tw_kv.key_bits = 2.
  *
  * Conventions shared by every call
  *   - Every function returns a tw_status (0 = TW_OK).  Host-side argument
@@ -31,12 +33,14 @@
  *   contiguous (page_table == NULL):
  *     K, V        [B][Hk][N][128]
  *     codes (u8)  [B][Hk][N][64]   channel 2i in the low nibble of byte i
+                                 (key_bits 2: [B][Hk][N][32], channel 4i + j in
+                                 bits 2j, 2j + 1 of byte i)
  *     scales      [B][Hk][N][4]    one per group of 32 channels
  *     zeros       [B][Hk][N][4]
  *     meta        [B][Hk][ceil(N/16)][2][128]   row 0 = min, row 1 = max
  *   paged (page_table != NULL), pool page P = page_table[b][pg]:
  *     K, V        [num_pool_pages][Hk][16][128]
- *     codes       [num_pool_pages][Hk][16][64]
+ *     codes       [num_pool_pages][Hk][16][64]   (key_bits 2: [..][32])
  *     scales      [num_pool_pages][Hk][16][4]
  *     zeros       [num_pool_pages][Hk][16][4]
  *     meta        [num_pool_pages][Hk][2][128]
@@ -84,6 +88,8 @@ typedef struct tw_kv {
   int32_t num_pool_pages;     /* pages in the pool (paged only) */
   int32_t page_size;          /* must be 16 */
   int32_t head_dim;           /* must be 128 */
+  int32_t key_bits;           /* width of the quantised key cache: 4 (or 0, read as 4)
+                                 or 2; any other value gives TW_ERR_UNSUPPORTED */
 } tw_kv;
 
 /* Name of a status code (static string). */
@@ -96,14 +102,16 @@ int tw_last_cuda_error(void);
 int tw_version(void);
 
 /*
- * Build the 4-bit key cache (prefill-time, once per token).
+ * Build the quantised key cache (prefill-time, once per token).
  * Source: the 4-bit key cache used to estimate attention weights
  * (atlas.scime.ai summary, "Approach"; 4-bit preferred to 2-bit, table of
  * measured effects; about 1/8 extra KV memory, "Limitations").
- * Per token and group of 32 channels, in IEEE fp32 round-to-nearest:
+ * Per token and group of 32 channels, in IEEE fp32 round-to-nearest, with
+ * n = 15 (kv->key_bits 4) or 3 (kv->key_bits 2):
  *   mn, mx = exact fp16 min / max (totalOrder: -0 < +0)
- *   scale = fp16_rn((mx - mn) / 15),  zero = mn,
- *   code  = clamp(round_half_even((x - mn) / scale), 0, 15), 0 if scale == 0.
+ *   scale = fp16_rn((mx - mn) / n),  zero = mn,
+ *   code  = clamp(round_half_even((x - mn) / scale), 0, n), 0 if scale == 0.
+ * codes are packed as "Layouts" states for the width.
  * Reads kv->k for tokens t < seq_lens[b]; writes codes/scales/zeros at the same
  * positions (other positions are left untouched).  Bit-exact with the CPU
  * definition.
@@ -165,7 +173,8 @@ int tw_select_pages(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
  * Twilight's top-p pruner (atlas.scime.ai summary, "Approach"; group-wise
  * under GQA, "Limitations").  Candidates of (b, KV head) are the valid tokens
  * of its cand_pages (ascending), or every token t < len when cand_pages is NULL
- * (base = full attention).  For each candidate i and query head h:
+ * (base = full attention).  For each candidate i and query head h, with the
+ * codes of the cache width kv->key_bits:
  *   l[i,h] = q_h . (zero + scale * code_i) / sqrt(128)          (fp32)
  *   w_h[i] = exp(l[i,h] - max_i l) / sum_i exp(l[i,h] - max_i l)
  * The set's weight is w_h (per-head sets) or the mean of w_h over the G heads

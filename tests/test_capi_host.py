@@ -68,6 +68,26 @@ def test_kv_descriptor_checks(lib):
     assert lib.tw_page_meta(ctypes.byref(bad), out, None) == _capi.TW_ERR_INVALID_ARG
     # empty batch: nothing to launch, success without a device
     assert lib.tw_quantize_keys(ctypes.byref(_kv(batch=0)), out, out, out, None) == _capi.TW_OK
+    # key-cache width: 0 (read as 4), 4 or 2; anything else is unsupported
+    for bits in (0, 2, 4):
+        assert lib.tw_quantize_keys(ctypes.byref(_kv(batch=0, key_bits=bits)), out, out, out,
+                                    None) == _capi.TW_OK
+    for bits in (1, 3, 8, -4):
+        assert lib.tw_quantize_keys(ctypes.byref(_kv(batch=0, key_bits=bits)), out, out, out,
+                                    None) == _capi.TW_ERR_UNSUPPORTED
+        assert lib.tw_append_keys(ctypes.byref(_kv(batch=0, key_bits=bits)), out, out, out, out,
+                                  None) == _capi.TW_ERR_UNSUPPORTED
+
+
+def test_struct_layout_matches_header():
+    """The ctypes mirror of tw_kv ends with key_bits, after head_dim."""
+    names = [f[0] for f in _capi.TwKv._fields_]
+    assert names[-2:] == ["head_dim", "key_bits"]
+    text = open(_capi.HEADER).read()
+    body = text[text.index("typedef struct tw_kv {"):text.index("} tw_kv;")]
+    import re
+    fields = re.findall(r"\b([a-z_]+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
+    assert fields == names
 
 
 def test_topp_and_select_argument_checks(lib):

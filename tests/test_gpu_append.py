@@ -36,14 +36,14 @@ def _start_lengths(final, steps):
     return start
 
 
-def _check_cache(w, codes, scales, zeros, meta):
+def _check_cache(w, codes, scales, zeros, meta, key_bits=4):
     x = O.SeqInputs.from_workload(w)
     table = x.page_table
     for b in range(w.B):
         L = int(w.seq_lens[b])
         for hk in range(w.Hk):
             ks = O.sequence_rows(x.k, table, b, hk, L)
-            rc, rs, rz = O.quantize_keys(ks)
+            rc, rs, rz = O.quantize_keys(ks, key_bits)
             assert np.array_equal(gpu_rows(codes, table, b, hk, L), rc), (b, hk)
             assert np.array_equal(gpu_rows(scales, table, b, hk, L).view(np.uint16),
                                   rs.view(np.uint16)), (b, hk)
@@ -54,10 +54,12 @@ def _check_cache(w, codes, scales, zeros, meta):
 
 
 CASES = [
-    dict(seed=41, B=4, Hq=4, Hk=2, N=300, paged=False, steps=1),
-    dict(seed=42, B=4, Hq=8, Hk=2, N=400, paged=True, steps=1),
-    dict(seed=43, B=3, Hq=4, Hk=4, N=500, paged=False, steps=37),
-    dict(seed=44, B=5, Hq=8, Hk=1, N=700, paged=True, steps=40),
+    dict(seed=41, B=4, Hq=4, Hk=2, N=300, paged=False, steps=1, bits=4),
+    dict(seed=42, B=4, Hq=8, Hk=2, N=400, paged=True, steps=1, bits=4),
+    dict(seed=43, B=3, Hq=4, Hk=4, N=500, paged=False, steps=37, bits=4),
+    dict(seed=44, B=5, Hq=8, Hk=1, N=700, paged=True, steps=40, bits=4),
+    dict(seed=46, B=4, Hq=4, Hk=2, N=300, paged=False, steps=1, bits=2),
+    dict(seed=47, B=5, Hq=8, Hk=1, N=700, paged=True, steps=40, bits=2),
 ]
 
 
@@ -69,14 +71,14 @@ def test_append_matches_rebuild(c):
     final = [int(x) for x in w.seq_lens]
     start = _start_lengths(final, c["steps"])
     w0 = dataclasses.replace(w, seq_lens=torch.tensor(start, dtype=torch.int32))
-    kv, keys, meta, _ = prepare(w0, "cuda")
+    kv, keys, meta, _ = prepare(w0, "cuda", c["bits"])
     fin = torch.tensor(final, dtype=torch.int32, device="cuda")
     for _ in range(max(f - s for f, s in zip(final, start))):
         torch.minimum(kv.seq_lens + 1, fin, out=kv.seq_lens)
         append_keys(kv, keys, meta)
     torch.cuda.synchronize()
     assert [int(x) for x in kv.seq_lens.cpu()] == final
-    _check_cache(w, np16(keys.codes), np16(keys.scales), np16(keys.zeros), np16(meta))
+    _check_cache(w, np16(keys.codes), np16(keys.scales), np16(keys.zeros), np16(meta), c["bits"])
 
 
 def test_step_with_append_equals_append_then_step():

@@ -29,9 +29,9 @@ def _lib():
     _capi.load()
 
 
-def run_gpu(w, budget, p, gm):
+def run_gpu(w, budget, p, gm, key_bits=4):
     from adaptive_top_sparse_quest_b200 import DecodeStep, prepare
-    kv, keys, meta, q = prepare(w, "cuda")
+    kv, keys, meta, q = prepare(w, "cuda", key_bits)
     step = DecodeStep(kv, keys, meta, w.Hq, budget, p, gm)
     step(q)
     torch.cuda.synchronize()
@@ -41,14 +41,14 @@ def run_gpu(w, budget, p, gm):
                 lse=np16(step.lse), step=step, kv=kv, keys=keys, meta_t=meta, q=q)
 
 
-def check_units(w, g, budget, p, gm, units, check_cache=True):
+def check_units(w, g, budget, p, gm, units, check_cache=True, key_bits=4):
     x = O.SeqInputs.from_workload(w)
     table = x.page_table
     G = w.Hq // w.Hk
     group_sets = gm == 1 or G == 1
     stats = {"near": 0, "cut": 0, "sets": 0, "max_err": 0.0}
     for (b, hk) in units:
-        res = O.oracle_unit(x, b, hk, budget, p, gm)
+        res = O.oracle_unit(x, b, hk, budget, p, gm, key_bits=key_bits)
         L = res["len"]
         if check_cache:
             assert np.array_equal(gpu_rows(g["codes"], table, b, hk, L), res["codes"])
@@ -100,6 +100,55 @@ def test_small_parity(c):
     units = [(b, h) for b in range(w.B) for h in range(w.Hk)]
     st = check_units(w, g, c["budget"], c["p"], c["gm"], units)
     assert st["cut"] <= max(1, st["sets"] // 20)
+
+
+# the 2-bit key cache of the quantisation ablation, through the same path
+SMALL_2BIT = [
+    dict(seed=31, B=2, Hq=2, Hk=2, N=777, paged=False, budget=160, p=0.85, gm=0),
+    dict(seed=32, B=3, Hq=8, Hk=2, N=1000, paged=True, budget=256, p=0.85, gm=1),
+    dict(seed=33, B=2, Hq=8, Hk=1, N=2049, paged=False, budget=None, p=0.7, gm=1),
+    dict(seed=34, B=2, Hq=4, Hk=4, N=1500, paged=True, budget=None, p=0.9, gm=0),
+    dict(seed=35, B=1, Hq=4, Hk=2, N=12000, paged=False, budget=None, p=0.85, gm=1),
+]
+
+
+@pytest.mark.parametrize("c", SMALL_2BIT, ids=lambda c: f"s{c['seed']}")
+def test_small_parity_two_bit_keys(c):
+    w = W.random_small(c["seed"], B=c["B"], Hq=c["Hq"], Hk=c["Hk"], N=c["N"], paged=c["paged"],
+                       budget_tokens=c["budget"], p=c["p"], group_mode=c["gm"])
+    g = run_gpu(w, c["budget"], c["p"], c["gm"], key_bits=2)
+    assert g["codes"].shape[-1] == 32
+    units = [(b, h) for b in range(w.B) for h in range(w.Hk)]
+    st = check_units(w, g, c["budget"], c["p"], c["gm"], units, key_bits=2)
+    assert st["cut"] <= max(1, st["sets"] // 20)
+
+
+@pytest.mark.parametrize("key_bits", [4, 2])
+def test_retained_mass_through_the_library(key_bits):
+    """The exact attention mass a selection keeps, read from the library alone
+    as exp(lse of the selection - lse of all candidates) (the step run again
+    with p = 1), equals the oracle's retained mass of the GPU's own selection."""
+    from adaptive_top_sparse_quest_b200 import DecodeStep
+    w = W.random_small(36, B=2, Hq=8, Hk=2, N=1800, paged=True, budget_tokens=512,
+                       group_mode=1)
+    g = run_gpu(w, 512, 0.85, 1, key_bits)
+    full = DecodeStep(g["kv"], g["keys"], g["meta_t"], w.Hq, 512, 1.0, 1)
+    full(g["q"])
+    torch.cuda.synchronize()
+    lse1 = np16(full.lse)
+    x = O.SeqInputs.from_workload(w)
+    G = w.Hq // w.Hk
+    for b in range(w.B):
+        for hk in range(w.Hk):
+            res = O.oracle_unit(x, b, hk, 512, 0.85, 1, key_bits=key_bits)
+            k_seq = O.sequence_rows(x.k, x.page_table, b, hk, res["len"])
+            s = b * w.Hk + hk
+            toks = g["idx"][s, :int(g["count"][s])]
+            pos = np.searchsorted(res["cand_tokens"], toks)
+            for hq in range(hk * G, (hk + 1) * G):
+                ref = O.retained_mass(x.q[b, hq], k_seq[res["cand_tokens"]], pos)
+                got = math.exp(float(g["lse"][b, hq]) - float(lse1[b, hq]))
+                assert abs(got - ref) <= 5e-4, (b, hq, got, ref)
 
 
 def test_tiny_single_head_full_size():
