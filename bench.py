@@ -464,8 +464,9 @@ def main():
     traffic = None
     try:   # ncu DRAM bytes per launch, valid only for the sources they were taken on
         tr = json.load(open(TRAFFIC_PATH))
+        sect = "kernels" if args.key_bits == 4 else f"kernels_key_bits_{args.key_bits}"
         if tr.get("src_hash") == src_hash() and tr.get("workload") == w.name:
-            traffic = tr.get("kernels", {}).get(dom, {}).get("dram_bytes_per_launch")
+            traffic = tr.get(sect, {}).get(dom, {}).get("dram_bytes_per_launch")
     except Exception:
         pass
     clocks = sampler.summary(t_start - 0.05, t_load_end + 0.05) if sampler else None
