@@ -64,6 +64,7 @@ _SIGS = {
                                              c_vp, c_i32, c_vp, ctypes.c_double, c_i32, c_vp,
                                              c_i32, c_vp, c_vp]),
     "tw_decode_step": (ctypes.c_int, [ctypes.POINTER(TwStep), c_vp]),
+    "tw_decode_step_host": (ctypes.c_int, [ctypes.POINTER(TwStep), c_vp, c_vp, c_vp]),
     "tw_decode_step_num_kernels": (ctypes.c_int, [ctypes.POINTER(TwStep)]),
     "tw_decode_step_kernel_name": (ctypes.c_char_p, [ctypes.POINTER(TwStep), c_i32]),
     "tw_decode_step_profiled": (ctypes.c_int, [ctypes.POINTER(TwStep), ctypes.POINTER(c_vp), c_i32,

@@ -302,6 +302,7 @@ class DecodeStep:
         self.ws = new_workspace(kv.B, Hq, kv.Hk, kv.N, self.capacity, dev)
         self._q = None
         self._s = None
+        self._q_stage = None   # device staging of the query for run_host
 
     def _struct(self, q: torch.Tensor) -> TwStep:
         if self._s is not None and self._q is q:
@@ -332,6 +333,28 @@ class DecodeStep:
         s = self._struct(q)
         check(lib.tw_decode_step(ctypes.byref(s), _stream(stream)), "tw_decode_step")
         return self.out
+
+    def run_host(self, q_host: torch.Tensor, out_host: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        """One step with the query taken from, and the output returned to,
+        pinned host memory (tw_decode_step_host): the copies run as kernels of
+        the step's launch chain.  q_host / out_host: pinned CPU fp16
+        [B][Hq][128].  The step's device q / out buffers serve as staging.
+        Synchronise the stream before reading out_host."""
+        lib = _capi.load()
+        shape = (self.kv.B, self.Hq, HEAD_DIM)
+        if out_host is None:
+            out_host = torch.empty(shape, dtype=torch.float16).pin_memory()
+        for t, name in ((q_host, "q_host"), (out_host, "out_host")):
+            if t.dtype != torch.float16 or t.is_cuda or not t.is_pinned() or \
+                    not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be a contiguous pinned CPU fp16 tensor {shape}")
+        if self._q_stage is None:
+            self._q_stage = torch.empty(shape, dtype=torch.float16, device=self.kv.k.device)
+        s = self._struct(self._q_stage)
+        check(lib.tw_decode_step_host(ctypes.byref(s), q_host.data_ptr(), out_host.data_ptr(),
+                                      _stream(stream)), "tw_decode_step_host")
+        return out_host
 
     def kernel_names(self):
         lib = _capi.load()

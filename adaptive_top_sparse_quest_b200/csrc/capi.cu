@@ -199,9 +199,23 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 int group_sets_of(int Hq, int Hk, int group_mode) { return (group_mode || Hq == Hk) ? 1 : 0; }
 
+// Device address of the page-locked host memory at p (allocated or registered
+// page-locked and mapped into the device's address space); nullptr for
+// pageable, device or unknown memory.
+const void* host_mapped(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 // The fused step, optionally recording an event before the first kernel and
-// after each kernel.
-int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaStream_t st) {
+// after each kernel, and optionally staging q in from and out back to
+// page-locked host memory with copy kernels in the same launch chain.
+int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaStream_t st,
+                     const uint16_t* q_host = nullptr, uint16_t* out_host = nullptr) {
   if (!s) return TW_ERR_INVALID_ARG;
   tw::Layout L;
   TW_TRY(check_kv(&s->kv, true, true, &L));
@@ -214,11 +228,23 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   TW_TRY(check_topp(s->q, Hq, L, s->codes, s->scales, s->zeros, cand, s->cand_stride, s->ncand,
                     s->p, s->group_mode, s->idx, s->capacity, s->count));
   TW_TRY(check_decode(s->q, Hq, L, s->idx, s->capacity, s->count, s->group_mode, s->out, s->lse));
+  const void* q_in = nullptr;
+  void* out_back = nullptr;
+  if (q_host || out_host) {
+    if (!q_host || !out_host || !aligned(q_host, 16) || !aligned(out_host, 16))
+      return TW_ERR_INVALID_ARG;
+    if (L.B > 0) {
+      q_in = host_mapped(q_host);
+      out_back = const_cast<void*>(host_mapped(out_host));
+      if (!q_in || !out_back) return TW_ERR_INVALID_ARG;
+    }
+  }
   if (L.B == 0) return TW_OK;
   const Plan plan = make_plan(L.B, Hq, L.Hk, L.N, s->capacity);
   TW_TRY(check_ws(s->ws, s->ws_bytes, plan.total));
   int sms = 0;
   TW_TRY(device_check(&sms));
+  const int64_t qo_bytes = (int64_t)L.B * Hq * tw::kHeadDim * 2;
   const int gs = group_sets_of(Hq, L.Hk, s->group_mode);
   const auto* q = reinterpret_cast<const __half*>(s->q);
   // programmatic dependent launch overlaps each kernel's launch with its
@@ -228,6 +254,10 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   Marker mk{events, n_events, st};
   cudaError_t e;
   if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  if (q_in) {   // the query comes in from host memory first
+    e = tw::launch_copy16(q_in, const_cast<uint16_t*>(s->q), qo_bytes, true, st, pdl);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   if (s->append_keys) {   // the newest token of every sequence joins the int4 cache and metadata
     e = tw::launch_append_keys(L, reinterpret_cast<const __half*>(s->kv.k),
                                const_cast<uint8_t*>(s->codes),
@@ -270,6 +300,10 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   e = tw::launch_sparse_decode(L, q, Hq, gs, K, V, rows, s->capacity, s->count, part, done, out,
                                s->lse, st, pdl);
   if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  if (out_back) {   // and the attention output goes back to host memory last
+    e = tw::launch_copy16(out, out_back, qo_bytes, false, st, pdl);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return check_launch();
 }
 
@@ -440,6 +474,12 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
 
 int tw_decode_step(const tw_step* step, void* stream) {
   return decode_step_impl(step, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+int tw_decode_step_host(const tw_step* step, const uint16_t* q_host, uint16_t* out_host,
+                        void* stream) {
+  if (!q_host || !out_host) return TW_ERR_INVALID_ARG;
+  return decode_step_impl(step, nullptr, 0, static_cast<cudaStream_t>(stream), q_host, out_host);
 }
 
 int tw_decode_step_num_kernels(const tw_step* step) {

@@ -86,6 +86,8 @@ cudaError_t launch_page_topk(const Layout& L, const float* scores, int budget_pa
                              cudaStream_t st, bool pdl);
 cudaError_t launch_resolve_pages(const Layout& L, const int32_t* cand, int cand_stride,
                                  uint32_t* row0, cudaStream_t st, bool pdl);
+cudaError_t launch_copy16(const void* src, void* dst, int64_t bytes, bool early, cudaStream_t st,
+                          bool pdl);
 cudaError_t launch_resolve_rows(const Layout& L, int Hq, int group_sets, const int32_t* idx,
                                 int icap, const int32_t* count, uint32_t* rows, cudaStream_t st,
                                 bool pdl);

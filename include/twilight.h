@@ -259,6 +259,22 @@ typedef struct tw_step {
 
 int tw_decode_step(const tw_step* step, void* stream);
 
+/* tw_decode_step with the query read from, and the attention output written
+ * to, page-locked host memory: q_host [B][Hq][128] fp16 is copied into
+ * step->q, the step runs, and step->out is copied to out_host [B][Hq][128],
+ * all enqueued on `stream` as kernels of one launch chain (a step moves only
+ * a few KB each way, less than a copy engine's fixed cost).  step->q and
+ * step->out stay the device staging buffers; lse stays on the device.
+ * q_host and out_host must be 16-byte aligned and lie in page-locked host
+ * memory mapped into the device's address space (cudaHostAlloc /
+ * cudaMallocHost, or cudaHostRegister with cudaHostRegisterMapped);
+ * pageable memory gives TW_ERR_INVALID_ARG before anything is launched.  As
+ * with cudaMemcpyAsync, q_host is read and out_host written when the stream
+ * reaches the call: do not write q_host or read out_host until the stream
+ * has passed it. */
+int tw_decode_step_host(const tw_step* step, const uint16_t* q_host, uint16_t* out_host,
+                        void* stream);
+
 /* Profiling variant of tw_decode_step: records events[0] before the first
  * kernel and events[i + 1] after kernel i on `stream` (events are
  * cudaEvent_t, n_events >= tw_decode_step_num_kernels(step) + 1). */

@@ -79,6 +79,16 @@ def test_kv_descriptor_checks(lib):
                                   None) == _capi.TW_ERR_UNSUPPORTED
 
 
+def test_host_staged_step_argument_checks(lib):
+    # null host buffers or a null step: rejected before any device work
+    assert lib.tw_decode_step_host(None, 1 << 20, 1 << 20, None) == _capi.TW_ERR_INVALID_ARG
+    st = _capi.TwStep()
+    assert lib.tw_decode_step_host(ctypes.byref(st), None, 1 << 20, None) == \
+        _capi.TW_ERR_INVALID_ARG
+    assert lib.tw_decode_step_host(ctypes.byref(st), 1 << 20, None, None) == \
+        _capi.TW_ERR_INVALID_ARG
+
+
 def test_struct_layout_matches_header():
     """The ctypes mirror of tw_kv ends with key_bits, after head_dim."""
     names = [f[0] for f in _capi.TwKv._fields_]
