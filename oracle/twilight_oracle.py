@@ -52,6 +52,16 @@ notes of this repository):
      2-bit for stable cumulative weights, table of measured effects) is R1
      with 3 in place of 15: scale = fp16_rn((max - min) / 3), codes 0..3,
      four per byte, channel 4i + j in bits 2j, 2j + 1 of byte i.
+  R9 the Double-Sparsity-style base selector (DS is named as a base selector
+     Twilight builds on: "Builds on", "Key results"; the pages give no
+     mechanism) is read as DS's published idea, synthetic: per KV head a set
+     of r "label" channels (given as input; real DS finds them by offline
+     calibration on trained weights), a label cache holding those channels of
+     every key, a token-level score
+         s_h[t] = sum_j q_h[c_j] * k_t[c_j]   (fp32, products exact, summed
+                  j = 0 .. r-1 left to right; group heads added in order)
+     and the min(budget, len) tokens with the largest score (ties to the lower
+     token index) as the candidate set, ascending.
 """
 from __future__ import annotations
 
@@ -72,6 +82,7 @@ __all__ = [
     "estimate_logits", "softmax_weights", "group_weights", "topp_select", "sparse_attention",
     "SeqInputs", "sequence_rows", "oracle_unit", "oracle_decode", "int4_cache_bytes_per_token",
     "key_cache_bytes_per_token", "kv_cache_bytes_per_token", "KEY_BITS", "retained_mass",
+    "label_cache", "label_scores", "select_tokens",
 ]
 
 KEY_BITS = (4, 2)   # key-cache widths: 4-bit (R1) and the ablation's 2-bit (R8)
@@ -246,6 +257,41 @@ def select_pages(scores: np.ndarray, budget_tokens: int) -> np.ndarray:
     return np.sort(order[:kp]).astype(np.int64)
 
 
+# ----------------------------------------------------------------------------- R9
+def label_cache(k_seq: np.ndarray, channels) -> np.ndarray:
+    """The label cache of a token-level base selector (reading R9): the fp16
+    values of the given channels of every key, [T][r], exact copies."""
+    ch = np.asarray(channels, np.int64)
+    return np.asarray(k_seq, np.float16)[:, ch].copy()
+
+
+def label_scores(q_group: np.ndarray, labels: np.ndarray, channels) -> np.ndarray:
+    """Token scores from the label channels (reading R9), fp32.  For each query
+    head h of the group, s_h[t] = sum over j = 0 .. r-1, left to right, of
+    q_h[c_j] * label[t][j] (each product exact in fp32, each add rounded);
+    heads are added in order: ((s_0 + s_1) + s_2) + ...  Returns [T]."""
+    q = np.asarray(q_group, np.float16).astype(np.float32)[:, np.asarray(channels, np.int64)]
+    lab = np.asarray(labels, np.float16).astype(np.float32)
+    total = None
+    for h in range(q.shape[0]):
+        s = np.zeros(lab.shape[0], np.float32)
+        for j in range(lab.shape[1]):
+            s = s + q[h, j] * lab[:, j]
+        total = s if total is None else total + s
+    if total is None:
+        total = np.zeros(lab.shape[0], np.float32)
+    return total.astype(np.float32)
+
+
+def select_tokens(scores: np.ndarray, budget_tokens: int) -> np.ndarray:
+    """Token-level top-k (reading R9): the min(budget, T) tokens with the
+    largest score, ties to the lower token index, returned ascending."""
+    T = len(scores)
+    k = min(int(budget_tokens), T)
+    order = np.lexsort((np.arange(T), -np.asarray(scores, np.float64)))
+    return np.sort(order[:k]).astype(np.int64)
+
+
 def candidate_tokens(pages: Optional[np.ndarray], length: int) -> np.ndarray:
     """Token indices (ascending) of the candidate pages, valid tokens only; None
     means every token of the sequence is a candidate (base = full attention)."""
@@ -377,7 +423,7 @@ def sequence_rows(arr: np.ndarray, page_table, b: int, h: int, length: int) -> n
 
 def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: float,
                 group_mode: int, sel_override: Optional[dict] = None,
-                key_bits: int = 4) -> dict:
+                key_bits: int = 4, label_channels=None) -> dict:
     """Every result of the decode path for one (sequence, KV head).
 
     Returns a dict with the quantised key cache (`key_bits` wide), page meta,
@@ -385,7 +431,9 @@ def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: 
     selections / thresholds, and the attention output of each query head of the
     group.  `sel_override` maps a query head to the selected token list to
     attend over (used to check the attention stage on another implementation's
-    selection)."""
+    selection).  With `label_channels` ([Hk][r]) and a budget, the base
+    selector is the token-level label-channel one (R9) instead of Quest's
+    pages: "pages" is then None and "label_scores" holds the token scores."""
     L = int(x.seq_lens[b])
     G = x.Hq // x.Hk
     heads = list(range(hk * G, (hk + 1) * G))
@@ -397,10 +445,16 @@ def oracle_unit(x: SeqInputs, b: int, hk: int, budget_tokens: Optional[int], p: 
     res = {"len": L, "codes": codes, "scales": scales, "zeros": zeros, "meta": meta}
     if budget_tokens is None:
         pages, scores = None, None
+        toks = candidate_tokens(None, L)
+    elif label_channels is not None:
+        ch = np.asarray(label_channels, np.int64)[hk]
+        pages, scores = None, None
+        res["label_scores"] = label_scores(qg, label_cache(k_seq, ch), ch)
+        toks = select_tokens(res["label_scores"], budget_tokens)
     else:
         scores = quest_page_scores(qg, meta)
         pages = select_pages(scores, budget_tokens)
-    toks = candidate_tokens(pages, L)
+        toks = candidate_tokens(pages, L)
     res.update(scores=scores, pages=pages, cand_tokens=toks)
     logits = estimate_logits(qg, codes[toks], scales[toks], zeros[toks], key_bits)   # [C][G]
     res["logits"] = logits

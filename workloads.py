@@ -265,6 +265,22 @@ def random_small(seed: int, device="cpu", B: int = 2, Hq: int = 4, Hk: int = 2, 
     return w
 
 
+def label_channels(w: Workload, r: int = 16, seed: int = 7) -> list:
+    """Label channels [Hk][r] for a token-level base selector: a seeded stand-in
+    for offline calibration on trained weights.  The workload's planted outlier
+    channels (if any) come first, then distinct seeded random channels."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    planted = []
+    if isinstance(w.heavy, dict):
+        planted = [int(c) for c in w.heavy.get("outlier_channels", [])][:r]
+    out = []
+    for _ in range(w.Hk):
+        rest = [int(c) for c in torch.randperm(HEAD_DIM, generator=g) if int(c) not in planted]
+        out.append(planted + rest[:r - len(planted)])
+    return out
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama2_mha": llama2_mha,
