@@ -5,6 +5,7 @@ thresholding, and split-K sparse attention over the survivors.
 The CUDA library (lib/libtwilight.so, C ABI in include/twilight.h) does all the
 work; this package only marshals PyTorch tensors into it.
 """
-from .api import (DecodeStep, Int4Keys, KVCache, append_keys, page_meta, prepare,  # noqa: F401
-                  quantize_keys, select_pages, sparse_decode, topp_prune, workspace_bytes,
-                  new_workspace)
+from .api import (DecodeStep, Int4Keys, KVCache, LabelDecodeStep, append_keys,  # noqa: F401
+                  label_cache, new_workspace, page_meta, prepare, quantize_keys, select_pages,
+                  select_tokens, sparse_decode, token_workspace_bytes, topp_prune,
+                  topp_prune_tokens, workspace_bytes)

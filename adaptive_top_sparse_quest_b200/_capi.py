@@ -63,6 +63,14 @@ _SIGS = {
     "tw_topp_prune_noalloc": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_vp, c_vp,
                                              c_vp, c_i32, c_vp, ctypes.c_double, c_i32, c_vp,
                                              c_i32, c_vp, c_vp]),
+    "tw_label_cache": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_i32, c_vp, c_vp]),
+    "tw_token_workspace_size": (ctypes.c_int, [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                               ctypes.POINTER(c_size)]),
+    "tw_select_tokens": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_vp, c_i32,
+                                        c_i32, c_vp, c_i32, c_vp, c_vp, c_size, c_vp]),
+    "tw_topp_prune_tokens": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(TwKv), c_vp, c_vp, c_vp,
+                                            c_vp, c_i32, c_vp, ctypes.c_double, c_i32, c_vp,
+                                            c_i32, c_vp, c_vp, c_size, c_vp]),
     "tw_decode_step": (ctypes.c_int, [ctypes.POINTER(TwStep), c_vp]),
     "tw_decode_step_host": (ctypes.c_int, [ctypes.POINTER(TwStep), c_vp, c_vp, c_vp]),
     "tw_decode_step_num_kernels": (ctypes.c_int, [ctypes.POINTER(TwStep)]),

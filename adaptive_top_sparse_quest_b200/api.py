@@ -382,3 +382,159 @@ def prepare(w, device=None, key_bits: int = 4):
     keys = quantize_keys(kv)
     meta = page_meta(kv)
     return kv, keys, meta, w.q
+
+
+# ----------------------------------------------------------------------------- label selector
+def label_cache(kv: KVCache, channels: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Label cache of the token-level label-channel selector (tw_label_cache):
+    the fp16 values of channels[h] (int32 CUDA [Hk][r]) of every key row."""
+    lib = _capi.load()
+    _need(channels, torch.int32, "channels")
+    r = int(channels.shape[-1])
+    if tuple(channels.shape) != (kv.Hk, r):
+        raise ValueError(f"channels must be [{kv.Hk}][r]")
+    if out is None:
+        out = torch.zeros(kv.row_shape(r), dtype=torch.float16, device=kv.k.device)
+    s = kv.struct()
+    check(lib.tw_label_cache(ctypes.byref(s), _ptr(channels), r, _ptr(out), _stream(stream)),
+          "tw_label_cache")
+    return out
+
+
+def token_workspace_bytes(B, Hq, Hk, N, cand_stride, capacity, key_bits=4) -> int:
+    lib = _capi.load()
+    n = ctypes.c_size_t(0)
+    check(lib.tw_token_workspace_size(B, Hq, Hk, N, cand_stride, capacity, key_bits,
+                                      ctypes.byref(n)), "tw_token_workspace_size")
+    return int(n.value)
+
+
+def _token_ws(kv, Hq, stride, capacity, device):
+    n = max(token_workspace_bytes(kv.B, Hq, kv.Hk, kv.N, stride, capacity, kv.key_bits), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def select_tokens(q: torch.Tensor, kv: KVCache, labels: torch.Tensor, channels: torch.Tensor,
+                  budget_tokens: int, ws: Optional[torch.Tensor] = None, stream=None):
+    """Token-level label-channel pre-selection (tw_select_tokens) ->
+    (cand_tokens [B][Hk][stride], ncand [B][Hk]), stride = min(budget, N)."""
+    lib = _capi.load()
+    _need(q, torch.float16, "q")
+    Hq = int(q.shape[1])
+    r = int(channels.shape[-1])
+    stride = max(1, min(int(budget_tokens), kv.N))
+    cand = torch.zeros((kv.B, kv.Hk, stride), dtype=torch.int32, device=q.device)
+    ncand = torch.zeros((kv.B, kv.Hk), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = _token_ws(kv, Hq, stride, stride, q.device)
+    s = kv.struct()
+    check(lib.tw_select_tokens(_ptr(q), Hq, ctypes.byref(s), _ptr(labels), _ptr(channels), r,
+                               int(budget_tokens), _ptr(cand), stride, _ptr(ncand), _ptr(ws),
+                               ws.numel(), _stream(stream)), "tw_select_tokens")
+    return cand, ncand
+
+
+def topp_prune_tokens(q: torch.Tensor, kv: KVCache, keys: Int4Keys, cand: torch.Tensor,
+                      ncand: torch.Tensor, p: float, group_mode: int = 0,
+                      capacity: Optional[int] = None, ws: Optional[torch.Tensor] = None,
+                      stream=None):
+    """Twilight top-p over token candidates (tw_topp_prune_tokens) -> (idx, count)."""
+    lib = _capi.load()
+    _need(q, torch.float16, "q")
+    _check_keys(kv, keys)
+    Hq = int(q.shape[1])
+    stride = int(cand.shape[-1])
+    capacity = stride if capacity is None else int(capacity)
+    U = num_sets(kv, Hq, group_mode)
+    idx = torch.zeros((U, capacity), dtype=torch.int32, device=q.device)
+    count = torch.zeros((U,), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = _token_ws(kv, Hq, stride, capacity, q.device)
+    s = kv.struct()
+    check(lib.tw_topp_prune_tokens(_ptr(q), Hq, ctypes.byref(s), _ptr(keys.codes),
+                                   _ptr(keys.scales), _ptr(keys.zeros), _ptr(cand), stride,
+                                   _ptr(ncand), float(p), int(group_mode), _ptr(idx), capacity,
+                                   _ptr(count), _ptr(ws), ws.numel(), _stream(stream)),
+          "tw_topp_prune_tokens")
+    return idx, count
+
+
+class LabelDecodeStep:
+    """A decode step with the token-level label-channel base selector:
+    tw_select_tokens -> tw_topp_prune_tokens -> tw_sparse_decode on one
+    stream with pre-allocated buffers (no host synchronisation)."""
+
+    NAMES = ("select_tokens", "topp_prune_tokens", "sparse_decode")
+    LAUNCHES = 2 + 4 + 2   # kernels of the three calls
+
+    def __init__(self, kv: KVCache, keys: Int4Keys, labels: torch.Tensor, channels: torch.Tensor,
+                 Hq: int, budget_tokens: int, p: float, group_mode: int = 0,
+                 with_lse: bool = True):
+        _check_keys(kv, keys)
+        self.kv, self.keys, self.labels, self.channels = kv, keys, labels, channels
+        self.Hq, self.budget, self.p, self.group_mode = Hq, int(budget_tokens), float(p), \
+            int(group_mode)
+        dev = kv.k.device
+        self.stride = max(1, min(self.budget, kv.N))
+        self.capacity = self.stride
+        self.cand = torch.zeros((kv.B, kv.Hk, self.stride), dtype=torch.int32, device=dev)
+        self.ncand = torch.zeros((kv.B, kv.Hk), dtype=torch.int32, device=dev)
+        U = num_sets(kv, Hq, group_mode)
+        self.idx = torch.zeros((U, self.capacity), dtype=torch.int32, device=dev)
+        self.count = torch.zeros((U,), dtype=torch.int32, device=dev)
+        self.out = torch.zeros((kv.B, Hq, HEAD_DIM), dtype=torch.float16, device=dev)
+        self.lse = torch.zeros((kv.B, Hq), dtype=torch.float32, device=dev) if with_lse else None
+        n = max(token_workspace_bytes(kv.B, Hq, kv.Hk, kv.N, self.stride, self.capacity,
+                                      kv.key_bits),
+                workspace_bytes(kv.B, Hq, kv.Hk, kv.N, self.capacity), 256)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self._kvs = kv.struct()
+        self._q_stage = None
+
+    def _calls(self, q: torch.Tensor, stream):
+        lib = _capi.load()
+        st = _stream(stream)
+        kvs, ws, nws = ctypes.byref(self._kvs), _ptr(self.ws), self.ws.numel()
+        r = int(self.channels.shape[-1])
+        yield lambda: check(lib.tw_select_tokens(
+            _ptr(q), self.Hq, kvs, _ptr(self.labels), _ptr(self.channels), r, self.budget,
+            _ptr(self.cand), self.stride, _ptr(self.ncand), ws, nws, st), "tw_select_tokens")
+        yield lambda: check(lib.tw_topp_prune_tokens(
+            _ptr(q), self.Hq, kvs, _ptr(self.keys.codes), _ptr(self.keys.scales),
+            _ptr(self.keys.zeros), _ptr(self.cand), self.stride, _ptr(self.ncand), self.p,
+            self.group_mode, _ptr(self.idx), self.capacity, _ptr(self.count), ws, nws, st),
+            "tw_topp_prune_tokens")
+        yield lambda: check(lib.tw_sparse_decode(
+            _ptr(q), self.Hq, kvs, _ptr(self.idx), self.capacity, _ptr(self.count),
+            self.group_mode, _ptr(self.out), _ptr(self.lse), ws, nws, st), "tw_sparse_decode")
+
+    def __call__(self, q: torch.Tensor, stream=None) -> torch.Tensor:
+        _need(q, torch.float16, "q")
+        for call in self._calls(q, stream):
+            call()
+        return self.out
+
+    def kernel_names(self):
+        return list(self.NAMES)
+
+    def profiled(self, q: torch.Tensor, events, stream=None) -> None:
+        """One step with events[0] before and events[i + 1] after call i."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        events[0].record(s)
+        for i, call in enumerate(self._calls(q, stream)):
+            call()
+            events[i + 1].record(s)
+
+    def run_host(self, q_host: torch.Tensor, out_host: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        """One step from and to pinned host memory (copy-engine transfers)."""
+        if out_host is None:
+            out_host = torch.empty(tuple(self.out.shape), dtype=torch.float16).pin_memory()
+        if self._q_stage is None:
+            self._q_stage = torch.empty(tuple(self.out.shape), dtype=torch.float16,
+                                        device=self.kv.k.device)
+        self._q_stage.copy_(q_host, non_blocking=True)
+        self(self._q_stage, stream)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host

@@ -8,6 +8,7 @@
 
 #include "twilight.h"
 #include "tw_kernels.h"
+#include "tw_label.h"
 
 namespace {
 
@@ -307,6 +308,29 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
   return check_launch();
 }
 
+// Workspace of tw_topp_prune_tokens: the pruner's own regions for the
+// contiguous cache of candidate rows (B * Hk one-head sequences of cand_stride
+// rows, G query heads each), then that cache's codes, scales and zeros.
+struct TokenPlan {
+  Plan topp;
+  size_t vcodes_off, vscales_off, vzeros_off, total;
+};
+
+TokenPlan make_token_plan(int B, int Hq, int Hk, int cand_stride, int capacity, int kbits) {
+  TokenPlan t;
+  t.topp = make_plan(B * Hk, Hq / Hk, 1, cand_stride, capacity);
+  const size_t rows = (size_t)B * Hk * cand_stride;
+  t.vcodes_off = align256(t.topp.topp_end);
+  t.vscales_off = t.vcodes_off + align256(rows * (size_t)(tw::kHeadDim * kbits / 8));
+  t.vzeros_off = t.vscales_off + align256(rows * tw::kGroups * sizeof(uint16_t));
+  t.total = t.vzeros_off + align256(rows * tw::kGroups * sizeof(uint16_t));
+  return t;
+}
+
+size_t label_scores_bytes(int B, int Hk, int N) {
+  return align256((size_t)B * Hk * N * sizeof(float));
+}
+
 }  // namespace
 
 extern "C" {
@@ -468,6 +492,125 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
     e = tw::launch_sparse_decode(L, reinterpret_cast<const __half*>(q), num_q_heads, gs, K, V,
                                  rows, capacity, count, part, done,
                                  reinterpret_cast<__half*>(out), lse, st, false);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+int tw_label_cache(const tw_kv* kv, const int32_t* channels, int32_t r, uint16_t* labels,
+                   void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, true, false, &L));
+  if (!channels || !aligned(channels, 4) || !labels || !aligned(labels, 2))
+    return TW_ERR_INVALID_ARG;
+  if (r < 1 || r > tw::kMaxLabelChannels) return TW_ERR_UNSUPPORTED;
+  if ((int64_t)L.B * L.N == 0) return TW_OK;
+  int sms = 0;
+  TW_TRY(device_check(&sms));
+  const cudaError_t e =
+      tw::launch_label_cache(L, reinterpret_cast<const __half*>(kv->k), channels, r,
+                             reinterpret_cast<__half*>(labels), static_cast<cudaStream_t>(stream),
+                             sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+int tw_token_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t max_seq_len, int32_t cand_stride, int32_t capacity,
+                            int32_t key_bits, size_t* bytes) {
+  if (!bytes || batch < 0 || num_kv_heads < 1 || max_seq_len < 0 || cand_stride < 1 ||
+      capacity < cand_stride)
+    return TW_ERR_INVALID_ARG;
+  if (key_bits != 0 && key_bits != 2 && key_bits != 4) return TW_ERR_UNSUPPORTED;
+  TW_TRY(check_heads(num_q_heads, num_kv_heads));
+  const size_t a = label_scores_bytes(batch, num_kv_heads, max_seq_len);
+  const size_t b = make_token_plan(batch, num_q_heads, num_kv_heads, cand_stride, capacity,
+                                   key_bits == 2 ? 2 : 4).total;
+  *bytes = a > b ? a : b;
+  return TW_OK;
+}
+
+int tw_select_tokens(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                     const uint16_t* labels, const int32_t* channels, int32_t r,
+                     int32_t budget_tokens, int32_t* cand_tokens, int32_t cand_stride,
+                     int32_t* ncand, void* ws, size_t ws_bytes, void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, false, false, &L));
+  TW_TRY(check_heads(num_q_heads, L.Hk));
+  if (!q || !aligned(q, 16) || !labels || !aligned(labels, 2) || !channels ||
+      !aligned(channels, 4) || !cand_tokens || !aligned(cand_tokens, 4) || !ncand ||
+      !aligned(ncand, 4))
+    return TW_ERR_INVALID_ARG;
+  if (r < 1 || r > tw::kMaxLabelChannels) return TW_ERR_UNSUPPORTED;
+  if (budget_tokens < 1) return TW_ERR_INVALID_ARG;
+  const int keep = budget_tokens < L.N ? budget_tokens : L.N;
+  if (cand_stride < keep || cand_stride < 1) return TW_ERR_CAPACITY;
+  if ((int64_t)L.B * L.Hk > 65535) return TW_ERR_UNSUPPORTED;
+  if (L.B == 0) return TW_OK;
+  TW_TRY(check_ws(ws, ws_bytes, label_scores_bytes(L.B, L.Hk, L.N)));
+  TW_TRY(device_check(nullptr));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = reinterpret_cast<float*>(ws);
+  cudaError_t e = tw::launch_label_scores(L, reinterpret_cast<const __half*>(q), num_q_heads,
+                                          reinterpret_cast<const __half*>(labels), channels, r,
+                                          scores, st);
+  if (e == cudaSuccess)
+    e = tw::launch_token_topk(L, scores, budget_tokens, cand_tokens, cand_stride, ncand, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch();
+}
+
+int tw_topp_prune_tokens(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                         const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                         const int32_t* cand_tokens, int32_t cand_stride, const int32_t* ncand,
+                         double p, int32_t group_mode, int32_t* idx, int32_t capacity,
+                         int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  tw::Layout L;
+  TW_TRY(check_kv(kv, false, false, &L));
+  TW_TRY(check_heads(num_q_heads, L.Hk));
+  if (!cand_tokens || !aligned(cand_tokens, 4) || !ncand || !aligned(ncand, 4) ||
+      cand_stride < 1)
+    return TW_ERR_INVALID_ARG;
+  if ((int64_t)L.B * L.Hk * cand_stride >= (int64_t)tw::kNoRow) return TW_ERR_UNSUPPORTED;
+  // the candidate rows form a contiguous cache of B * Hk one-head sequences
+  // (lengths ncand) of cand_stride rows, on which the page-free pruner runs
+  const int G = num_q_heads / L.Hk;
+  tw::Layout Lv;
+  Lv.B = L.B * L.Hk;
+  Lv.Hk = 1;
+  Lv.N = cand_stride;
+  Lv.seq_lens = ncand;
+  Lv.page_table = nullptr;
+  Lv.max_pages = (cand_stride + tw::kPage - 1) / tw::kPage;
+  Lv.pool_pages = 0;
+  Lv.kbits = L.kbits;
+  TW_TRY(check_topp(q, G, Lv, codes, scales, zeros, nullptr, 0, nullptr, p, group_mode, idx,
+                    capacity, count));
+  if (L.B == 0) return TW_OK;
+  const TokenPlan plan = make_token_plan(L.B, num_q_heads, L.Hk, cand_stride, capacity, L.kbits);
+  TW_TRY(check_ws(ws, ws_bytes, plan.total));
+  int sms = 0;
+  TW_TRY(device_check(&sms));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* vcodes = reinterpret_cast<uint8_t*>(wsp(ws, plan.vcodes_off));
+  auto* vscales = reinterpret_cast<__half*>(wsp(ws, plan.vscales_off));
+  auto* vzeros = reinterpret_cast<__half*>(wsp(ws, plan.vzeros_off));
+  float* logits = reinterpret_cast<float*>(wsp(ws, plan.topp.logits_off));
+  float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.topp.stats_off));
+  const int gs = group_sets_of(num_q_heads, L.Hk, group_mode);
+  const int nsets = gs ? L.B * L.Hk : L.B * num_q_heads;
+  cudaError_t e = tw::launch_gather_keys(L, cand_tokens, cand_stride, ncand, codes,
+                                         reinterpret_cast<const __half*>(scales),
+                                         reinterpret_cast<const __half*>(zeros), vcodes, vscales,
+                                         vzeros, st, sms);
+  if (e == cudaSuccess)
+    e = tw::launch_estimate(Lv, reinterpret_cast<const __half*>(q), G, vcodes, vscales, vzeros,
+                            nullptr, 0, nullptr, nullptr, plan.topp.lcap, cand_stride, logits,
+                            stats, st, sms, false);
+  if (e == cudaSuccess)
+    e = tw::launch_topp(Lv, G, gs, nullptr, 0, nullptr, nullptr, plan.topp.lcap, cand_stride,
+                        logits, stats, p, idx, nullptr, capacity, count, nullptr, st, false);
+  if (e == cudaSuccess)
+    e = tw::launch_map_tokens(nsets, G, gs, cand_tokens, cand_stride, idx, capacity, count, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }

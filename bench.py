@@ -59,6 +59,9 @@ def parse():
                     help="rotating cache copies (0: enough to exceed L2 several times)")
     ap.add_argument("--key-bits", type=int, default=4, choices=[4, 2],
                     help="width of the quantised key cache used for the weight estimate")
+    ap.add_argument("--selector", default="quest", choices=["quest", "label"],
+                    help="base selector: Quest pages, or token-level label channels "
+                         "(synthetic Double Sparsity, 16 channels per KV head)")
     return ap.parse_args()
 
 
@@ -67,24 +70,31 @@ def make_workload(name, device):
     return W.CONFIGS[name](device=device)
 
 
-def workload_config(w, copies=None, copy_bytes=None, key_bits=4):
+def workload_config(w, copies=None, copy_bytes=None, key_bits=4, selector="quest"):
     c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hk,
          "context": w.N, "paged": w.paged, "budget_tokens": w.budget_tokens, "p": w.p,
          "group_mode": w.group_mode, "head_dim": 128, "page_size": 16, "key_bits": key_bits,
-         "key_group": 32}
+         "key_group": 32, "selector": selector}
+    if selector == "label":
+        c["label_channels"] = LABEL_R
     if copies:
         c["l2"] = (f"inputs larger than L2: {copies} rotating cache copies, "
                    f"{copy_bytes / 1e9:.2f} GB each")
     return c
 
 
+# Device sources of the kernels the traffic record measures (and the headers
+# they include): the record is used only while these bytes are unchanged.
+TRAFFIC_SOURCES = ("cache_build.cu", "decode.cu", "estimate.cu", "host_io.cu", "resolve.cu",
+                   "select.cu", "topp.cu", "tw_common.cuh", "tw_kernels.h")
+
+
 def src_hash():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "adaptive_top_sparse_quest_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in TRAFFIC_SOURCES:
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -174,12 +184,13 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def cpu_step_sample(w_cpu, seconds: float, max_units=None, key_bits=4):
+def cpu_step_sample(w_cpu, seconds: float, max_units=None, key_bits=4, label_channels=None):
     """Time the oracle's decode step (page scores, top-K_p, quantised-key
     estimate, top-p, sparse attention) on (b, kv head) units of the workload
     until `seconds` of CPU work; the key cache and page metadata are built
     first, untimed, as at prefill.  Returns (us per full step, units timed,
-    total units, threads)."""
+    total units, threads).  With label_channels the base selector is the
+    token-level label-channel one instead of Quest's pages."""
     try:
         from threadpoolctl import threadpool_limits
         limiter = threadpool_limits(limits=1)
@@ -203,12 +214,17 @@ def cpu_step_sample(w_cpu, seconds: float, max_units=None, key_bits=4):
         v_seq = O.sequence_rows(x.v, x.page_table, b, hk, L)
         codes, scales, zeros = O.quantize_keys(k_seq, key_bits)
         meta = O.page_meta(k_seq, L) if w_cpu.budget_tokens else None
+        labels = O.label_cache(k_seq, label_channels[hk]) if label_channels is not None else None
         qg = x.q[b, hk * G:(hk + 1) * G]
         t0 = time.perf_counter()
         pages = None
-        if w_cpu.budget_tokens:
-            pages = O.select_pages(O.quest_page_scores(qg, meta), w_cpu.budget_tokens)
-        toks = O.candidate_tokens(pages, L)
+        if labels is not None:
+            toks = O.select_tokens(O.label_scores(qg, labels, label_channels[hk]),
+                                   w_cpu.budget_tokens)
+        else:
+            if w_cpu.budget_tokens:
+                pages = O.select_pages(O.quest_page_scores(qg, meta), w_cpu.budget_tokens)
+            toks = O.candidate_tokens(pages, L)
         lg = O.estimate_logits(qg, codes[toks], scales[toks], zeros[toks], key_bits)
         if w_cpu.group_mode and G > 1:
             sel = O.topp_select(O.group_weights(lg), w_cpu.p)[0]
@@ -233,9 +249,14 @@ def run_reference(args):
         return 0
     import torch
     w = make_workload(args.config, "cpu")
+    chans = None
+    if args.selector == "label":
+        import workloads as W
+        chans = W.label_channels(w, r=LABEL_R)
     per = []
     for i in range(args.warmup + args.steps):
-        us, n, tot, cores = cpu_step_sample(w, 0.0, max_units=1, key_bits=args.key_bits)
+        us, n, tot, cores = cpu_step_sample(w, 0.0, max_units=1, key_bits=args.key_bits,
+                                            label_channels=chans)
         if i >= args.warmup:
             per.append(us)
     value = statistics.mean(per)
@@ -244,7 +265,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": value / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, key_bits=args.key_bits),
+        "config": workload_config(w, key_bits=args.key_bits, selector=args.selector),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"each step: 1 random (sequence, KV head) unit of {tot}, "
                                    "scaled by the unit count"},
@@ -255,6 +276,24 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+LABEL_R = 16
+
+
+def label_algorithmic_bytes(w, step, key_bits=4):
+    """Bytes the label-selector step must move (per call): the label cache
+    (2 B per label channel per token per KV head) and the scores written and
+    read back (4 + 4 B); the candidates' quantised keys read, copied and read
+    again by the estimate (3 x (128 * key_bits / 8 + 16) B); the selected
+    tokens' fp16 K+V rows (512 B per token per set)."""
+    import torch
+    toks = int(w.seq_lens.to(torch.int64).sum()) * w.Hk
+    cand_tokens = int(step.ncand.to(torch.int64).sum())
+    kept = step.count.to(torch.int64).cpu()
+    return {"select_tokens": toks * (2 * LABEL_R + 8),
+            "topp_prune_tokens": cand_tokens * 3 * (128 * key_bits // 8 + 16),
+            "sparse_decode": int(kept.sum()) * 512}, cand_tokens, kept
+
+
 def algorithmic_bytes(w, step, key_bits=4):
     """Bytes the step must move (per kernel): page metadata scanned (512 B per
     page per KV head), quantised candidate keys (128 * key_bits / 8 B of codes
@@ -302,7 +341,8 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    from adaptive_top_sparse_quest_b200 import (DecodeStep, KVCache, _capi, append_keys, page_meta,
+    from adaptive_top_sparse_quest_b200 import (DecodeStep, KVCache, LabelDecodeStep, _capi,
+                                                append_keys, label_cache, page_meta,
                                                 quantize_keys)
     from adaptive_top_sparse_quest_b200 import build as _b
     _b.build()
@@ -344,6 +384,19 @@ def main():
     torch.cuda.synchronize()
     append_us = ea.elapsed_time(eb) * 1e3 / 20
 
+    label = args.selector == "label"
+    if label and not w.budget_tokens:
+        raise SystemExit("--selector label needs a workload with a token budget")
+    if label:
+        import workloads as W
+        channels = torch.tensor(W.label_channels(w, r=LABEL_R), dtype=torch.int32, device=dev)
+
+    def make_step(kv, keys, meta, p):
+        if label:
+            return LabelDecodeStep(kv, keys, label_cache(kv, channels), channels, w.Hq,
+                                   w.budget_tokens, p, w.group_mode)
+        return DecodeStep(kv, keys, meta, w.Hq, w.budget_tokens, p, w.group_mode)
+
     steps = []
     for r in range(R):
         if r == 0:
@@ -353,7 +406,7 @@ def main():
                          None if w.page_table is None else w.page_table.clone(), args.key_bits)
             keys = type(keys0)(keys0.codes.clone(), keys0.scales.clone(), keys0.zeros.clone())
             meta = meta0.clone()
-        steps.append(DecodeStep(kv, keys, meta, w.Hq, w.budget_tokens, w.p, w.group_mode))
+        steps.append(make_step(kv, keys, meta, w.p))
     q = w.q.contiguous()
     torch.cuda.synchronize()
 
@@ -439,8 +492,7 @@ def main():
     # the second lse from the same step run with p = 1 (outside the timed region)
     steps[0](q)
     lse_p = steps[0].lse.double().clone()
-    full = DecodeStep(steps[0].kv, steps[0].keys, steps[0].meta, w.Hq, w.budget_tokens, 1.0,
-                      w.group_mode)
+    full = make_step(steps[0].kv, steps[0].keys, getattr(steps[0], "meta", None), 1.0)
     full(q)
     torch.cuda.synchronize()
     retained = torch.exp(lse_p - full.lse.double()).flatten().cpu()
@@ -450,7 +502,10 @@ def main():
             dist.destroy_process_group()
         return 0
 
-    kb, cand_tokens, kept = algorithmic_bytes(w, steps[0], args.key_bits)
+    if label:
+        kb, cand_tokens, kept = label_algorithmic_bytes(w, steps[0], args.key_bits)
+    else:
+        kb, cand_tokens, kept = algorithmic_bytes(w, steps[0], args.key_bits)
     toks_total = int(w.seq_lens.to(torch.int64).sum()) * w.Hk
     pages_total = int(((w.seq_lens.to(torch.int64) + 15) // 16).sum()) * w.Hk
     total_b = sum(kb.values())
@@ -462,6 +517,8 @@ def main():
     try:   # ncu DRAM bytes per launch, valid only for the sources they were taken on
         tr = json.load(open(TRAFFIC_PATH))
         sect = "kernels" if args.key_bits == 4 else f"kernels_key_bits_{args.key_bits}"
+        if label:
+            sect = "kernels_label_selector"
         if tr.get("src_hash") == src_hash() and tr.get("workload") == w.name:
             traffic = tr.get(sect, {}).get(dom, {}).get("dram_bytes_per_launch")
     except Exception:
@@ -471,8 +528,9 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         w_cpu = w.to("cpu")
-        cpu_us, n_units, tot_units, cores = cpu_step_sample(w_cpu, args.cpu_seconds,
-                                                            key_bits=args.key_bits)
+        cpu_us, n_units, tot_units, cores = cpu_step_sample(
+            w_cpu, args.cpu_seconds, key_bits=args.key_bits,
+            label_channels=W.label_channels(w, r=LABEL_R) if label else None)
         cpu = {"value": cpu_us, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n_units} of {tot_units} (sequence, KV head) units of the same "
                          f"workload, single-threaded numpy, scaled to the full step"}
@@ -484,7 +542,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, R, copy_bytes, args.key_bits),
+        "config": workload_config(w, R, copy_bytes, args.key_bits, args.selector),
         "hbm_gbs": total_b / (us_per_step * 1e-6) / 1e9,
         "hbm_frac_of_measured": total_b / (us_per_step * 1e-6) / 1e9 / peak,
         "bytes_per_step": total_b,
@@ -507,8 +565,8 @@ def main():
             "append_keys_us": append_us},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": q.numel() * q.element_size(),
                 "d2h_bytes_per_step": steps[0].out.numel() * steps[0].out.element_size()},
-        "gpu_launches": args.steps * nk,
-        "e2e_gpu_launches": args.steps * (nk + 2),
+        "gpu_launches": args.steps * (LabelDecodeStep.LAUNCHES if label else nk),
+        "e2e_gpu_launches": args.steps * ((LabelDecodeStep.LAUNCHES if label else nk) + 2),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -228,6 +228,53 @@ int tw_topp_prune_noalloc(const uint16_t* q, int32_t num_q_heads, const tw_kv* k
                           double p, int32_t group_mode, int32_t* idx, int32_t capacity,
                           int32_t* count, void* stream);
 
+/*
+ * Token-level label-channel base selector: a synthetic stand-in for Double
+ * Sparsity, the other base selector Twilight builds on (atlas.scime.ai
+ * summary, "Builds on", "Key results"; the pages give no mechanism, so this
+ * follows Double Sparsity's published idea).  Per KV head h, r label channels
+ * channels[h][0 .. r) (device int32 [Hk][r], values in [0, 128); out-of-range
+ * values are clamped) stand in for offline calibration on trained weights.
+ * Use: tw_label_cache once per token (prefill), then per decode step
+ * tw_select_tokens -> tw_topp_prune_tokens -> tw_sparse_decode.
+ */
+
+/* labels[row][j] = K[row][channels[h][j]] (fp16, r per row, rows addressed
+ * like codes: [B][Hk][N][r] contiguous, [num_pool_pages][Hk][16][r] paged) for
+ * every valid token.  1 <= r <= 32. */
+int tw_label_cache(const tw_kv* kv, const int32_t* channels, int32_t r, uint16_t* labels,
+                   void* stream);
+
+/* Workspace bytes for tw_select_tokens and tw_topp_prune_tokens (the maximum
+ * of the two) with these sizes; key_bits as in tw_kv. */
+int tw_token_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t max_seq_len, int32_t cand_stride, int32_t capacity,
+                            int32_t key_bits, size_t* bytes);
+
+/* For each (b, KV head h): score[t] = sum over the G query heads of the group,
+ * in head order, of sum_{j = 0 .. r-1, in order} q_hq[c_j] * labels[t][j]
+ * (fp32, products exact, each sum rounded), and the min(budget_tokens,
+ * len_b) tokens with the largest score (ties to the lower token index)
+ * written ascending to cand_tokens[b][h][0 ..), their number to ncand[b][h].
+ * cand_stride >= min(budget_tokens, N); budget_tokens >= 1; B * Hk <= 65535.
+ * Bit-exact token ids with the CPU definition. */
+int tw_select_tokens(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                     const uint16_t* labels, const int32_t* channels, int32_t r,
+                     int32_t budget_tokens, int32_t* cand_tokens, int32_t cand_stride,
+                     int32_t* ncand, void* ws, size_t ws_bytes, void* stream);
+
+/* tw_topp_prune over token candidates: cand_tokens[b][h][0 .. ncand[b][h])
+ * (ascending valid token ids, ncand <= cand_stride) instead of pages.  The
+ * same estimate, threshold and tie rule as tw_topp_prune; idx holds token ids
+ * (ascending), count the kept numbers.  capacity >= cand_stride; workspace
+ * from tw_token_workspace_size.  Token ids outside [0, len) give unspecified
+ * results (they read a clamped row, never outside the cache). */
+int tw_topp_prune_tokens(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
+                         const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                         const int32_t* cand_tokens, int32_t cand_stride, const int32_t* ncand,
+                         double p, int32_t group_mode, int32_t* idx, int32_t capacity,
+                         int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
 /* One decode step: [tw_append_keys when append_keys != 0] -> tw_select_pages
  * (skipped when budget_tokens <= 0, every token is then a candidate) ->
  * tw_topp_prune -> tw_sparse_decode, enqueued back to back on one stream with
