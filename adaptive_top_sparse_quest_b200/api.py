@@ -402,6 +402,32 @@ def label_cache(kv: KVCache, channels: torch.Tensor, out: Optional[torch.Tensor]
     return out
 
 
+def _check_labels(kv: KVCache, labels: torch.Tensor, channels: torch.Tensor) -> int:
+    """Label cache and channels of a KV cache: fp16 rows of r values, int32
+    [Hk][r] channels.  Returns r."""
+    _need(labels, torch.float16, "labels")
+    _need(channels, torch.int32, "channels")
+    r = int(channels.shape[-1]) if channels.dim() == 2 else -1
+    if tuple(channels.shape) != (kv.Hk, r) or not 1 <= r <= 32:
+        raise ValueError(f"channels must be int32 [{kv.Hk}][r] with 1 <= r <= 32")
+    if tuple(labels.shape) != kv.row_shape(r):
+        raise ValueError(f"labels must be {kv.row_shape(r)}, got {tuple(labels.shape)}")
+    return r
+
+
+def _check_cand_tokens(kv: KVCache, cand: torch.Tensor, ncand: torch.Tensor) -> int:
+    """Token candidates [B][Hk][stride] and their counts [B][Hk] (int32).
+    Returns stride."""
+    _need(cand, torch.int32, "cand")
+    _need(ncand, torch.int32, "ncand")
+    stride = int(cand.shape[-1]) if cand.dim() == 3 else -1
+    if tuple(cand.shape) != (kv.B, kv.Hk, stride) or stride < 1:
+        raise ValueError(f"cand must be int32 [{kv.B}][{kv.Hk}][stride]")
+    if tuple(ncand.shape) != (kv.B, kv.Hk):
+        raise ValueError(f"ncand must be int32 [{kv.B}][{kv.Hk}]")
+    return stride
+
+
 def token_workspace_bytes(B, Hq, Hk, N, cand_stride, capacity, key_bits=4) -> int:
     lib = _capi.load()
     n = ctypes.c_size_t(0)
@@ -422,7 +448,7 @@ def select_tokens(q: torch.Tensor, kv: KVCache, labels: torch.Tensor, channels: 
     lib = _capi.load()
     _need(q, torch.float16, "q")
     Hq = int(q.shape[1])
-    r = int(channels.shape[-1])
+    r = _check_labels(kv, labels, channels)
     stride = max(1, min(int(budget_tokens), kv.N))
     cand = torch.zeros((kv.B, kv.Hk, stride), dtype=torch.int32, device=q.device)
     ncand = torch.zeros((kv.B, kv.Hk), dtype=torch.int32, device=q.device)
@@ -444,7 +470,7 @@ def topp_prune_tokens(q: torch.Tensor, kv: KVCache, keys: Int4Keys, cand: torch.
     _need(q, torch.float16, "q")
     _check_keys(kv, keys)
     Hq = int(q.shape[1])
-    stride = int(cand.shape[-1])
+    stride = _check_cand_tokens(kv, cand, ncand)
     capacity = stride if capacity is None else int(capacity)
     U = num_sets(kv, Hq, group_mode)
     idx = torch.zeros((U, capacity), dtype=torch.int32, device=q.device)
@@ -472,6 +498,7 @@ class LabelDecodeStep:
                  Hq: int, budget_tokens: int, p: float, group_mode: int = 0,
                  with_lse: bool = True):
         _check_keys(kv, keys)
+        _check_labels(kv, labels, channels)
         self.kv, self.keys, self.labels, self.channels = kv, keys, labels, channels
         self.Hq, self.budget, self.p, self.group_mode = Hq, int(budget_tokens), float(p), \
             int(group_mode)
