@@ -122,3 +122,23 @@ def test_group_weights_properties():
     # the group weight is the average, so it is between the per-head extremes
     per = np.stack([O.softmax_weights(l[:, h]) for h in range(4)], 1)
     assert np.all(w <= per.max(1) + 1e-15) and np.all(w >= per.min(1) - 1e-15)
+
+
+def test_group_weights_hand_worked_example():
+    """Hand-derived group weights and group top-p (tests/golden/
+    group_weights_worked_example.json): separates the mean of the per-head
+    normalised weights from the softmax of the mean logits."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "group_weights_worked_example.json")))
+    l = np.log(np.array(g["logits_ln"], np.float64))
+    w = O.group_weights(l)
+    np.testing.assert_allclose(w, np.array(g["expected_weights_num84"]) / 84.0, rtol=0, atol=1e-15)
+    for case in g["topp_cases"]:
+        sel = O.topp_select(w, case["p"])[0]
+        assert sel.tolist() == case["keep"], case
+    # the wrong reading keeps a different set at p = 0.40
+    wrong = O.softmax_weights(l.mean(1))
+    assert O.topp_select(wrong, 0.40)[0].tolist() == g["mean_logit_reading_keep_at_0_40"]
+    assert O.topp_select(w, 0.40)[0].tolist() != g["mean_logit_reading_keep_at_0_40"]
