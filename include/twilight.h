@@ -153,7 +153,13 @@ int tw_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                       int32_t max_seq_len, int32_t capacity, size_t* bytes);
 
 /*
- * Quest pre-selection (the base selector).  For each (b, KV head):
+ * Quest pre-selection (the base selector).  Twilight prunes on top of a base
+ * selector, and Quest is one of the two it builds on; Quest ranks 16-token
+ * pages by a bound computed from the page's per-channel key min / max (its
+ * max-pooled page layout is why Twilight's pruning is hierarchical:
+ * atlas.scime.ai summary, "Surprising findings"; "Builds on").  The pages give
+ * no formula; the bound below is Quest's published criterion.
+ * For each (b, KV head):
  *   score[pg] = sum over the G query heads of the group, in head order, of
  *               sum_j max(q_j * min_j, q_j * max_j)      (fp32, fixed order:
  *               16 chunks of 8 channels summed left to right, then chunk c
@@ -195,10 +201,14 @@ int tw_topp_prune(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
 
 /*
  * Exact attention over the selected tokens' fp16 K/V (split-K flash decoding
- * with a log-sum-exp merge).  For query head hq of sequence b, with S its
- * selection set: out = sum_{i in S} softmax(q . k_i / sqrt(128)) v_i (fp32
- * accumulation, fp16 result); lse[b][hq] = log sum exp (natural log).  An
- * empty set gives out = 0 and lse = -inf.  lse may be NULL.
+ * with a log-sum-exp merge).  After the base selector and the top-p pruner,
+ * attention runs over the surviving tokens only (atlas.scime.ai summary,
+ * "Approach": select, then prune, then sparse attention; the authors' kernels
+ * build on FlashInfer's sparse attention, "Experimental setup").  For query
+ * head hq of sequence b, with S its selection set:
+ *   out = sum_{i in S} softmax(q . k_i / sqrt(128)) v_i
+ * (fp32 accumulation, fp16 result); lse[b][hq] = log sum exp (natural log).
+ * An empty set gives out = 0 and lse = -inf.  lse may be NULL.
  */
 int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
                      const int32_t* idx, int32_t capacity, const int32_t* count,
