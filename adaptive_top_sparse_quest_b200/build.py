@@ -49,21 +49,48 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
+def _objdir() -> str:
+    return os.path.join(LIB_DIR, "obj")
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    """Compile every .cu under csrc/ into lib/libtwilight.so (sm_100a)."""
+    """Compile every .cu under csrc/ (one nvcc process per file, in parallel)
+    and link lib/libtwilight.so (sm_100a)."""
     if not force and up_to_date():
         return LIB
-    os.makedirs(LIB_DIR, exist_ok=True)
+    import concurrent.futures as cf
+    os.makedirs(_objdir(), exist_ok=True)
+    nvcc = _nvcc()
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    srcs = sources()
+
+    def one(src):
+        obj = os.path.join(_objdir(), os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc, *compile_flags, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-c",
+               "-o", obj, src]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, cmd, r
+
+    keep = {os.path.basename(x)[:-3] + ".o" for x in srcs}
+    for f in os.listdir(_objdir()):   # objects of sources that no longer exist
+        if f.endswith(".o") and f not in keep:
+            os.remove(os.path.join(_objdir(), f))
+    objs = []
+    with cf.ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        for src, obj, cmd, r in ex.map(one, srcs):
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            if r.returncode != 0:
+                raise RuntimeError(f"nvcc failed on {src}:\n" + r.stdout + r.stderr)
+            if verbose and (r.stdout or r.stderr):
+                print(r.stdout + r.stderr)
+            objs.append(obj)
     tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
-           "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), flush=True)
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
+           "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
-    if verbose and (r.stdout or r.stderr):
-        print(r.stdout + r.stderr)
+        raise RuntimeError("nvcc link failed:\n" + r.stdout + r.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -83,13 +83,16 @@ int check_heads(int Hq, int Hk) {
   return TW_OK;
 }
 
-// Workspace regions, in order: status word | page scores | first physical row
-// of each candidate page | logits | softmax statistics | physical rows of the
-// kept tokens | per-set completion counters | attention partial records.  The
-// status word collects device-side error bits (a bounded wait that gave up).
+// Workspace regions, in order: status word | logits of the selection sets
+// that exceed shared memory | score keys of caches too long for shared memory
+// | physical rows of the kept tokens | per-set completion counters |
+// attention partial records.  The status word collects device-side error bits
+// (a bounded wait that gave up); the caller zeroes it once after allocating.
+// tw_topp_prune uses the regions up to topp_end, tw_select_pages up to
+// scores_end.
 struct Plan {
-  size_t status_off, scores_off, row0_off, logits_off, stats_off, rows_off, done_off, part_off;
-  size_t scores_end, topp_end, total;
+  size_t status_off, logits_off, keys_off, rows_off, done_off, part_off;
+  size_t topp_end, scores_end, total;
   int lcap;
 };
 
@@ -97,17 +100,14 @@ Plan make_plan(int B, int Hq, int Hk, int N, int cap) {
   Plan p;
   const int G = Hq / Hk;
   const int64_t pmax = (N + tw::kPage - 1) / tw::kPage;
-  p.lcap = (int)(((int64_t)cap + tw::kEstTile - 1) / tw::kEstTile * tw::kEstTile);
+  p.lcap = (int)(((int64_t)cap + 63) / 64 * 64);
   p.status_off = 0;
-  p.scores_off = 256;
-  p.scores_end = p.scores_off + align256((size_t)B * Hk * pmax * sizeof(float));
-  p.row0_off = p.scores_end;
-  p.logits_off = p.row0_off + align256((size_t)B * Hk * pmax * sizeof(uint32_t));
-  p.stats_off = p.logits_off + align256((size_t)B * Hk * p.lcap * G * sizeof(float));
-  p.topp_end = p.stats_off +
-               align256((size_t)B * Hk * (p.lcap / tw::kStatSpan) * G * sizeof(float2));
+  p.logits_off = 256;
+  p.topp_end = p.logits_off + align256((size_t)B * Hk * G * (size_t)p.lcap * sizeof(float));
+  p.keys_off = p.topp_end;
+  p.scores_end = p.keys_off + align256((size_t)B * Hk * pmax * sizeof(uint32_t));
   const size_t nsets = (size_t)B * (Hq > Hk ? Hq : Hk);
-  p.rows_off = p.topp_end;
+  p.rows_off = p.scores_end;
   p.done_off = p.rows_off + align256(nsets * (size_t)cap * sizeof(uint32_t));
   p.part_off = p.done_off + align256(nsets * sizeof(int32_t));
   p.total = p.part_off + align256(tw::decode_part_floats(B, Hq, Hk) * sizeof(float));
@@ -200,6 +200,55 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 int group_sets_of(int Hq, int Hk, int group_mode) { return (group_mode || Hq == Hk) ? 1 : 0; }
 
+// Selection-stage arguments shared by every call: layout, query and the
+// workspace status word.
+tw::SpArgs sp_args(const tw::Layout& L, const uint16_t* q, int Hq, void* ws, const Plan& plan) {
+  tw::SpArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.L = L;
+  a.q = reinterpret_cast<const __half*>(q);
+  a.Hq = Hq;
+  a.status = reinterpret_cast<int*>(wsp(ws, plan.status_off));
+  return a;
+}
+
+void set_prune(tw::SpArgs* a, const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+               int group_sets, double p, int32_t* idx, uint32_t* rows, int icap, int32_t* count,
+               int32_t* done) {
+  a->codes = codes;
+  a->scales = reinterpret_cast<const __half*>(scales);
+  a->zeros = reinterpret_cast<const __half*>(zeros);
+  a->group_sets = group_sets;
+  a->p = p;
+  a->idx = idx;
+  a->rows = rows;
+  a->icap = icap;
+  a->count = count;
+  a->done = done;
+}
+
+// Candidate pages per unit at most: the Quest budget, the caller's list
+// stride, or every page.
+int selection_pages(const tw::SpArgs& a) {
+  const int mp = a.L.max_pages;
+  if (a.meta) return a.budget_pages < mp ? a.budget_pages : mp;
+  if (a.cand) return a.cand_stride < mp ? a.cand_stride : mp;
+  return mp;
+}
+
+// Launch the selection stages on one cluster per unit, with the keys and
+// logits in the workspace when they exceed shared memory.
+int run_select_prune(tw::SpArgs* a, void* ws, const Plan& plan, int sms, cudaStream_t st,
+                     bool pdl) {
+  const int sel = selection_pages(*a);
+  if (sel > tw::select_prune_max_pages()) return TW_ERR_UNSUPPORTED;
+  a->gkeys = reinterpret_cast<uint32_t*>(wsp(ws, plan.keys_off));
+  a->glogits = reinterpret_cast<float*>(wsp(ws, plan.logits_off));
+  a->lcap = plan.lcap;
+  const cudaError_t e = tw::launch_select_prune(*a, sel, sms, st, pdl);
+  return e == cudaSuccess ? TW_OK : cuda_fail(e);
+}
+
 // Device address of the page-locked host memory at p (allocated or registered
 // page-locked and mapped into the device's address space); nullptr for
 // pageable, device or unknown memory.
@@ -269,31 +318,20 @@ int decode_step_impl(const tw_step* s, void* const* events, int n_events, cudaSt
                                st, sms, pdl);
     if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   }
-  float* scores = reinterpret_cast<float*>(wsp(s->ws, plan.scores_off));
-  // physical rows: the selector writes the candidate pages' first rows, the
-  // top-p kernel the kept tokens' rows (without selection the estimate and
-  // top-p kernels compute page rows themselves)
-  uint32_t* row0 = use_select ? reinterpret_cast<uint32_t*>(wsp(s->ws, plan.row0_off)) : nullptr;
   uint32_t* rows = reinterpret_cast<uint32_t*>(wsp(s->ws, plan.rows_off));
-  if (use_select) {
-    e = tw::launch_page_scores(L, q, Hq, reinterpret_cast<const __half*>(s->meta), scores, st,
-                               sms, pdl);
-    if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
-    e = tw::launch_page_topk(L, scores, s->budget_tokens / tw::kPage, s->cand_pages,
-                             s->cand_stride, s->ncand, row0, st, pdl);
-    if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
-  }
-  float* logits = reinterpret_cast<float*>(wsp(s->ws, plan.logits_off));
-  float2* stats = reinterpret_cast<float2*>(wsp(s->ws, plan.stats_off));
-  const int cmax = candidates_max(L, cand, s->cand_stride);
-  e = tw::launch_estimate(L, q, Hq, s->codes, reinterpret_cast<const __half*>(s->scales),
-                          reinterpret_cast<const __half*>(s->zeros), cand, s->cand_stride,
-                          s->ncand, row0, plan.lcap, cmax, logits, stats, st, sms, pdl);
-  if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   int32_t* done = reinterpret_cast<int32_t*>(wsp(s->ws, plan.done_off));
-  e = tw::launch_topp(L, Hq, gs, cand, s->cand_stride, s->ncand, row0, plan.lcap, cmax, logits,
-                      stats, s->p, s->idx, rows, s->capacity, s->count, done, st, pdl);
-  if (e != cudaSuccess || (e = mk.mark()) != cudaSuccess) return cuda_fail(e);
+  tw::SpArgs a = sp_args(L, s->q, Hq, s->ws, plan);
+  if (use_select) {
+    a.meta = reinterpret_cast<const __half*>(s->meta);
+    a.budget_pages = s->budget_tokens / tw::kPage;
+    a.cand = s->cand_pages;
+    a.cand_stride = s->cand_stride;
+    a.ncand = s->ncand;
+  }
+  set_prune(&a, s->codes, s->scales, s->zeros, gs, s->p, s->idx, rows, s->capacity, s->count,
+            done);
+  TW_TRY(run_select_prune(&a, s->ws, plan, sms, st, pdl));
+  if ((e = mk.mark()) != cudaSuccess) return cuda_fail(e);
   float* part = reinterpret_cast<float*>(wsp(s->ws, plan.part_off));
   const auto* K = reinterpret_cast<const __half*>(s->kv.k);
   const auto* V = reinterpret_cast<const __half*>(s->kv.v);
@@ -320,7 +358,7 @@ TokenPlan make_token_plan(int B, int Hq, int Hk, int cand_stride, int capacity, 
   TokenPlan t;
   t.topp = make_plan(B * Hk, Hq / Hk, 1, cand_stride, capacity);
   const size_t rows = (size_t)B * Hk * cand_stride;
-  t.vcodes_off = align256(t.topp.topp_end);
+  t.vcodes_off = align256(t.topp.scores_end);
   t.vscales_off = t.vcodes_off + align256(rows * (size_t)(tw::kHeadDim * kbits / 8));
   t.vzeros_off = t.vscales_off + align256(rows * tw::kGroups * sizeof(uint16_t));
   t.total = t.vzeros_off + align256(rows * tw::kGroups * sizeof(uint16_t));
@@ -419,15 +457,13 @@ int tw_select_pages(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   TW_TRY(check_ws(ws, ws_bytes, plan.scores_end));
   int sms = 0;
   TW_TRY(device_check(&sms));
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* scores = reinterpret_cast<float*>(wsp(ws, plan.scores_off));
-  cudaError_t e = tw::launch_page_scores(L, reinterpret_cast<const __half*>(q), num_q_heads,
-                                         reinterpret_cast<const __half*>(meta), scores, st, sms,
-                                         false);
-  if (e == cudaSuccess)
-    e = tw::launch_page_topk(L, scores, budget_tokens / tw::kPage, cand_pages, cand_stride,
-                             ncand, nullptr, st, false);
-  if (e != cudaSuccess) return cuda_fail(e);
+  tw::SpArgs a = sp_args(L, q, num_q_heads, ws, plan);
+  a.meta = reinterpret_cast<const __half*>(meta);
+  a.budget_pages = budget_tokens / tw::kPage;
+  a.cand = cand_pages;
+  a.cand_stride = cand_stride;
+  a.ncand = ncand;
+  TW_TRY(run_select_prune(&a, ws, plan, sms, static_cast<cudaStream_t>(stream), false));
   return check_launch();
 }
 
@@ -445,24 +481,13 @@ int tw_topp_prune(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
   TW_TRY(check_ws(ws, ws_bytes, plan.topp_end));
   int sms = 0;
   TW_TRY(device_check(&sms));
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* logits = reinterpret_cast<float*>(wsp(ws, plan.logits_off));
-  float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.stats_off));
-  const int cmax = candidates_max(L, cand_pages, cand_stride);
-  // caller-given candidate pages: locate their rows first
-  uint32_t* row0 = cand_pages ? reinterpret_cast<uint32_t*>(wsp(ws, plan.row0_off)) : nullptr;
-  cudaError_t e = cudaSuccess;
-  if (cand_pages) e = tw::launch_resolve_pages(L, cand_pages, cand_stride, row0, st, false);
-  if (e == cudaSuccess)
-    e = tw::launch_estimate(L, reinterpret_cast<const __half*>(q), num_q_heads, codes,
-                            reinterpret_cast<const __half*>(scales),
-                            reinterpret_cast<const __half*>(zeros), cand_pages, cand_stride,
-                            ncand, row0, plan.lcap, cmax, logits, stats, st, sms, false);
-  if (e == cudaSuccess)
-    e = tw::launch_topp(L, num_q_heads, group_sets_of(num_q_heads, L.Hk, group_mode), cand_pages,
-                        cand_stride, ncand, row0, plan.lcap, cmax, logits, stats, p, idx,
-                        nullptr, capacity, count, nullptr, st, false);
-  if (e != cudaSuccess) return cuda_fail(e);
+  tw::SpArgs a = sp_args(L, q, num_q_heads, ws, plan);
+  a.cand = const_cast<int32_t*>(cand_pages);
+  a.cand_stride = cand_stride;
+  a.ncand = const_cast<int32_t*>(ncand);
+  set_prune(&a, codes, scales, zeros, group_sets_of(num_q_heads, L.Hk, group_mode), p, idx,
+            nullptr, capacity, count, nullptr);
+  TW_TRY(run_select_prune(&a, ws, plan, sms, static_cast<cudaStream_t>(stream), false));
   return check_launch();
 }
 
@@ -594,23 +619,19 @@ int tw_topp_prune_tokens(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv
   auto* vcodes = reinterpret_cast<uint8_t*>(wsp(ws, plan.vcodes_off));
   auto* vscales = reinterpret_cast<__half*>(wsp(ws, plan.vscales_off));
   auto* vzeros = reinterpret_cast<__half*>(wsp(ws, plan.vzeros_off));
-  float* logits = reinterpret_cast<float*>(wsp(ws, plan.topp.logits_off));
-  float2* stats = reinterpret_cast<float2*>(wsp(ws, plan.topp.stats_off));
   const int gs = group_sets_of(num_q_heads, L.Hk, group_mode);
   const int nsets = gs ? L.B * L.Hk : L.B * num_q_heads;
   cudaError_t e = tw::launch_gather_keys(L, cand_tokens, cand_stride, ncand, codes,
                                          reinterpret_cast<const __half*>(scales),
                                          reinterpret_cast<const __half*>(zeros), vcodes, vscales,
                                          vzeros, st, sms);
-  if (e == cudaSuccess)
-    e = tw::launch_estimate(Lv, reinterpret_cast<const __half*>(q), G, vcodes, vscales, vzeros,
-                            nullptr, 0, nullptr, nullptr, plan.topp.lcap, cand_stride, logits,
-                            stats, st, sms, false);
-  if (e == cudaSuccess)
-    e = tw::launch_topp(Lv, G, gs, nullptr, 0, nullptr, nullptr, plan.topp.lcap, cand_stride,
-                        logits, stats, p, idx, nullptr, capacity, count, nullptr, st, false);
-  if (e == cudaSuccess)
-    e = tw::launch_map_tokens(nsets, G, gs, cand_tokens, cand_stride, idx, capacity, count, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  tw::SpArgs a = sp_args(Lv, q, G, ws, plan.topp);
+  set_prune(&a, vcodes, reinterpret_cast<const uint16_t*>(vscales),
+            reinterpret_cast<const uint16_t*>(vzeros), gs, p, idx, nullptr, capacity, count,
+            nullptr);
+  TW_TRY(run_select_prune(&a, ws, plan.topp, sms, st, false));
+  e = tw::launch_map_tokens(nsets, G, gs, cand_tokens, cand_stride, idx, capacity, count, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
@@ -627,20 +648,17 @@ int tw_decode_step_host(const tw_step* step, const uint16_t* q_host, uint16_t* o
 
 int tw_decode_step_num_kernels(const tw_step* step) {
   if (!step) return -TW_ERR_INVALID_ARG;
-  return (step->budget_tokens > 0 ? 5 : 3) + (step->append_keys ? 1 : 0);
+  return 2 + (step->append_keys ? 1 : 0);
 }
 
 const char* tw_decode_step_kernel_name(const tw_step* step, int32_t i) {
-  static const char* with_select[5] = {"page_scores", "page_topk", "estimate", "topp",
-                                       "sparse_decode"};
-  static const char* no_select[3] = {"estimate", "topp", "sparse_decode"};
   if (!step) return nullptr;
   if (step->append_keys) {
     if (i == 0) return "append_keys";
     --i;
   }
-  if (step->budget_tokens > 0) return (i >= 0 && i < 5) ? with_select[i] : nullptr;
-  return (i >= 0 && i < 3) ? no_select[i] : nullptr;
+  if (i == 0) return step->budget_tokens > 0 ? "select_prune" : "prune";
+  return i == 1 ? "sparse_decode" : nullptr;
 }
 
 int tw_decode_step_profiled(const tw_step* step, void* const* events, int32_t n_events,

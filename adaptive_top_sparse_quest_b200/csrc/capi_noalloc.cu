@@ -5,18 +5,22 @@
 // records the decode step into a CUDA graph and forbids allocation while it
 // records, a plugin whose enqueue hook may not allocate, or an embedded
 // server that fixes its device memory at start-up.  This entry point takes the
-// same inputs and outputs as tw_topp_prune but keeps its scratch (logits and
-// softmax statistics) in one fixed array compiled into the library.
+// same inputs and outputs as tw_topp_prune but keeps its scratch (a status
+// word and the selection sets' logits) in one fixed array compiled into the
+// library.
 //
 // The array lives in device memory on every GPU that loads the library, for
 // the life of the process.  In host code its name stands for a host-side
 // placeholder, not a device address, so the first call on each device asks the
 // runtime for the array's device address with that device current and reuses
 // it afterwards.  That first call should therefore happen before any stream
-// capture.  All calls share the array, so calls whose work overlaps on the GPU
+// capture, and the cached address is valid for the life of the device's
+// primary context (a cudaDeviceReset between calls would leave it stale).
+// All calls share the array, so calls whose work overlaps on the GPU
 // (different streams, or different host threads) race on it; the array keeps
 // whatever the last call left in it, and nothing in it needs to start at zero
-// because every byte this call reads was written by the same call.
+// because every byte this call reads was written by the same call (the
+// status word is only ever or-ed into).
 #include <atomic>
 
 #include "twilight.h"

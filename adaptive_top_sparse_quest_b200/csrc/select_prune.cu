@@ -1,0 +1,1420 @@
+// Twilight's selection stages for one (sequence, KV head) unit on one
+// thread-block cluster: Quest page scores and top-K_p pages, then the
+// quantised-key weight estimate, the top-p threshold and the compaction of the
+// kept tokens.
+//
+// Method ("Twilight: Adaptive Attention Sparsity with Hierarchical Top-p
+// Pruning", atlas.scime.ai summary): a base selector pre-selects candidates
+// and top-p over the candidates' estimated attention weights prunes them
+// ("Approach"); Quest, the base selector here, ranks 16-token pages by a bound
+// from the page's per-channel key min / max ("Surprising findings", "Builds
+// on"); the weights are estimated from the 4-bit key cache ("Approach"; the
+// 2-bit cache of the quantisation ablation, table of measured effects, runs
+// through the same code); under GQA the budget is group-wise ("Limitations").
+//
+// Work split.  A unit is processed by one cluster of CS CTAs (CS = 1..16).
+//   Phase 1 (scores, top-K_p).  CTA r scores pages [r P / CS, (r+1) P / CS) of
+//   the unit's P pages: their 512-byte metadata records stream through a
+//   shared-memory ring filled by bulk copies.  Each page's score key is stored
+//   into every CTA's key array (distributed shared memory), so after one
+//   cluster barrier every CTA holds all P keys and runs the same radix select
+//   on its own: the K_p best pages (ties to the lower page) and their
+//   ascending order, with no further exchange.  CTA r then owns the share
+//   [r K_p / CS, (r+1) K_p / CS) of the candidate list.
+//   Phase 2 (estimate, top-p).  Each CTA streams its share's quantised key
+//   rows (whole 16-row pages) through a second ring, computes the logits of
+//   every query head of the group on the tensor cores (mma.sync, codes as the
+//   A operand) into shared memory and keeps per-head (max, sum 2^(l - max)).
+//   One exchange of those pairs gives every CTA the unit's softmax statistics.
+//   Each thread then holds the weights of R consecutive candidates of its
+//   CTA's share in registers, and the threshold is found most significant
+//   digit first (12 + 9 + 9 bits of the fp32 weight) over exact integer
+//   masses; the CTAs reduce-scatter their digit histograms through
+//   distributed shared memory.  The kept tokens are compacted in ascending
+//   order with their physical K/V rows for the attention kernel.
+//
+// The score of a page is a deterministic fp32 sum in one fixed order, so the
+// selected page ids are an exact integer result: products of two fp16 values
+// are exact in fp32; each lane of a half-warp sums its 8 channels left to
+// right; the 16 lane sums are combined by xor-butterfly 8, 4, 2, 1 (fp32
+// addition is commutative, so both butterfly partners hold the same value);
+// the group's heads are added in head order.  Each channel's bound term
+// max(q min, q max) equals q+ max + q- min with q+ = max(q, 0), q- = min(q, 0)
+// (one of the two products is zero), so it is accumulated with two fused
+// multiply-adds whose single rounding is the rounding of the sum.
+//
+// Streaming: cp.async.bulk copies complete on a stage's "full" mbarrier
+// together with their byte count; the consumer warps release the stage on
+// its "empty" mbarrier and warp 0 refills it.  The scales and zeros of the
+// quantised rows (8 bytes per row, whose start need not be 16-byte aligned in
+// a contiguous cache) arrive by 8-byte cp.async that signal the same full
+// mbarrier.  No copy uses cluster multicast.  Every wait is bounded
+// (tw_bulk.cuh).
+#include "tw_bulk.cuh"
+#include "tw_common.cuh"
+#include "tw_kernels.h"
+
+namespace tw {
+
+constexpr int kSpWarps = kSpThreads / 32;
+constexpr int kMetaStagePages = 32;                      // 16 KB of page records per stage
+constexpr int kMetaStageBytes = kMetaStagePages * 2 * kHeadDim * 2;
+constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
+constexpr int kEstStageTok = kEstStagePages * kPage;
+constexpr int kSpBins = 4096;                            // first digit of the searches: 12 bits
+constexpr int kSpBinList = 32;                           // a first-digit bin this small is resolved directly
+constexpr float kEstL2Scale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
+constexpr double kSpMassEps = 1e-12;           // exact ties at p resolve as in real arithmetic
+constexpr float kSpMassScale = 1099511627776.0f;   // 2^40
+
+template <int BITS>
+struct SpKeyWidth {
+  static_assert(BITS == 4 || BITS == 2, "key-cache width");
+  static constexpr int kRowBytes = kHeadDim * BITS / 8;
+  static constexpr int kLaneBytes = kGroup * BITS / 8;
+  static constexpr float kCentre = BITS == 4 ? 8.f : 2.f;
+  static constexpr int kStageBytes = kEstStageTok * (kRowBytes + 2 * kGroups * 2);
+  // channel that feeds MMA k-slot pair j, element hi, at K-step s (offset in the lane's group)
+  __device__ static constexpr int chan(int s, int j, int hi) {
+    return BITS == 4 ? 8 * (s >> 1) + 2 * (s & 1) + j + 4 * hi
+                     : 16 * (s >> 2) + 2 * (s & 3) + j + 8 * hi;
+  }
+};
+
+// Fixed part of the shared memory; the phase regions follow it.
+struct SpFixed {
+  uint64_t full1[kSpMaxStages], empty1[kSpMaxStages];
+  uint64_t full2[kSpMaxStages], empty2[kSpMaxStages];
+  uint32_t pg[kSpSharePages];     // this CTA's share of the candidate list: page ids
+  uint32_t r0[kSpSharePages];     // first physical row of each page
+  int32_t nrow[kSpSharePages];    // valid rows of each page (0: not a page of the sequence)
+  float2 wstat[kSpWarps][8];      // per warp and head: (max, sum 2^(l - max))
+  float2 mz_loc[8];               // this CTA's pair per head
+  float2 mz_all[kSpMaxCluster][8];   // every CTA's pair per head
+  unsigned long long wsuf[kSpWarps];
+  unsigned long long slice_tot;
+  unsigned long long sh_above;
+  int sh_d;
+  int sh_need;
+  uint32_t sh_pref;
+  int2 scan2[kSpWarps + 1];
+  unsigned scan[kSpWarps + 1];
+  uint32_t wmin[kSpWarps], wmax[kSpWarps];
+  unsigned blk[2];
+  unsigned pre[4];
+  uint32_t lst_key[kSpBinList];   // the weights of the threshold's first-digit bin
+  uint32_t lst_pos[kSpBinList];   // and their positions in the set
+  int lst_n;
+  uint32_t res_theta;
+  unsigned long long res_need;
+};
+
+constexpr size_t kSpFixedBytes = (sizeof(SpFixed) + 127) / 128 * 128;
+
+size_t sp_fixed_bytes() { return kSpFixedBytes; }
+
+__device__ __forceinline__ void cp_async8_sm(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+
+// All of this thread's earlier cp.async arrive on `bar` when they complete.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory index of element i of an array padded by one word per 32:
+// a thread's run of E consecutive elements (E <= 32) is then conflict-free
+// when the threads of a warp read their runs in step.
+__host__ __device__ __forceinline__ int sp_pad(int i) { return i + (i >> 5); }
+
+__device__ __forceinline__ float sp_h(uint32_t w, int hi) {
+  return __half2float(__ushort_as_half((unsigned short)((w >> (16 * hi)) & 0xFFFFu)));
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide scans over the 256 threads (all threads call them).
+
+__device__ __forceinline__ int2 sp_scan2(int2 v, int2* sh, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int2 incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int tx = __shfl_up_sync(0xffffffffu, incl.x, o);
+    const int ty = __shfl_up_sync(0xffffffffu, incl.y, o);
+    if (lane >= o) {
+      incl.x += tx;
+      incl.y += ty;
+    }
+  }
+  __syncthreads();   // sh is free
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  int2 before = make_int2(0, 0), tot = make_int2(0, 0);
+#pragma unroll
+  for (int w = 0; w < kSpWarps; ++w) {
+    const int2 x = sh[w];
+    if (w < warp) {
+      before.x += x.x;
+      before.y += x.y;
+    }
+    tot.x += x.x;
+    tot.y += x.y;
+  }
+  *total = tot;
+  return make_int2(before.x + incl.x - v.x, before.y + incl.y - v.y);
+}
+
+__device__ __forceinline__ unsigned sp_scan(unsigned v, unsigned* sh, unsigned* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  __syncthreads();
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  unsigned before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kSpWarps; ++w) {
+    const unsigned x = sh[w];
+    if (w < warp) before += x;
+    tot += x;
+  }
+  *total = tot;
+  return before + incl - v;
+}
+
+// ---------------------------------------------------------------------------
+// Phase 1: Quest page scores of this CTA's slice, keys to every CTA.
+
+// One page's score: this lane's 8 channels of the min and max rows, the
+// query channels of the group's heads (q+ / q- split for G <= 4, plain q for
+// G = 8), the fixed summation order.
+template <int G>
+struct ScoreQ {
+  static constexpr bool kSplit = G <= 4;
+  float a[G][8];   // q+ (split) or q
+  float c[kSplit ? G : 1][8];   // q- (split)
+};
+
+template <int G>
+__device__ __forceinline__ float page_score(const ScoreQ<G>& Q, uint4 mn4, uint4 mx4,
+                                            unsigned hmask) {
+  const uint32_t wn[4] = {mn4.x, mn4.y, mn4.z, mn4.w};
+  const uint32_t wx[4] = {mx4.x, mx4.y, mx4.z, mx4.w};
+  float mn[8], mx[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    mn[j] = sp_h(wn[j >> 1], j & 1);
+    mx[j] = sp_h(wx[j >> 1], j & 1);
+  }
+  float total = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float s;
+    if (ScoreQ<G>::kSplit) {
+      s = __fmul_rn(Q.a[g][0], mx[0]);
+      s = __fmaf_rn(Q.c[ScoreQ<G>::kSplit ? g : 0][0], mn[0], s);
+#pragma unroll
+      for (int j = 1; j < 8; ++j) {
+        s = __fmaf_rn(Q.a[g][j], mx[j], s);
+        s = __fmaf_rn(Q.c[ScoreQ<G>::kSplit ? g : 0][j], mn[j], s);
+      }
+    } else {
+      s = fmaxf(__fmul_rn(Q.a[g][0], mn[0]), __fmul_rn(Q.a[g][0], mx[0]));
+#pragma unroll
+      for (int j = 1; j < 8; ++j)
+        s = __fadd_rn(s, fmaxf(__fmul_rn(Q.a[g][j], mn[j]), __fmul_rn(Q.a[g][j], mx[j])));
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(hmask, s, o, 16));
+    total = (g == 0) ? s : __fadd_rn(total, s);
+  }
+  return total;
+}
+
+// Radix select of the K largest of P keys (ties to the lower index), by the
+// whole CTA: returns through fx the threshold key and the number of keys
+// equal to it that are kept (the lowest-index ones).  Thread t owns the E
+// consecutive keys [t E, t E + E).  hist: kSpBins ints, zero on entry and exit.
+template <typename KeyAt>
+__device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& fx) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = (P + kSpThreads - 1) / kSpThreads;
+  const int i0 = tid * E, i1 = min(P, i0 + E);
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll 1
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = key_at(i);
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    fx.wmin[warp] = kmin;
+    fx.wmax[warp] = kmax;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kSpWarps; ++w) {
+    kmin = min(kmin, fx.wmin[w]);
+    kmax = max(kmax, fx.wmax[w]);
+  }
+  // the keys share the bits above the highest bit where the smallest and
+  // largest differ; the digits start below that common prefix
+  int nb = 32 - __clz((int)(kmin ^ kmax));
+  uint32_t pmask = nb >= 32 ? 0u : ~((1u << nb) - 1u);
+  uint32_t prefix = kmin & pmask;
+  int need = K;
+#pragma unroll 1
+  for (int round = 0; nb > 0; ++round) {
+    const int width = min(round == 0 ? 12 : 10, nb);
+    const int shift = nb - width;
+    const uint32_t dm = (1u << width) - 1u;
+    nb = shift;
+#pragma unroll 1
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = key_at(i);
+      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dm], 1);
+    }
+    __syncthreads();
+    // thread t holds digits [t bpt, t bpt + bpt); suffix sums from the top
+    const int bins = 1 << width;
+    const int bpt = bins > kSpThreads ? bins / kSpThreads : 1;
+    const bool holder = tid * bpt < bins;
+    int mine = 0;
+    if (holder) {
+#pragma unroll 1
+      for (int k = 0; k < bpt; ++k) mine += hist[tid * bpt + k];
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += t;
+    }
+    if (lane == 0) fx.scan2[warp].x = incl;
+    __syncthreads();
+    int above = incl - mine;
+#pragma unroll
+    for (int w = 0; w < kSpWarps; ++w)
+      if (w > warp) above += fx.scan2[w].x;
+    // the digit d of the K-th largest key: suffix(d) >= need > suffix(d + 1);
+    // when the keys of that digit are exactly the ones still needed, all of
+    // them are kept and the search ends here
+    if (holder) {
+#pragma unroll 1
+      for (int k = bpt - 1; k >= 0; --k) {
+        const int d = tid * bpt + k;
+        const int here = above + hist[d];
+        if (here >= need && above < need) {
+          fx.sh_d = d;
+          fx.sh_need = above;
+          fx.blk[0] = here == need ? 1u : 0u;
+        }
+        above = here;
+      }
+    }
+    __syncthreads();   // every thread is done reading the histogram
+    if (holder) {
+#pragma unroll 1
+      for (int k = 0; k < bpt; ++k) hist[tid * bpt + k] = 0;
+    }
+    need -= fx.sh_need;
+    prefix |= (uint32_t)fx.sh_d << shift;
+    pmask |= dm << shift;
+    const bool whole = fx.blk[0] != 0u;
+    __syncthreads();   // sh_d / sh_need / scan2 / blk are rewritten by the next round
+    if (whole) {   // keep every key >= prefix: the keys equal to it count as ties, all taken
+      need = 0x7FFFFFFF;
+      break;
+    }
+  }
+  if (tid == 0) {
+    fx.sh_pref = prefix;
+    fx.sh_need = need;
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Phase 2 helpers: MMA fragments of the estimate.
+
+__device__ __forceinline__ void sp_mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                            uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Nibbles e and e+4 of W as the half2 (c_e - 8, c_{e+4} - 8), exact.
+__device__ __forceinline__ uint32_t sp_nib_pair(uint32_t W, int e) {
+  uint32_t x = ((W >> (4 * e)) & 0x000F000Fu) | 0x64006400u;   // (1024 + c) as fp16
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64086408u));   // minus 1032
+  return r;
+}
+
+// 2-bit codes m and m+8 of W as the half2 (c_m - 2, c_{m+8} - 2), exact.
+__device__ __forceinline__ uint32_t sp_crumb_pair(uint32_t W, int m) {
+  uint32_t x = ((W >> (2 * m)) & 0x00030003u) | 0x64006400u;
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64026402u));   // minus 1026
+  return r;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t sp_code_pair(const uint32_t* W, int s, int j) {
+  if (BITS == 4) return sp_nib_pair(W[s >> 1], 2 * (s & 1) + j);
+  return sp_crumb_pair(W[s >> 2], 2 * (s & 3) + j);
+}
+
+__device__ __forceinline__ uint32_t sp_pack_h2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+// ---------------------------------------------------------------------------
+// Phase 2: the threshold search.
+
+struct SpSearch {
+  uint32_t prefix, pmask;
+  unsigned long long A, T;   // mass above the prefix range; target mass
+};
+
+__device__ __forceinline__ unsigned long long sp_mass(float w) {
+  return __float2ull_rz(w * kSpMassScale);
+}
+
+__device__ __forceinline__ unsigned long long sp_join(uint32_t hi, uint32_t lo) {
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// The weights of a selection set live in shared (or global) memory at
+// wbuf[wi(lp)] for the CTA's local positions lp; thread t owns the R
+// consecutive positions [t R, t R + R) (-1 marks an invalid position).
+struct SpWeights {
+  float* base;
+  bool pad;   // shared-memory positions padded one word per 32
+  int lp0, R, npos;
+  __device__ __forceinline__ float at(int i) const {
+    const int lp = lp0 + i;
+    return base[pad ? sp_pad(lp) : lp];
+  }
+};
+
+// Histogram the masses of this thread's weights that lie in the current
+// prefix range by digit (key >> shift) & dm: exact 64-bit sums from native
+// 32-bit atomics on a low and a high word with an explicit carry.
+__device__ __forceinline__ void mass_hist(const SpWeights& W, int shift, uint32_t dm,
+                                          const SpSearch& s, uint32_t* hlo, uint32_t* hhi) {
+#pragma unroll 1
+  for (int i = 0; i < W.R; ++i) {
+    if (W.lp0 + i >= W.npos) break;
+    const float w = W.at(i);
+    if (w >= 0.f) {
+      const uint32_t key = __float_as_uint(w);
+      if ((key & s.pmask) == s.prefix) {
+        const unsigned long long F = sp_mass(w);
+        const uint32_t dg = (key >> shift) & dm;
+        const uint32_t lo = (uint32_t)F;
+        const uint32_t old = atomicAdd(&hlo[dg], lo);
+        const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
+        if (up) atomicAdd(&hhi[dg], up);
+      }
+    }
+  }
+}
+
+// Mass of digit d summed over every CTA of the cluster (the CTAs' words are
+// requested before any is added).
+__device__ __forceinline__ unsigned long long cluster_bin(const uint32_t* hlo,
+                                                          const uint32_t* hhi, int d, int CS) {
+  uint32_t lv[kSpMaxCluster], hv[kSpMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kSpMaxCluster; ++r) {
+    lv[r] = hv[r] = 0u;
+    if (r < CS) {
+      lv[r] = ld_peer_u32(peer_addr(&hlo[d], r));
+      hv[r] = ld_peer_u32(peer_addr(&hhi[d], r));
+    }
+  }
+  unsigned long long t = 0;
+#pragma unroll
+  for (int r = 0; r < kSpMaxCluster; ++r) t += sp_join(hv[r], lv[r]);
+  return t;
+}
+
+// One digit of the threshold search (NB digits; NB = 4096 for the first).
+// CTA cr owns the slice [cr NB / CS, (cr + 1) NB / CS) of the digits; thread t
+// of it reduces bpt consecutive digits of the slice, summed over every CTA of
+// the cluster (CS = 1: its own histogram only) and written back over this
+// CTA's own words of those digits (no peer reads them).  The mass scan runs
+// from the top digit down; the one thread whose digit holds the crossing of
+// the target writes it into every CTA.  The first step also sets the target
+// from the total mass and returns false if that is zero.  Leaves this CTA's
+// histogram zeroed.
+__device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, double p, int CS,
+                           int cr, uint32_t* hlo, uint32_t* hhi, SpFixed& fx, SpSearch& s) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  mass_hist(W, shift, dm, s, hlo, hhi);
+  if (CS > 1) cluster_sync();   // every CTA's histogram is complete
+  else __syncthreads();
+  const int SB = NB / CS;                                    // digits of this CTA's slice
+  const int bpt = SB > kSpThreads ? SB / kSpThreads : 1;     // digits per thread (<= 16)
+  const int first = cr * SB + tid * bpt;
+  const bool holder = tid * bpt < SB;
+  unsigned long long mine = 0;   // this thread's digits' mass
+  if (holder) {
+#pragma unroll 1
+    for (int k = 0; k < bpt; ++k) {
+      const int d = first + k;
+      const unsigned long long v = CS == 1 ? sp_join(hhi[d], hlo[d]) : cluster_bin(hlo, hhi, d, CS);
+      if (CS > 1) {
+        hlo[d] = (uint32_t)v;
+        hhi[d] = (uint32_t)(v >> 32);
+      }
+      mine += v;
+    }
+  }
+  unsigned long long incl = mine;   // suffix over this warp's higher lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  if (lane == 0) fx.wsuf[warp] = incl;
+  __syncthreads();
+  unsigned long long after = incl - mine;   // digits of this slice above this thread's
+  unsigned long long slice = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kSpWarps; ++w2) {
+    const unsigned long long x = fx.wsuf[w2];
+    slice += x;
+    if (w2 > warp) after += x;
+  }
+  unsigned long long total = slice, higher = 0;
+  if (CS > 1) {
+    if (tid == 0) fx.slice_tot = slice;
+    cluster_sync();   // slice totals published; no peer reads this CTA's histogram any more
+    unsigned long long tots[kSpMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kSpMaxCluster; ++r)
+      tots[r] = r < CS ? ld_peer_u64(peer_addr(&fx.slice_tot, r)) : 0ull;
+    total = 0;
+#pragma unroll
+    for (int r = 0; r < kSpMaxCluster; ++r) {
+      total += tots[r];
+      if (r > cr) higher += tots[r];
+    }
+  }
+  bool ok = true;
+  if (NB == kSpBins) {
+    if (total == 0) {
+      ok = false;
+    } else {
+      const double tf = ceil((p - kSpMassEps) * (double)total);
+      unsigned long long T = tf < 1.0 ? 1ull : (unsigned long long)tf;
+      s.T = T > total ? total : T;
+    }
+  }
+  if (ok && holder) {
+    // the digit d with A + suffix(d) >= T > A + suffix(d + 1); one thread holds it
+    unsigned long long above = s.A + higher + after;
+#pragma unroll 1
+    for (int k = bpt - 1; k >= 0; --k) {
+      const int d = first + k;
+      const unsigned long long here = above + sp_join(hhi[d], hlo[d]);
+      if (here >= s.T && above < s.T) {
+        for (int r = 0; r < CS; ++r) {
+          st_peer_u32(peer_addr(&fx.sh_d, r), (uint32_t)d);
+          st_peer_u64(peer_addr(&fx.sh_above, r), above - s.A);
+        }
+      }
+      above = here;
+    }
+  }
+  __syncthreads();   // every thread is done with the histogram words it holds
+  for (int i = tid; i < NB; i += kSpThreads) hlo[i] = hhi[i] = 0u;
+  if (CS > 1) cluster_sync();   // the digit is in every CTA's shared memory
+  else __syncthreads();
+  if (ok) {
+    s.A += fx.sh_above;
+    s.prefix |= (uint32_t)fx.sh_d << shift;
+    s.pmask |= dm << shift;
+  }
+  __syncthreads();   // sh_d / sh_above / wsuf are rewritten by the next step
+  return ok;
+}
+
+// After the first digit: when the weights inside the threshold's digit (over
+// the whole cluster) number at most kSpBinList, gather them into every CTA
+// and resolve the threshold directly.  Sorted by weight descending, ties by
+// ascending set position, the cut is the first weight at which the mass above
+// the digit plus the running mass reaches the target; theta is its value and
+// r_need the number of weights equal to it up to and including it (the same
+// theta and tie count as the remaining digit steps would give).  Returns
+// false (the same in every CTA) when the digit holds more weights.  pos0:
+// this CTA's first set position.
+__device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos0, int CS,
+                                  SpFixed& fx, uint32_t* theta, unsigned long long* r_need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) fx.lst_n = 0;
+  __syncthreads();
+#pragma unroll 1
+  for (int i = 0; i < W.R; ++i) {
+    if (W.lp0 + i >= W.npos) break;
+    const float w = W.at(i);
+    if (w < 0.f) continue;
+    const uint32_t key = __float_as_uint(w);
+    if ((key & s.pmask) == s.prefix) {
+      const int slot = atomicAdd(&fx.lst_n, 1);
+      if (slot < kSpBinList) {
+        fx.lst_key[slot] = key;
+        fx.lst_pos[slot] = (uint32_t)(pos0 + W.lp0 + i);
+      }
+    }
+  }
+  if (CS > 1) cluster_sync();   // every CTA's list is complete
+  else __syncthreads();
+  // every CTA's count (lanes r < CS), and the gathered list in warp 0
+  int cnt = 0;
+  if (lane < CS) cnt = (int)ld_peer_u32(peer_addr(&fx.lst_n, (uint32_t)lane));
+  int before = cnt;   // inclusive prefix over the CTAs
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, before, o);
+    if (lane >= o) before += t;
+  }
+  const int n = __shfl_sync(0xffffffffu, before, 31);
+  const bool over = __any_sync(0xffffffffu, cnt > kSpBinList);
+  const bool small = !over && n <= kSpBinList;
+  if (small && warp == 0) {
+    // lane i < n takes element i of the concatenated lists (CTA r holds
+    // elements [before_r - cnt_r, before_r))
+    uint32_t key = 0, pos = 0xFFFFFFFFu;
+    const bool mine = lane < n;
+    int src = 0, start = 0;
+#pragma unroll 1
+    for (int r = 0; r < CS; ++r) {
+      const int end = __shfl_sync(0xffffffffu, before, r);
+      const int c = __shfl_sync(0xffffffffu, cnt, r);
+      if (lane >= end - c && lane < end) {
+        src = r;
+        start = end - c;
+      }
+    }
+    if (mine) {
+      key = ld_peer_u32(peer_addr(&fx.lst_key[lane - start], (uint32_t)src));
+      pos = ld_peer_u32(peer_addr(&fx.lst_pos[lane - start], (uint32_t)src));
+    }
+    // rank in the order (weight descending, position ascending)
+    int rank = 0;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+      const uint32_t pj = __shfl_sync(0xffffffffu, pos, j);
+      if (j < n && mine && (kj > key || (kj == key && pj < pos))) ++rank;
+    }
+    const unsigned long long F = mine ? sp_mass(__uint_as_float(key)) : 0ull;
+    unsigned long long cum = s.A;   // mass above the digit plus every weight up to this one
+    int ties = 0;                   // weights equal to this one up to and including it
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+      const int rj = __shfl_sync(0xffffffffu, rank, j);
+      const unsigned long long Fj = __shfl_sync(0xffffffffu, F, j);
+      const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+      if (j < n && mine && rj <= rank) {
+        cum += Fj;
+        if (kj == key) ++ties;
+      }
+    }
+    const bool cut = mine && cum >= s.T && cum - F < s.T;
+    if (cut) {
+      fx.res_theta = key;
+      fx.res_need = (unsigned long long)ties;
+    }
+  }
+  __syncthreads();
+  *theta = fx.res_theta;
+  *r_need = fx.res_need;
+  return small;
+}
+
+// ---------------------------------------------------------------------------
+template <int G, int BITS>
+__global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
+  using KW = SpKeyWidth<BITS>;
+  extern __shared__ __align__(128) unsigned char sp_smem[];
+  SpFixed& fx = *reinterpret_cast<SpFixed*>(sp_smem);
+  unsigned char* region = sp_smem + kSpFixedBytes;
+  const Layout& L = a.L;
+  const int CS = (int)cluster_size(), cr = (int)cluster_rank();
+  const int u = blockIdx.x / CS;
+  const int b = u / L.Hk, hk = u % L.Hk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool do_select = a.meta != nullptr, do_prune = a.codes != nullptr;
+  const bool paged = L.page_table != nullptr;
+  if (tid == 0) {
+    for (int s = 0; s < kSpMaxStages; ++s) {
+      mbar_init(&fx.full1[s], 1);
+      mbar_init(&fx.empty1[s], kSpWarps);
+      mbar_init(&fx.full2[s], 1 + 32);   // the byte-count arrival + warp 0's cp.async arrivals
+      mbar_init(&fx.empty2[s], kSpWarps);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  const int len = L.len(b);
+  const int P = (len + kPage - 1) / kPage;
+  int nsel = 0;          // candidate pages of the unit
+  int s0 = 0, ns = 0;    // this CTA's share: list entries [s0, s0 + ns)
+  bool failed = false;
+
+  if (do_select) {
+    // ---------------- phase 1: page scores of pages [pA, pB) ----------------
+    const int pA = (int)((int64_t)cr * P / CS), pB = (int)((int64_t)(cr + 1) * P / CS);
+    const int npg = pB - pA;
+    const int nst = (npg + kMetaStagePages - 1) / kMetaStagePages;
+    unsigned char* ring = region;
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(region + (size_t)a.s1 * kMetaStageBytes);
+    const bool gk = a.gkeys != nullptr;   // keys in global memory (P above the shared capacity)
+    uint32_t* gkeys = gk ? a.gkeys + (int64_t)u * L.max_pages : nullptr;
+    const __half* meta = a.meta;
+    const int64_t meta_unit = (int64_t)u * L.max_pages;   // contiguous record index of page 0
+    auto pt_of = [&](int k) -> int {   // warp 0: page-table entry of page lane of stage k
+      const int pg = pA + k * kMetaStagePages + lane;
+      if (!paged || k >= nst || pg >= pB) return 0;
+      const int e = L.page_table[(int64_t)b * L.max_pages + pg];
+      return (unsigned)e < (unsigned)L.pool_pages ? e : 0;
+    };
+    auto issue1 = [&](int k, int slot, int ptv) {   // warp 0
+      const int n = min(kMetaStagePages, npg - k * kMetaStagePages);
+      unsigned char* dst = ring + (size_t)slot * kMetaStageBytes;
+      if (paged) {
+        if (lane < n)
+          bulk_g2s(dst + lane * 512, meta + ((int64_t)ptv * L.Hk + hk) * (2 * kHeadDim), 512,
+                   &fx.full1[slot]);
+      } else if (lane == 0) {
+        bulk_g2s(dst, meta + (meta_unit + pA + (int64_t)k * kMetaStagePages) * (2 * kHeadDim),
+                 (uint32_t)n * 512u, &fx.full1[slot]);
+      }
+      if (lane == 0) mbar_arrive_tx(&fx.full1[slot], (uint32_t)n * 512u);
+    };
+    int ptn = 0;
+    if (warp == 0) {
+      int ptq[kSpMaxStages];
+#pragma unroll
+      for (int k = 0; k < kSpMaxStages; ++k) ptq[k] = (k < a.s1) ? pt_of(k) : 0;
+#pragma unroll
+      for (int k = 0; k < kSpMaxStages; ++k)
+        if (k < a.s1 && k < nst) issue1(k, k, ptq[k]);
+      ptn = pt_of(a.s1);
+    }
+    // the query channels of this lane (8 per head) for the group's heads
+    const int l16 = lane & 15, hw = tid >> 4;
+    const unsigned hmask = 0xFFFFu << (lane & 16);
+    ScoreQ<G> Q;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint4 r = __ldg(reinterpret_cast<const uint4*>(
+          a.q + ((int64_t)b * a.Hq + hk * G + g) * kHeadDim + l16 * 8));
+      const uint32_t wq[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float x = sp_h(wq[j >> 1], j & 1);
+        if (ScoreQ<G>::kSplit) {
+          Q.a[g][j] = x >= 0.f ? x : 0.f;
+          Q.c[ScoreQ<G>::kSplit ? g : 0][j] = x >= 0.f ? 0.f : x;
+        } else {
+          Q.a[g][j] = x;
+        }
+      }
+    }
+    for (int j = 0; j < nst; ++j) {
+      const int slot = j % a.s1;
+      const uint32_t par = (uint32_t)((j / a.s1) & 1);
+      if (!failed) failed = !mbar_wait(&fx.full1[slot], par, a.status);
+      const int n = min(kMetaStagePages, npg - j * kMetaStagePages);
+      const unsigned char* st = ring + (size_t)slot * kMetaStageBytes;
+#pragma unroll
+      for (int k = 0; k < kMetaStagePages / 16; ++k) {
+        const int i = hw + 16 * k;
+        if (i < n) {   // uniform across the half-warp
+          const uint4* rec = reinterpret_cast<const uint4*>(st + i * 512);
+          const float score = page_score<G>(Q, rec[l16], rec[16 + l16], hmask);
+          const uint32_t key = f_key(score);
+          const int pg = pA + j * kMetaStagePages + i;
+          if (gk) {
+            if (l16 == 0) gkeys[pg] = key;
+          } else if (l16 < CS) {
+            st_peer_u32(peer_addr(&skeys[sp_pad(pg)], (uint32_t)l16), key);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&fx.empty1[slot]);
+      if (warp == 0 && j + a.s1 < nst) {
+        if (!failed) failed = !mbar_wait(&fx.empty1[slot], par, a.status);
+        issue1(j + a.s1, slot, ptn);
+        ptn = pt_of(j + a.s1 + 1);
+      }
+    }
+    cluster_sync();   // every CTA holds all P keys (or they are in global memory)
+
+    // ---------------- top-K_p and this CTA's share of the candidate list ----------------
+    const int K = min(a.budget_pages, P);
+    auto key_at = [&](int i) -> uint32_t { return gk ? __ldcg(gkeys + i) : skeys[sp_pad(i)]; };
+    int* hist = reinterpret_cast<int*>(ring);   // the meta ring is idle now
+    for (int i = tid; i < kSpBins; i += kSpThreads) hist[i] = 0;
+    __syncthreads();
+    const bool all = K >= P;
+    if (!all) topk_threshold(key_at, P, K, hist, fx);
+    const uint32_t thr = all ? 0u : fx.sh_pref;
+    const int need = all ? 0 : fx.sh_need;
+    const int E = (P + kSpThreads - 1) / kSpThreads;
+    const int i0 = tid * E, i1 = min(P, i0 + E);
+    int n_gt = 0, n_eq = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = all ? 1u : key_at(i);
+      if (all || k > thr) ++n_gt;
+      else if (k == thr) ++n_eq;
+    }
+    int2 tot;
+    const int2 ex = sp_scan2(make_int2(n_gt, n_eq), fx.scan2, &tot);
+    nsel = K;
+    s0 = (int)((int64_t)cr * K / CS);
+    ns = (int)((int64_t)(cr + 1) * K / CS) - s0;
+    int take = ex.y < need ? min(n_eq, need - ex.y) : 0;
+    int pos = ex.x + min(need, ex.y);
+    int32_t* cand_u = a.cand + (int64_t)u * a.cand_stride;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = all ? 1u : key_at(i);
+      bool sel = all || k > thr;
+      if (!sel && k == thr && take > 0) {
+        sel = true;
+        --take;
+      }
+      if (sel) {
+        if (pos >= s0 && pos < s0 + ns) {
+          fx.pg[pos - s0] = (uint32_t)i;
+          cand_u[pos] = i;
+        }
+        ++pos;
+      }
+    }
+    if (cr == 0 && tid == 0) a.ncand[u] = K;
+    __syncthreads();
+  } else {
+    // ---------------- caller's candidate pages, or every page ----------------
+    if (a.cand) {
+      const int lim = min(a.cand_stride, L.max_pages);
+      nsel = max(0, min(a.ncand[u], lim));
+    } else {
+      nsel = P;
+    }
+    s0 = (int)((int64_t)cr * nsel / CS);
+    ns = (int)((int64_t)(cr + 1) * nsel / CS) - s0;
+    for (int i = tid; i < ns; i += kSpThreads)
+      fx.pg[i] = a.cand ? (uint32_t)a.cand[(int64_t)u * a.cand_stride + s0 + i] : (uint32_t)(s0 + i);
+    __syncthreads();
+  }
+  // physical rows of the share's pages (page ids outside the sequence: no rows)
+  for (int i = tid; i < ns; i += kSpThreads) {
+    const int pg = (int)fx.pg[i];
+    const bool valid = pg >= 0 && pg < P;
+    fx.nrow[i] = valid ? min(kPage, len - pg * kPage) : 0;
+    fx.r0[i] = valid ? (uint32_t)L.page_row(b, hk, pg) : 0u;
+  }
+  __syncthreads();
+
+  if (do_prune) {
+    // ---------------- phase 2: weight estimate of the share ----------------
+    const int nst = (ns + kEstStagePages - 1) / kEstStagePages;
+    unsigned char* ring = region;
+    const int ring_bytes = max(a.s2 * KW::kStageBytes, 2 * kSpBins * 4);
+    // logits [head][local position]: in shared memory (positions padded one
+    // word per 32, so a thread's run of R consecutive positions is free of
+    // bank conflicts) or at the set's positions [s0 * 16, ..) of the global
+    // logits
+    float* lbase;
+    int64_t hstride;
+    const bool lpad = a.glogits == nullptr;
+    if (!lpad) {
+      lbase = a.glogits + (int64_t)u * G * a.lcap + (int64_t)s0 * kPage;
+      hstride = a.lcap;
+    } else {
+      lbase = reinterpret_cast<float*>(region + ring_bytes);
+      hstride = sp_pad(a.share_cap * kPage);
+    }
+    auto lidx = [&](int h, int lp) -> int64_t { return h * hstride + (lpad ? sp_pad(lp) : lp); };
+    const uint8_t* codes = a.codes;
+    const __half* scales = a.scales;
+    const __half* zeros = a.zeros;
+    auto issue2 = [&](int k, int slot) {   // warp 0
+      const int npgs = min(kEstStagePages, ns - k * kEstStagePages);
+      unsigned char* st = ring + (size_t)slot * KW::kStageBytes;
+      unsigned char* st_codes = st;
+      unsigned char* st_scales = st + kEstStageTok * KW::kRowBytes;
+      unsigned char* st_zeros = st_scales + kEstStageTok * kGroups * 2;
+      // lane i < npgs: page i of the stage; rows copied = its valid rows
+      // rounded up to the page, except where the page runs past the cache's
+      // allocation (a contiguous cache whose length is not a multiple of 16)
+      int crow = 0;
+      uint32_t r0 = 0;
+      if (lane < npgs) {
+        const int e = k * kEstStagePages + lane;
+        const int pg = (int)fx.pg[e];
+        r0 = fx.r0[e];
+        if (fx.nrow[e] > 0) crow = (!paged && pg * kPage + kPage > L.N) ? L.N - pg * kPage : kPage;
+        if (crow > 0)
+          bulk_g2s(st_codes + lane * kPage * KW::kRowBytes, codes + (size_t)r0 * KW::kRowBytes,
+                   (uint32_t)(crow * KW::kRowBytes), &fx.full2[slot]);
+      }
+      // scales and zeros: 8 bytes per row by cp.async, row x of the stage per lane
+#pragma unroll
+      for (int x0 = 0; x0 < kEstStageTok; x0 += 32) {
+        const int x = x0 + lane, pi = x >> 4, r = x & 15;
+        const int cr_p = __shfl_sync(0xffffffffu, crow, pi);
+        const uint32_t r0_p = __shfl_sync(0xffffffffu, r0, pi);
+        if (r < cr_p) {
+          cp_async8_sm(st_scales + x * 8, scales + ((size_t)r0_p + r) * kGroups);
+          cp_async8_sm(st_zeros + x * 8, zeros + ((size_t)r0_p + r) * kGroups);
+        }
+      }
+      cp_async_arrive_noinc(&fx.full2[slot]);
+      uint32_t bytes = (uint32_t)(crow * KW::kRowBytes);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+      if (lane == 0) mbar_arrive_tx(&fx.full2[slot], bytes);
+    };
+    if (warp == 0) {
+      fence_proxy_async();   // the ring was written by threads before; the copies come after
+#pragma unroll 1
+      for (int k = 0; k < a.s2 && k < nst; ++k) issue2(k, k);
+    }
+    constexpr int HP = (G + 1) / 2;   // head pairs: one MMA N-block of 8 (head, group) columns each
+    const int gid = lane >> 2, t = lane & 3;
+    const int g0 = 2 * (t & 1);
+    uint32_t bfr[HP][8][2];
+    float Qv[HP][2];
+#pragma unroll
+    for (int hp = 0; hp < HP; ++hp) {
+      const int hb = 2 * hp + (gid >> 2);
+      const bool on = ((gid & 3) == t) && hb < G;
+      const __half* qb = a.q + ((int64_t)b * a.Hq + hk * G + min(hb, G - 1)) * kHeadDim;
+      const __half z = __float2half_rn(0.f);
+      const __half* qg = qb + kGroup * t;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+          bfr[hp][s][jj] = sp_pack_h2(on ? qg[KW::chan(s, jj, 0)] : z, on ? qg[KW::chan(s, jj, 1)] : z);
+      const int he = 2 * hp + (t >> 1);
+      const __half* qe = a.q + ((int64_t)b * a.Hq + hk * G + min(he, G - 1)) * kHeadDim;
+      float q0 = 0.f, q1 = 0.f;
+      for (int d = 0; d < kGroup; ++d) {
+        q0 += __half2float(qe[g0 * kGroup + d]);
+        q1 += __half2float(qe[(g0 + 1) * kGroup + d]);
+      }
+      Qv[hp][0] = q0;
+      Qv[hp][1] = q1;
+    }
+    float Mrun[HP], Zrun[HP];   // this lane's head (he) running statistics, owner lanes
+#pragma unroll
+    for (int hp = 0; hp < HP; ++hp) {
+      Mrun[hp] = -INFINITY;
+      Zrun[hp] = 0.f;
+    }
+    const bool owner = (t & 1) == 0;   // lanes t and t^1 hold the same logits
+    for (int j = 0; j < nst; ++j) {
+      const int slot = j % a.s2;
+      const uint32_t par = (uint32_t)((j / a.s2) & 1);
+      if (!failed) failed = !mbar_wait(&fx.full2[slot], par, a.status);
+      const unsigned char* st = ring + (size_t)slot * KW::kStageBytes;
+      const unsigned char* st_codes = st;
+      const __half* st_scales = reinterpret_cast<const __half*>(st + kEstStageTok * KW::kRowBytes);
+      const __half* st_zeros = st_scales + kEstStageTok * kGroups;
+      float lg[2][HP][2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int ca = warp * 32 + k * 16 + gid, cb = ca + 8;   // rows gid, gid + 8 of the tile
+        uint32_t WA[4], WB[4];
+        if (BITS == 4) {
+          const uint4 wa = *reinterpret_cast<const uint4*>(st_codes + ca * KW::kRowBytes + KW::kLaneBytes * t);
+          const uint4 wb = *reinterpret_cast<const uint4*>(st_codes + cb * KW::kRowBytes + KW::kLaneBytes * t);
+          WA[0] = wa.x, WA[1] = wa.y, WA[2] = wa.z, WA[3] = wa.w;
+          WB[0] = wb.x, WB[1] = wb.y, WB[2] = wb.z, WB[3] = wb.w;
+        } else {
+          const uint2 wa = *reinterpret_cast<const uint2*>(st_codes + ca * KW::kRowBytes + KW::kLaneBytes * t);
+          const uint2 wb = *reinterpret_cast<const uint2*>(st_codes + cb * KW::kRowBytes + KW::kLaneBytes * t);
+          WA[0] = wa.x, WA[1] = wa.y, WA[2] = WA[3] = 0u;
+          WB[0] = wb.x, WB[1] = wb.y, WB[2] = WB[3] = 0u;
+        }
+        const int ea = j * kEstStagePages + (ca >> 4), eb = j * kEstStagePages + (cb >> 4);
+        const bool va = ea < ns && (ca & 15) < fx.nrow[ea];
+        const bool vb = eb < ns && (cb & 15) < fx.nrow[eb];
+        // two accumulator chains (even and odd K-steps) halve the dependent MMA chain
+        float acc[HP][4], acc2[HP][4];
+#pragma unroll
+        for (int hp = 0; hp < HP; ++hp)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[hp][i] = acc2[hp][i] = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint32_t af[4] = {sp_code_pair<BITS>(WA, s, 0), sp_code_pair<BITS>(WB, s, 0),
+                                  sp_code_pair<BITS>(WA, s, 1), sp_code_pair<BITS>(WB, s, 1)};
+#pragma unroll
+          for (int hp = 0; hp < HP; ++hp)
+            sp_mma16816((s & 1) ? acc2[hp] : acc[hp], af, bfr[hp][s][0], bfr[hp][s][1]);
+        }
+#pragma unroll
+        for (int hp = 0; hp < HP; ++hp)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[hp][i] += acc2[hp][i];
+        const float2 fsa = __half22float2(*reinterpret_cast<const __half2*>(&st_scales[ca * kGroups + g0]));
+        const float2 fza = __half22float2(*reinterpret_cast<const __half2*>(&st_zeros[ca * kGroups + g0]));
+        const float2 fsb = __half22float2(*reinterpret_cast<const __half2*>(&st_scales[cb * kGroups + g0]));
+        const float2 fzb = __half22float2(*reinterpret_cast<const __half2*>(&st_zeros[cb * kGroups + g0]));
+        const float zza0 = __fmaf_rn(KW::kCentre, fsa.x, fza.x);
+        const float zza1 = __fmaf_rn(KW::kCentre, fsa.y, fza.y);
+        const float zzb0 = __fmaf_rn(KW::kCentre, fsb.x, fzb.x);
+        const float zzb1 = __fmaf_rn(KW::kCentre, fsb.y, fzb.y);
+#pragma unroll
+        for (int hp = 0; hp < HP; ++hp) {
+          float pa = __fmaf_rn(fsa.x, acc[hp][0], zza0 * Qv[hp][0]);
+          pa = __fmaf_rn(fsa.y, acc[hp][1], __fmaf_rn(zza1, Qv[hp][1], pa));
+          float pb = __fmaf_rn(fsb.x, acc[hp][2], zzb0 * Qv[hp][0]);
+          pb = __fmaf_rn(fsb.y, acc[hp][3], __fmaf_rn(zzb1, Qv[hp][1], pb));
+          pa += __shfl_xor_sync(0xffffffffu, pa, 1);   // + the other two groups
+          pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+          lg[k][hp][0] = va ? pa * kEstL2Scale : -INFINITY;
+          lg[k][hp][1] = vb ? pb * kEstL2Scale : -INFINITY;
+        }
+      }
+      const int cw0 = j * kEstStageTok + warp * 32;   // this warp's first local position
+#pragma unroll
+      for (int hp = 0; hp < HP; ++hp) {
+        const int he = 2 * hp + (t >> 1);
+        const bool hv = he < G;
+        if (owner && hv) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c0 = cw0 + k * 16 + gid;
+            if (c0 < ns * kPage) lbase[lidx(he, c0)] = lg[k][hp][0];
+            if (c0 + 8 < ns * kPage) lbase[lidx(he, c0 + 8)] = lg[k][hp][1];
+          }
+        }
+        float m = -INFINITY;
+        if (owner && hv) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) m = fmaxf(m, fmaxf(lg[k][hp][0], lg[k][hp][1]));
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float z = 0.f;
+        if (owner && hv && m != -INFINITY) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            z += exp2f(lg[k][hp][0] - m);
+            z += exp2f(lg[k][hp][1] - m);
+          }
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (m != -INFINITY) {
+          const float mn = fmaxf(Mrun[hp], m);
+          Zrun[hp] = (Mrun[hp] == -INFINITY ? 0.f : Zrun[hp] * exp2f(Mrun[hp] - mn)) +
+                     z * exp2f(m - mn);
+          Mrun[hp] = mn;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&fx.empty2[slot]);
+      if (warp == 0 && j + a.s2 < nst) {
+        if (!failed) failed = !mbar_wait(&fx.empty2[slot], par, a.status);
+        issue2(j + a.s2, slot);
+      }
+    }
+    // per-warp statistics -> the CTA's -> every CTA's, merged in rank order
+#pragma unroll
+    for (int hp = 0; hp < HP; ++hp) {
+      const int he = 2 * hp + (t >> 1);
+      if (gid == 0 && owner && he < G) fx.wstat[warp][he] = make_float2(Mrun[hp], Zrun[hp]);
+    }
+    __syncthreads();
+    if (tid < G) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kSpWarps; ++w) m = fmaxf(m, fx.wstat[w][tid].x);
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < kSpWarps; ++w) {
+        const float2 x = fx.wstat[w][tid];
+        if (x.x != -INFINITY) z += x.y * exp2f(x.x - m);
+      }
+      fx.mz_loc[tid] = make_float2(m, z);
+    }
+    __syncthreads();
+    if (tid < G * CS) {
+      const int h = tid % G, r = tid / G;
+      st_peer_f2(peer_addr(&fx.mz_all[cr][h], (uint32_t)r), fx.mz_loc[h]);
+    }
+    cluster_sync();
+    float Mh[G], iZ[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float m = -INFINITY;
+      for (int r = 0; r < CS; ++r) m = fmaxf(m, fx.mz_all[r][h].x);
+      float z = 0.f;
+      for (int r = 0; r < CS; ++r) {
+        const float2 x = fx.mz_all[r][h];
+        if (x.x != -INFINITY) z += x.y * exp2f(x.x - m);
+      }
+      Mh[h] = m;
+      iZ[h] = z > 0.f ? 1.0f / z : 0.f;
+    }
+
+    // ---------------- top-p per selection set ----------------
+    uint32_t* hlo = reinterpret_cast<uint32_t*>(ring);   // the estimate ring is idle now
+    uint32_t* hhi = hlo + kSpBins;
+    uint32_t* obuf = hlo;
+    const int npos = ns * kPage;                                  // local positions of the share
+    const int R = (npos + kSpThreads - 1) / kSpThreads;   // <= 32 (host-checked)
+    const int lp0 = tid * R;
+    const int nsets_u = a.group_sets ? 1 : G;
+    for (int hs = 0; hs < nsets_u; ++hs) {
+      const int set = a.group_sets ? u : b * a.Hq + hk * G + hs;
+      const int h0 = a.group_sets ? 0 : hs, nh = a.group_sets ? G : 1;
+      __syncthreads();   // the ring (or the previous set's staged output) is free
+      for (int i = tid; i < 2 * kSpBins; i += kSpThreads) hlo[i] = 0u;
+      // the set's weights, written over the logits of its first head (each
+      // thread reads and writes only its own positions)
+      SpWeights W{lbase + h0 * hstride, lpad, lp0, R, npos};
+#pragma unroll 1
+      for (int i = 0; i < R; ++i) {
+        const int lp = lp0 + i;
+        if (lp >= npos) break;
+        const bool ok = (lp & 15) < fx.nrow[lp >> 4];
+        float acc = 0.f;
+        if (ok) {
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            if (h >= h0 && h < h0 + nh) acc += exp2f(lbase[lidx(h, lp)] - Mh[h]) * iZ[h];
+          if (nh > 1) acc *= 1.0f / (float)nh;
+        }
+        lbase[lidx(h0, lp)] = ok ? acc : -1.0f;
+      }
+      const bool keep_all = a.p >= 1.0;
+      uint32_t theta = 0;
+      unsigned long long r_need = 0;
+      bool have = false;
+      if (!keep_all) {
+        SpSearch sr{0u, 0u, 0ull, 0ull};
+        // digits of the 30-bit weight key: bits 29..18, 17..9, 8..0
+        bool done_small = false;
+#pragma unroll 1
+        for (int step = 0; step < 3; ++step) {
+          const bool ok = digit_step(W, step == 0 ? 18 : (step == 1 ? 9 : 0),
+                                     step == 0 ? 0xFFFu : 0x1FFu, step == 0 ? kSpBins : 512, a.p,
+                                     CS, cr, hlo, hhi, fx, sr);
+          if (step == 0) {
+            have = ok;
+            if (have) done_small = resolve_small_bin(W, sr, s0 * kPage, CS, fx, &theta, &r_need);
+          }
+          if (!have || done_small) break;   // the same in every CTA of the cluster
+        }
+        if (have && !done_small) {
+          theta = sr.prefix;
+          unsigned long long Ft = sp_mass(__uint_as_float(theta));
+          if (Ft == 0) Ft = 1;
+          r_need = (sr.T - sr.A + Ft - 1) / Ft;
+        }
+      }
+      // compaction in ascending position order
+      unsigned n_gt = 0, n_eq = 0;
+#pragma unroll 1
+      for (int i = 0; i < R; ++i) {
+        if (lp0 + i >= npos) break;
+        const float w = W.at(i);
+        if (w < 0.f) continue;
+        const uint32_t key = __float_as_uint(w);
+        if (keep_all || (have && key > theta)) ++n_gt;
+        else if (have && key == theta) ++n_eq;
+      }
+      unsigned blk_total;
+      const unsigned ex = sp_scan((n_gt << 16) | n_eq, fx.scan, &blk_total);
+      unsigned gt_before = 0, eq_before = 0, gt_all = blk_total >> 16, eq_all = blk_total & 0xFFFFu;
+      if (CS > 1) {
+        if (tid == 0) {
+          fx.blk[0] = blk_total >> 16;
+          fx.blk[1] = blk_total & 0xFFFFu;
+        }
+        cluster_sync();
+        if (warp == 0) {
+          unsigned g = 0, e = 0, gb = 0, eb = 0;
+          if (lane < CS) {
+            g = ld_peer_u32(peer_addr(&fx.blk[0], (uint32_t)lane));
+            e = ld_peer_u32(peer_addr(&fx.blk[1], (uint32_t)lane));
+            if (lane < cr) {
+              gb = g;
+              eb = e;
+            }
+          }
+          g = warp_sum(g);
+          e = warp_sum(e);
+          gb = warp_sum(gb);
+          eb = warp_sum(eb);
+          if (lane == 0) {
+            fx.pre[0] = gb;
+            fx.pre[1] = eb;
+            fx.pre[2] = g;
+            fx.pre[3] = e;
+          }
+        }
+        __syncthreads();
+        gt_before = fx.pre[0];
+        eq_before = fx.pre[1];
+        gt_all = fx.pre[2];
+        eq_all = fx.pre[3];
+      }
+      const unsigned long long ties_before = (unsigned long long)eq_before + (ex & 0xFFFFu);
+      unsigned take = 0;
+      if (ties_before < r_need) take = (unsigned)min((unsigned long long)n_eq, r_need - ties_before);
+      const unsigned first = gt_before + (unsigned)min(r_need, (unsigned long long)eq_before);
+      const unsigned eq_blk = blk_total & 0xFFFFu;
+      const unsigned n_out =
+          (blk_total >> 16) +
+          (r_need > eq_before ? (unsigned)min((unsigned long long)eq_blk, r_need - eq_before) : 0u);
+      const unsigned lpos0 = (ex >> 16) + (unsigned)min(r_need, ties_before) -
+                             (unsigned)min(r_need, (unsigned long long)eq_before);
+      unsigned sel = 0;   // bit i: local position lp0 + i is kept (R <= 32)
+      {
+        unsigned taken = 0;
+#pragma unroll 1
+        for (int i = 0; i < R; ++i) {
+          if (lp0 + i >= npos) break;
+          const float w = W.at(i);
+          if (w < 0.f) continue;
+          const uint32_t key = __float_as_uint(w);
+          bool keep = keep_all || (have && key > theta);
+          if (!keep && have && key == theta && taken < take) {
+            keep = true;
+            ++taken;
+          }
+          if (keep) sel |= 1u << i;
+        }
+      }
+      for (int pass = 0; pass < (a.rows ? 2 : 1); ++pass) {
+        unsigned lp = lpos0;
+        unsigned m = sel;
+#pragma unroll 1
+        while (m) {
+          const int i = __ffs(m) - 1;
+          m &= m - 1;
+          const int e = (lp0 + i) >> 4, r = (lp0 + i) & 15;
+          obuf[lp++] = pass == 0 ? fx.pg[e] * kPage + (uint32_t)r : fx.r0[e] + (uint32_t)r;
+        }
+        __syncthreads();
+        uint32_t* dst = pass == 0 ? reinterpret_cast<uint32_t*>(a.idx + (int64_t)set * a.icap + first)
+                                  : a.rows + (int64_t)set * a.icap + first;
+        for (unsigned i = tid; i < n_out; i += kSpThreads) dst[i] = obuf[i];
+        __syncthreads();   // obuf is rewritten by the next pass
+      }
+      if (cr == 0 && tid == 0) {
+        a.count[set] = (int32_t)(gt_all + (unsigned)min(r_need, (unsigned long long)eq_all));
+        if (a.done) a.done[set] = 0;   // the attention kernel's per-set completion counter
+      }
+      if (CS > 1) cluster_sync();   // peers are done reading this CTA's totals
+    }
+  }
+  if (failed) {   // a wait gave up: give any copy still in flight time to land before exit
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < kWaitNs / 4) {
+    }
+  }
+  griddep_launch();
+  cluster_sync();   // no CTA leaves while a peer may still access its shared memory
+}
+
+// ---------------------------------------------------------------------------
+template <int G, int BITS>
+static cudaError_t sp_prepare() {
+  static std::atomic<int> attr_set[kMaxDevices];
+  return once_per_device(attr_set, [] {
+    cudaError_t e = cudaFuncSetAttribute(k_select_prune<G, BITS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSpMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_select_prune<G, BITS>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+  });
+}
+
+static cudaLaunchConfig_t sp_config(int units, int cs, size_t smem, cudaStream_t st,
+                                    cudaLaunchAttribute* attr, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units * (unsigned)cs);
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = (unsigned)cs;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cfg;
+}
+
+// Clusters of `cs` CTAs with `smem` bytes each that fit the device at once
+// (cached per device, cluster size and shared-memory size).
+template <int G, int BITS>
+static int sp_max_clusters(int cs, size_t smem) {
+  struct Entry { int dev, cs; size_t smem; int n; };
+  static Entry cache[64];
+  static std::atomic<int> ncache{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const int n = ncache.load(std::memory_order_acquire);
+  for (int i = 0; i < n && i < 64; ++i)
+    if (cache[i].dev == dev && cache[i].cs == cs && cache[i].smem == smem) return cache[i].n;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = sp_config(cs, cs, smem, nullptr, attr, false);
+  int m = 0;
+  if (cudaOccupancyMaxActiveClusters(&m, k_select_prune<G, BITS>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    m = 0;
+  }
+  const int slot = ncache.load(std::memory_order_acquire);
+  if (slot < 64) {   // a racing thread at worst stores the same answer twice
+    cache[slot] = Entry{dev, cs, smem, m};
+    ncache.store(slot + 1, std::memory_order_release);
+  }
+  return m;
+}
+
+// Shared memory of a launch with ring depths s1, s2.
+static size_t sp_smem_bytes(const SpShape& s, int kbits, int G, int max_pages, bool do_select,
+                      bool do_prune) {
+  const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * kbits / 8 + 2 * kGroups * 2);
+  size_t ra = 0, rb = 0;
+  if (do_select)
+    ra = (size_t)s.s1 * kMetaStageBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
+  if (do_prune) {
+    rb = (size_t)s.s2 * stage2 > (size_t)2 * kSpBins * 4 ? (size_t)s.s2 * stage2
+                                                         : (size_t)2 * kSpBins * 4;
+    if (s.logits_in_smem) rb += (size_t)sp_pad(s.share_cap * kPage) * G * sizeof(float);
+  }
+  return (kSpFixedBytes + (ra > rb ? ra : rb) + 127) / 128 * 128;
+}
+
+// Launch shape.  Each CTA's share of the candidate pages must fit
+// kSpSharePages.  When the units, one cluster each, can all run at once
+// with one CTA per SM, the cluster is the largest that allows that (an
+// occupancy query decides: a cluster of 16 needs 16 free SMs of one GPC),
+// and the rings take the whole shared memory (the bytes in flight per SM
+// set the streaming rate).  Otherwise the cluster is the smallest allowed
+// and the shared memory is sized for two CTAs per SM.
+template <int G, int BITS>
+static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, bool do_prune,
+                    int num_sms, SpShape* out) {
+  int cs_min = 1;
+  while (cs_min < kSpMaxCluster && (sel_pages + cs_min - 1) / cs_min > kSpSharePages) cs_min *= 2;
+  if ((sel_pages + cs_min - 1) / cs_min > kSpSharePages) return -1;
+  const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * BITS / 8 + 2 * kGroups * 2);
+  auto fill = [&](int cs, size_t budget, SpShape* s) {
+    s->cs = cs;
+    s->share_cap = (sel_pages + cs - 1) / cs;
+    s->keys_in_smem = max_pages <= kSpKeysCap;
+    s->logits_in_smem = (size_t)sp_pad(s->share_cap * kPage) * G * 4 <= (size_t)kSpLogitsSmem;
+    const size_t keys = s->keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0;
+    const size_t logits = s->logits_in_smem ? (size_t)sp_pad(s->share_cap * kPage) * G * 4 : 0;
+    const size_t room1 = budget > kSpFixedBytes + keys ? budget - kSpFixedBytes - keys : 0;
+    const size_t room2 = budget > kSpFixedBytes + logits ? budget - kSpFixedBytes - logits : 0;
+    s->s1 = (int)(room1 / kMetaStageBytes);
+    s->s2 = (int)(room2 / stage2);
+    const int need2 = (s->share_cap + kEstStagePages - 1) / kEstStagePages;   // stages of a share
+    s->s1 = s->s1 < 2 ? 2 : (s->s1 > kSpMaxStages ? kSpMaxStages : s->s1);
+    s->s2 = s->s2 < 2 ? 2 : (s->s2 > kSpMaxStages ? kSpMaxStages : s->s2);
+    if (s->s2 > need2 && need2 >= 2) s->s2 = need2;
+    s->smem = sp_smem_bytes(*s, BITS, G, max_pages, do_select, do_prune);
+  };
+  SpShape s;
+  const size_t big = 200 * 1024, two_per_sm = 110 * 1024;
+  for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
+    if ((long long)units * cs > num_sms) continue;
+    fill(cs, big, &s);
+    if (s.smem > kSpMaxSmem) continue;
+    if (sp_max_clusters<G, BITS>(cs, s.smem) >= units) {
+      *out = s;
+      return 0;
+    }
+  }
+  fill(cs_min, two_per_sm, &s);
+  if (s.smem > kSpMaxSmem) return -1;
+  *out = s;
+  return 0;
+}
+
+template <int G, int BITS>
+static cudaError_t sp_launch_t(SpArgs a, int sel_pages, int num_sms, cudaStream_t st, bool pdl) {
+  const cudaError_t prepared = sp_prepare<G, BITS>();
+  if (prepared != cudaSuccess) return prepared;
+  const int units = a.L.B * a.L.Hk;
+  SpShape sh;
+  if (sp_shape<G, BITS>(units, a.L.max_pages, sel_pages, a.meta != nullptr, a.codes != nullptr,
+                        num_sms, &sh) != 0)
+    return cudaErrorInvalidValue;
+  a.s1 = sh.s1;
+  a.s2 = sh.s2;
+  a.share_cap = sh.share_cap;
+  if (sh.keys_in_smem) a.gkeys = nullptr;
+  if (sh.logits_in_smem) a.glogits = nullptr;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = sp_config(units, sh.cs, sh.smem, st, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, k_select_prune<G, BITS>, a);
+}
+
+cudaError_t launch_select_prune(const SpArgs& a, int sel_pages, int num_sms, cudaStream_t st,
+                                bool pdl) {
+  const int G = a.Hq / a.L.Hk;
+  if (a.L.B * a.L.Hk == 0) return cudaSuccess;
+  const bool two = a.L.kbits == 2;
+#define TW_SP(GG)                                                                      \
+  case GG:                                                                             \
+    return two ? sp_launch_t<GG, 2>(a, sel_pages, num_sms, st, pdl)                    \
+               : sp_launch_t<GG, 4>(a, sel_pages, num_sms, st, pdl);
+  switch (G) {
+    TW_SP(1) TW_SP(2) TW_SP(4) TW_SP(8)
+  }
+#undef TW_SP
+  return cudaErrorInvalidValue;
+}
+
+// Largest candidate pages per unit the selection stages accept.
+int select_prune_max_pages() { return kSpSharePages * kSpMaxCluster; }
+
+}  // namespace tw

@@ -50,8 +50,10 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="llama2_mha",
+    ap.add_argument("--config", default="batched_paged",
                     choices=["llama2_mha", "llama3_gqa", "batched_paged", "sweep", "tiny"])
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads' step times in the JSON line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -70,23 +72,25 @@ def make_workload(name, device):
     return W.CONFIGS[name](device=device)
 
 
-def workload_config(w, copies=None, copy_bytes=None, key_bits=4, selector="quest"):
+def workload_config(w, key_bits=4, selector="quest"):
     c = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hk,
          "context": w.N, "paged": w.paged, "budget_tokens": w.budget_tokens, "p": w.p,
          "group_mode": w.group_mode, "head_dim": 128, "page_size": 16, "key_bits": key_bits,
          "key_group": 32, "selector": selector}
     if selector == "label":
         c["label_channels"] = LABEL_R
-    if copies:
-        c["l2"] = (f"inputs larger than L2: {copies} rotating cache copies, "
-                   f"{copy_bytes / 1e9:.2f} GB each")
     return c
+
+
+def l2_policy(copies, copy_bytes):
+    return (f"inputs larger than L2: {copies} rotating cache copies, "
+            f"{copy_bytes / 1e9:.2f} GB each")
 
 
 # Device sources of the kernels the traffic record measures (and the headers
 # they include): the record is used only while these bytes are unchanged.
-TRAFFIC_SOURCES = ("cache_build.cu", "decode.cu", "estimate.cu", "host_io.cu", "resolve.cu",
-                   "select.cu", "topp.cu", "tw_common.cuh", "tw_kernels.h")
+TRAFFIC_SOURCES = ("cache_build.cu", "decode.cu", "host_io.cu", "resolve.cu", "select_prune.cu",
+                   "tw_bulk.cuh", "tw_common.cuh", "tw_kernels.h")
 
 
 def src_hash():
@@ -184,63 +188,117 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle
+def _oracle_unit_inputs(x, w_cpu, b, hk, key_bits, label_channels):
+    """One (sequence, KV head) unit's cache companions, built as at prefill
+    (outside every timed region)."""
+    import oracle as O
+    G = x.Hq // x.Hk
+    L = int(x.seq_lens[b])
+    k_seq = O.sequence_rows(x.k, x.page_table, b, hk, L)
+    v_seq = O.sequence_rows(x.v, x.page_table, b, hk, L)
+    codes, scales, zeros = O.quantize_keys(k_seq, key_bits)
+    meta = O.page_meta(k_seq, L) if w_cpu.budget_tokens else None
+    labels = O.label_cache(k_seq, label_channels[hk]) if label_channels is not None else None
+    return dict(L=L, k=k_seq, v=v_seq, codes=codes, scales=scales, zeros=zeros, meta=meta,
+                labels=labels, qg=x.q[b, hk * G:(hk + 1) * G], hk=hk)
+
+
+def _oracle_unit_step(u, w_cpu, G, key_bits, label_channels):
+    """The oracle's decode step of one unit: base selector, quantised-key
+    estimate, top-p, sparse attention."""
+    import oracle as O
+    qg = u["qg"]
+    if u["labels"] is not None:
+        toks = O.select_tokens(O.label_scores(qg, u["labels"], label_channels[u["hk"]]),
+                               w_cpu.budget_tokens)
+    else:
+        pages = None
+        if w_cpu.budget_tokens:
+            pages = O.select_pages(O.quest_page_scores(qg, u["meta"]), w_cpu.budget_tokens)
+        toks = O.candidate_tokens(pages, u["L"])
+    lg = O.estimate_logits(qg, u["codes"][toks], u["scales"][toks], u["zeros"][toks], key_bits)
+    if w_cpu.group_mode and G > 1:
+        sel = O.topp_select(O.group_weights(lg), w_cpu.p)[0]
+        sels = [sel] * G
+    else:
+        sels = [O.topp_select(O.softmax_weights(lg[:, g]), w_cpu.p)[0] for g in range(G)]
+    for g in range(G):
+        t = toks[sels[g]]
+        O.sparse_attention(qg[g], u["k"][t], u["v"][t])
+
+
+def _single_thread_blas():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except Exception:
+        return None
+
+
 def cpu_step_sample(w_cpu, seconds: float, max_units=None, key_bits=4, label_channels=None):
     """Time the oracle's decode step (page scores, top-K_p, quantised-key
     estimate, top-p, sparse attention) on (b, kv head) units of the workload
-    until `seconds` of CPU work; the key cache and page metadata are built
-    first, untimed, as at prefill.  Returns (us per full step, units timed,
-    total units, threads).  With label_channels the base selector is the
-    token-level label-channel one instead of Quest's pages."""
-    try:
-        from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
-    except Exception:
-        limiter = None
+    until `seconds` of CPU work, single-threaded; the key cache and page
+    metadata are built first, untimed, as at prefill.  Returns (us per full
+    step, units timed, total units, threads).  With label_channels the base
+    selector is the token-level label-channel one instead of Quest's pages."""
+    limiter = _single_thread_blas()
     import numpy as np
 
     import oracle as O
     x = O.SeqInputs.from_workload(w_cpu)
     G = x.Hq // x.Hk
     units = [(b, h) for b in range(x.B) for h in range(x.Hk)]
-    rng = np.random.default_rng(0)
-    order = rng.permutation(len(units))
+    order = np.random.default_rng(0).permutation(len(units))
     spent, n = 0.0, 0
     for ui in order:
         if max_units is not None and n >= max_units:
             break
         b, hk = units[ui]
-        L = int(x.seq_lens[b])
-        k_seq = O.sequence_rows(x.k, x.page_table, b, hk, L)
-        v_seq = O.sequence_rows(x.v, x.page_table, b, hk, L)
-        codes, scales, zeros = O.quantize_keys(k_seq, key_bits)
-        meta = O.page_meta(k_seq, L) if w_cpu.budget_tokens else None
-        labels = O.label_cache(k_seq, label_channels[hk]) if label_channels is not None else None
-        qg = x.q[b, hk * G:(hk + 1) * G]
+        u = _oracle_unit_inputs(x, w_cpu, b, hk, key_bits, label_channels)
         t0 = time.perf_counter()
-        pages = None
-        if labels is not None:
-            toks = O.select_tokens(O.label_scores(qg, labels, label_channels[hk]),
-                                   w_cpu.budget_tokens)
-        else:
-            if w_cpu.budget_tokens:
-                pages = O.select_pages(O.quest_page_scores(qg, meta), w_cpu.budget_tokens)
-            toks = O.candidate_tokens(pages, L)
-        lg = O.estimate_logits(qg, codes[toks], scales[toks], zeros[toks], key_bits)
-        if w_cpu.group_mode and G > 1:
-            sel = O.topp_select(O.group_weights(lg), w_cpu.p)[0]
-            sels = [sel] * G
-        else:
-            sels = [O.topp_select(O.softmax_weights(lg[:, g]), w_cpu.p)[0] for g in range(G)]
-        for g in range(G):
-            t = toks[sels[g]]
-            O.sparse_attention(qg[g], k_seq[t], v_seq[t])
+        _oracle_unit_step(u, w_cpu, G, key_bits, label_channels)
         spent += time.perf_counter() - t0
         n += 1
         if spent >= seconds:
             break
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
+    if limiter is not None and hasattr(limiter, "unregister"):
+        limiter.unregister()
     return spent / n * len(units) * 1e6, n, len(units), 1
+
+
+def cpu_step_all_cores(w_cpu, per_unit_us: float, seconds: float, key_bits=4,
+                       label_channels=None):
+    """The same oracle step on all host cores: a thread pool with one worker
+    per core runs whole units concurrently (numpy releases the interpreter
+    lock in its array work; each worker's BLAS is single-threaded).  About
+    `seconds` of wall time from the single-thread per-unit cost; the inputs of
+    the sampled units are built first, untimed.  Returns (us per full step,
+    units timed, total units, threads)."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
+    import oracle as O
+    limiter = _single_thread_blas()
+    threads = os.cpu_count() or 1
+    x = O.SeqInputs.from_workload(w_cpu)
+    G = x.Hq // x.Hk
+    units = [(b, h) for b in range(x.B) for h in range(x.Hk)]
+    want = int(seconds * 1e6 / max(per_unit_us, 1.0) * threads)
+    n = max(threads, min(want, 4 * threads, len(units)))
+    n = min(n, len(units))
+    order = np.random.default_rng(1).permutation(len(units))[:n]
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        prepared = list(ex.map(lambda i: _oracle_unit_inputs(x, w_cpu, *units[i], key_bits,
+                                                             label_channels), order))
+        t0 = time.perf_counter()
+        list(ex.map(lambda u: _oracle_unit_step(u, w_cpu, G, key_bits, label_channels),
+                    prepared))
+        wall = time.perf_counter() - t0
+    if limiter is not None and hasattr(limiter, "unregister"):
+        limiter.unregister()
+    return wall / n * len(units) * 1e6, n, len(units), threads
 
 
 def run_reference(args):
@@ -295,11 +353,11 @@ def label_algorithmic_bytes(w, step, key_bits=4):
 
 
 def algorithmic_bytes(w, step, key_bits=4):
-    """Bytes the step must move (per kernel): page metadata scanned (512 B per
-    page per KV head), quantised candidate keys (128 * key_bits / 8 B of codes
-    + 16 B of scales and zeros per candidate token per KV head: 80 B at 4 bits,
-    48 B at 2 bits) and fp16 K+V rows of the selected tokens (512 B per token
-    per set)."""
+    """Bytes the step must move (per kernel): the selection kernel reads the
+    page metadata (512 B per page per KV head) and the quantised candidate keys
+    (128 * key_bits / 8 B of codes + 16 B of scales and zeros per candidate
+    token per KV head: 80 B at 4 bits, 48 B at 2 bits); the attention kernel
+    reads the fp16 K+V rows of the selected tokens (512 B per token per set)."""
     import torch
     lens = w.seq_lens.to(torch.int64).cpu()
     pages = (lens + 15) // 16
@@ -321,7 +379,81 @@ def algorithmic_bytes(w, step, key_bits=4):
     int4_b = cand_tokens * (128 * key_bits // 8 + 16)
     kept = step.count.to(torch.int64).cpu()
     kv_b = int(kept.sum()) * 512
-    return {"page_scores": meta_b, "estimate": int4_b, "sparse_decode": kv_b}, cand_tokens, kept
+    first = "select_prune" if w.budget_tokens else "prune"
+    return {first: meta_b + int4_b, "sparse_decode": kv_b}, cand_tokens, kept
+
+
+PER_CONFIGS = ("llama2_mha", "llama3_gqa", "sweep")
+NOMINAL_HBM_GBS = 8000.0
+
+
+def time_workload(w, dev, key_bits, steps, warmup):
+    """Device time of the decode step on another workload (the same rotating
+    cache copies and CUDA-event timing as the headline), with its algorithmic
+    bytes and roofline fractions."""
+    import torch
+
+    from adaptive_top_sparse_quest_b200 import DecodeStep, KVCache, page_meta, quantize_keys
+    kv0 = KVCache.from_workload(w, key_bits)
+    keys0 = quantize_keys(kv0)
+    meta0 = page_meta(kv0)
+    torch.cuda.synchronize()
+    copy_bytes = sum(t.numel() * t.element_size() for t in
+                     (w.k, w.v, keys0.codes, keys0.scales, keys0.zeros, meta0))
+    R = 1
+    while R * min(copy_bytes, 4 * 114e6) < 4 * L2_BYTES and R < 16:
+        R += 1
+    R = max(R, 4)
+    steps_l = []
+    for r in range(R):
+        if r == 0:
+            kv, keys, meta = kv0, keys0, meta0
+        else:
+            kv = KVCache(w.k.clone(), w.v.clone(), w.seq_lens.clone(),
+                         None if w.page_table is None else w.page_table.clone(), key_bits)
+            keys = type(keys0)(keys0.codes.clone(), keys0.scales.clone(), keys0.zeros.clone())
+            meta = meta0.clone()
+        steps_l.append(DecodeStep(kv, keys, meta, w.Hq, w.budget_tokens, w.p, w.group_mode))
+    q = w.q.contiguous()
+    for i in range(max(3, warmup)):
+        steps_l[i % R](q)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st = torch.cuda.current_stream()
+    e0.record(st)
+    for i in range(steps):
+        steps_l[i % R](q)
+    e1.record(st)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    kb, cand_tokens, kept = algorithmic_bytes(w, steps_l[0], key_bits)
+    total = sum(kb.values())
+    peak, peak_kind = hbm_peak()
+    gbs = total / (us * 1e-6) / 1e9
+    out = {"workload": w.name, "us_per_step": us, "bytes_per_step": total, "hbm_gbs": gbs,
+           "frac_of_measured": gbs / peak, "frac_of_nominal_8000": gbs / NOMINAL_HBM_GBS,
+           "peak_kind": peak_kind, "kept_tokens_mean": float(kept.double().mean()),
+           "candidates_per_set": cand_tokens / max(1, w.B * w.Hk), "steps": steps,
+           "l2": l2_policy(R, copy_bytes)}
+    del steps_l, kv0, keys0, meta0
+    torch.cuda.empty_cache()
+    return out
+
+
+def per_config_times(headline, dev, key_bits, steps, warmup):
+    """The other single-GPU workloads' step times (the sweep at tau = 1, p = 0.85)."""
+    import workloads as W
+    res = {}
+    for name in PER_CONFIGS:
+        if name == headline:
+            continue
+        if name == "sweep":
+            w = W.sweep_point(W.concentration_sweep(device=dev), 1.0, 0.85)
+        else:
+            w = W.CONFIGS[name](device=dev)
+        res[name] = time_workload(w, dev, key_bits, steps, warmup)
+        del w
+    return res
 
 
 def main():
@@ -531,9 +663,18 @@ def main():
         cpu_us, n_units, tot_units, cores = cpu_step_sample(
             w_cpu, args.cpu_seconds, key_bits=args.key_bits,
             label_channels=W.label_channels(w, r=LABEL_R) if label else None)
+        per_unit = cpu_us / tot_units
+        all_us, n_all, _, threads = cpu_step_all_cores(
+            w_cpu, per_unit, args.cpu_seconds, key_bits=args.key_bits,
+            label_channels=W.label_channels(w, r=LABEL_R) if label else None)
         cpu = {"value": cpu_us, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n_units} of {tot_units} (sequence, KV head) units of the same "
-                         f"workload, single-threaded numpy, scaled to the full step"}
+                         f"workload, single-threaded numpy, scaled to the full step",
+               "all_cores": {"value": all_us, "unit": UNIT, "cores": threads,
+                             "nproc": os.cpu_count(),
+                             "sample": f"{n_all} of {tot_units} units run concurrently by "
+                                       f"{threads} worker threads, wall time scaled to the "
+                                       f"full step"}}
 
     sets = kept.numel()
     cands_per_set = cand_tokens / max(1, w.B * w.Hk)
@@ -542,7 +683,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, R, copy_bytes, args.key_bits, args.selector),
+        "config": workload_config(w, args.key_bits, args.selector),
+        "l2": l2_policy(R, copy_bytes),
         "hbm_gbs": total_b / (us_per_step * 1e-6) / 1e9,
         "hbm_frac_of_measured": total_b / (us_per_step * 1e-6) / 1e9 / peak,
         "bytes_per_step": total_b,
@@ -555,7 +697,10 @@ def main():
                           "std": float(retained.std()) if retained.numel() > 1 else 0.0,
                           "min": float(retained.min()), "max": float(retained.max()),
                           "heads": retained.numel()},
-        "kernel_us": kernel_us,
+        "step_us": us_per_step,
+        "kernel_us_serialised": kernel_us,
+        "kernel_us_note": "each kernel bracketed by events with no overlap between kernels "
+                          "(programmatic dependent launch off); step_us is the overlapped step",
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": kb[dom]},
@@ -570,6 +715,11 @@ def main():
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
+    if world == 1 and not args.no_per_config and args.selector == "quest":
+        del steps
+        torch.cuda.empty_cache()
+        line["per_config"] = per_config_times(args.config, dev, args.key_bits,
+                                              max(20, min(args.steps, 200)), args.warmup)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -223,13 +223,17 @@ int tw_sparse_decode(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,
  * it exists only for that calling constraint.
  * Same inputs, outputs and results as tw_topp_prune; the scratch is one fixed
  * array of TW_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library, resident
- * on every GPU that loads it until the process exits.  Shapes whose scratch
- * (logits and softmax statistics, about B * Hk * capacity * G * 4 bytes, plus
- * 4 bytes per page of the B * Hk * ceil(N / 16) cache pages) does not fit
- * return TW_ERR_CAPACITY before any device work.  The first call on a
- * device looks up the array's device address (TW_ERR_CUDA if that fails), so
- * make it before any stream capture.  Every call shares the array: calls that
- * overlap on the GPU race.  Nothing in it needs to start at zero.
+ * on every GPU that loads it until the process exits.  A call needs
+ *   256 + align256(B * Hk * G * lcap * 4) bytes of it,
+ * lcap = capacity rounded up to a multiple of 64 and align256 rounding up to a
+ * multiple of 256 (a status word, then room for the selection sets' logits);
+ * a call that needs more returns TW_ERR_CAPACITY before any device work.  The
+ * first call on a device looks up the array's device address (TW_ERR_CUDA if
+ * that fails) and keeps it for later calls on that device, so make it before
+ * any stream capture; the address stays valid for the life of the device's
+ * primary context (no cudaDeviceReset between calls).  Every call shares the
+ * array: calls that overlap on the GPU race.  Nothing in it needs to start at
+ * zero.
  */
 #define TW_NOALLOC_SCRATCH_BYTES (8u << 20)
 int tw_topp_prune_noalloc(const uint16_t* q, int32_t num_q_heads, const tw_kv* kv,

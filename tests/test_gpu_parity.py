@@ -242,19 +242,36 @@ def _full(w, units, budget, p, gm):
 @pytest.mark.slow
 def test_full_llama2_mha_32k():
     w = W.llama2_mha(device="cuda")
-    _full(w, [(0, 0), (0, 17), (0, 31)], w.budget_tokens, w.p, 0)
+    _full(w, [(0, h) for h in range(w.Hk)], w.budget_tokens, w.p, 0)
 
 
 @pytest.mark.slow
 def test_full_llama3_gqa_128k():
     w = W.llama3_gqa(device="cuda")
-    _full(w, [(0, 0), (0, 3), (0, 7)], w.budget_tokens, w.p, 1)
+    _full(w, [(0, h) for h in range(w.Hk)], w.budget_tokens, w.p, 1)
+
+
+def _spread_units(w, n):
+    """n (sequence, KV head) units spread over the batch: every sequence, the
+    shortest and longest ones with all their heads, the rest by a fixed stride."""
+    lens = w.seq_lens.cpu().tolist()
+    short, long_ = lens.index(min(lens)), lens.index(max(lens))
+    step = max(1, w.Hk // 8)
+    units = [(short, h) for h in range(0, w.Hk, step)][:8]
+    units += [(long_, h) for h in range(step // 2, w.Hk, step)][:8]
+    k = 0
+    while len(units) < n:
+        u = (k % w.B, (k * 7 + k // w.B) % w.Hk)
+        if u not in units:
+            units.append(u)
+        k += 1
+    return units[:n]
 
 
 @pytest.mark.slow
 def test_full_batched_paged():
     w = W.batched_paged(device="cuda")
-    _full(w, [(0, 0), (7, 12), (15, 31)], w.budget_tokens, w.p, 0)
+    _full(w, _spread_units(w, 64), w.budget_tokens, w.p, 0)
 
 
 @pytest.mark.slow

@@ -80,3 +80,42 @@ def test_noalloc_rejects_oversized_scratch(lib):
     st = lib.tw_topp_prune_noalloc(p, 8, ctypes.byref(s), p, p, p, None, 0, None, 0.9, 1, p,
                                    65536, p, None)
     assert st == _capi.TW_ERR_CAPACITY
+
+
+def _scratch_need(B, Hk, G, capacity):
+    """Bytes of the array a call needs: a 256-byte status word, then the logits
+    of the selection sets, B * Hk * G * lcap floats with lcap = capacity rounded
+    up to a multiple of 64, the region rounded up to 256 bytes."""
+    lcap = (capacity + 63) // 64 * 64
+    return 256 + (B * Hk * G * lcap * 4 + 255) // 256 * 256
+
+
+def test_noalloc_limit_just_above_is_rejected_on_the_host(lib):
+    from adaptive_top_sparse_quest_b200 import _capi
+    cap = 2097089   # lcap 2097152: 256 + 8 MiB, one region step over the array
+    assert _scratch_need(1, 1, 1, cap) > 8 << 20
+    s = _capi.TwKv()
+    s.k = s.v = 1 << 20
+    s.batch, s.num_kv_heads, s.max_seq_len = 1, 1, 4096
+    s.page_size, s.head_dim = 16, 128
+    p = 1 << 20
+    st = lib.tw_topp_prune_noalloc(p, 1, ctypes.byref(s), p, p, p, None, 0, None, 0.9, 0, p,
+                                   cap, p, None)
+    assert st == _capi.TW_ERR_CAPACITY
+
+
+def test_noalloc_limit_just_below_runs_and_matches(lib):
+    """capacity 2097088 needs exactly the 8 MiB of the array and must run."""
+    from adaptive_top_sparse_quest_b200 import _capi, prepare, topp_prune
+    cap = 2097088
+    assert _scratch_need(1, 1, 1, cap) == 8 << 20
+    w = W.random_small(33, B=1, Hq=1, Hk=1, N=4096, budget_tokens=None, p=0.9, group_mode=0)
+    kv, keys, meta, q = prepare(w, "cuda")
+    idx_ref, cnt_ref = topp_prune(q, kv, keys, None, None, 0.9, 0, capacity=cap)
+    for _ in range(2):
+        st, idx, cnt = _noalloc(lib, q, kv, keys, None, None, 0.9, 0, cap, 1)
+        assert st == _capi.TW_OK, lib.tw_status_string(st)
+        torch.cuda.synchronize()
+        n = int(cnt_ref[0])
+        assert int(cnt[0]) == n
+        assert torch.equal(idx[0, :n], idx_ref[0, :n])
