@@ -57,8 +57,9 @@
 namespace tw {
 
 constexpr int kSpWarps = kSpThreads / 32;
-constexpr int kMetaStagePages = 32;                      // 16 KB of page records per stage
-constexpr int kMetaStageBytes = kMetaStagePages * 2 * kHeadDim * 2;
+constexpr int kMetaStagePages = 64;     // page records per score stage at most (32 KB); a launch
+                                        // uses 64, or 32 when two CTAs share an SM
+constexpr int kMetaRecBytes = 2 * kHeadDim * 2;          // one page's min and max rows
 constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
 constexpr int kEstStageTok = kEstStagePages * kPage;
 constexpr int kSpBins = 4096;                            // first digit of the searches: 12 bits
@@ -83,11 +84,14 @@ struct SpKeyWidth {
 
 // Fixed part of the shared memory; the phase regions follow it.
 struct SpFixed {
-  uint64_t full1[kSpMaxStages], empty1[kSpMaxStages];
-  uint64_t full2[kSpMaxStages], empty2[kSpMaxStages];
+  __align__(16) __half qs[8][kHeadDim];   // the unit's query heads
+  uint64_t full1[kSpMaxStages];
+  int32_t pt1[kSpMaxStages][kMetaStagePages];   // paged: pool pages of each ring stage
+  uint64_t full2[kSpMaxStages];
   uint32_t pg[kSpSharePages];     // this CTA's share of the candidate list: page ids
   uint32_t r0[kSpSharePages];     // first physical row of each page
   int32_t nrow[kSpSharePages];    // valid rows of each page (0: not a page of the sequence)
+  int32_t crow[kSpSharePages];    // rows of each page copied (whole page, short at the allocation end)
   float2 wstat[kSpWarps][8];      // per warp and head: (max, sum 2^(l - max))
   float2 mz_loc[8];               // this CTA's pair per head
   float2 mz_all[kSpMaxCluster][8];   // every CTA's pair per head
@@ -113,6 +117,11 @@ constexpr size_t kSpFixedBytes = (sizeof(SpFixed) + 127) / 128 * 128;
 
 size_t sp_fixed_bytes() { return kSpFixedBytes; }
 
+__device__ __forceinline__ void cp_async16_sm(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async8_sm(void* smem, const void* gmem) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem)
                : "memory");
@@ -132,6 +141,13 @@ __device__ __forceinline__ void fence_proxy_async() {
 // a thread's run of E consecutive elements (E <= 32) is then conflict-free
 // when the threads of a warp read their runs in step.
 __host__ __device__ __forceinline__ int sp_pad(int i) { return i + (i >> 5); }
+
+// Words of a padded digit histogram of kSpBins bins (the bins a thread scans
+// are consecutive, so their padded words are conflict-free across a warp).
+constexpr int kSpHistWords = kSpBins + kSpBins / 32;
+constexpr int kSpHistBytes = kSpHistWords * 8;   // a digit histogram of 64-bit words
+constexpr int kSpLoBits = 19;
+constexpr int kPtAhead = 6;   // iterations between a page-table load and its store (< kSpWarps)   // low bits of a mass in a bin word's low half
 
 __device__ __forceinline__ float sp_h(uint32_t w, int hi) {
   return __half2float(__ushort_as_half((unsigned short)((w >> (16 * hi)) & 0xFFFFu)));
@@ -201,42 +217,90 @@ __device__ __forceinline__ unsigned sp_scan(unsigned v, unsigned* sh, unsigned* 
 template <int G>
 struct ScoreQ {
   static constexpr bool kSplit = G <= 4;
-  float a[G][8];   // q+ (split) or q
-  float c[kSplit ? G : 1][8];   // q- (split)
+  // split form: q+ = max(q, 0) and q- = min(q, 0) as fp16 bit patterns (exact);
+  // plain form: q as fp32
+  uint32_t ap[kSplit ? G : 1][4], an[kSplit ? G : 1][4];   // channel pairs (2i, 2i + 1)
+  float a[kSplit ? 1 : G][8];
 };
 
+// fp32 d = a * b + c for fp16 a, b: the product is exact in fp32 and the sum
+// is rounded once, as fmaf on the converted operands.
+__device__ __forceinline__ float fma_h(unsigned short a, unsigned short b, float c) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ unsigned short h_part(uint32_t w, int hi) {
+  return (unsigned short)((w >> (16 * hi)) & 0xFFFFu);
+}
+
+// The lane's partial of head g over its 8 channels of a page, left to right:
+// max(q_j min_j, q_j max_j) summed in fp32.
 template <int G>
-__device__ __forceinline__ float page_score(const ScoreQ<G>& Q, uint4 mn4, uint4 mx4,
-                                            unsigned hmask) {
-  const uint32_t wn[4] = {mn4.x, mn4.y, mn4.z, mn4.w};
-  const uint32_t wx[4] = {mx4.x, mx4.y, mx4.z, mx4.w};
-  float mn[8], mx[8];
+__device__ __forceinline__ float lane_partial(const ScoreQ<G>& Q, int g, const uint32_t (&wn)[4],
+                                              const uint32_t (&wx)[4]) {
+  if (ScoreQ<G>::kSplit) {
+    const int gs = ScoreQ<G>::kSplit ? g : 0;
+    // channel j: q+ max + q- min (one of the two is zero)
+    float s = fma_h(h_part(Q.ap[gs][0], 0), h_part(wx[0], 0), -0.0f);
+    s = fma_h(h_part(Q.an[gs][0], 0), h_part(wn[0], 0), s);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    mn[j] = sp_h(wn[j >> 1], j & 1);
-    mx[j] = sp_h(wx[j >> 1], j & 1);
+    for (int j = 1; j < 8; ++j) {
+      s = fma_h(h_part(Q.ap[gs][j >> 1], j & 1), h_part(wx[j >> 1], j & 1), s);
+      s = fma_h(h_part(Q.an[gs][j >> 1], j & 1), h_part(wn[j >> 1], j & 1), s);
+    }
+    return s;
   }
+  const int ga = ScoreQ<G>::kSplit ? 0 : g;
+  float s = fmaxf(__fmul_rn(Q.a[ga][0], sp_h(wn[0], 0)), __fmul_rn(Q.a[ga][0], sp_h(wx[0], 0)));
+#pragma unroll
+  for (int j = 1; j < 8; ++j) {
+    const float mn = sp_h(wn[j >> 1], j & 1), mx = sp_h(wx[j >> 1], j & 1);
+    s = __fadd_rn(s, fmaxf(__fmul_rn(Q.a[ga][j], mn), __fmul_rn(Q.a[ga][j], mx)));
+  }
+  return s;
+}
+
+// Scores of the NP (2 or 4) pages hw + 16 k of a ring stage, by the 16 lanes
+// of half-warp hw: each lane's partials, then per head the 16-lane sum in the
+// xor-butterfly order 8, 4, 2, 1, heads added in order.  The butterfly runs
+// transposed: at offset 8 a lane keeps the half of the pages on its side and
+// sends the other half, at offset 4 again, so each exchange moves one value
+// per page-pair instead of one per page; every page's sum is formed by the
+// same additions as a plain butterfly.  Lane l16 returns the score of page
+// (l16 >> 2) & 3 (NP = 4) or (l16 >> 3) & 1 (NP = 2).
+template <int G, int NP>
+__device__ __forceinline__ float page_scores(const ScoreQ<G>& Q, const unsigned char* st, int hw,
+                                             int l16, unsigned hmask) {
+  uint32_t wn[NP][4], wx[NP][4];
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    const uint4* rec = reinterpret_cast<const uint4*>(st + (hw + 16 * k) * 512);
+    const uint4 mn = rec[l16], mx = rec[16 + l16];
+    wn[k][0] = mn.x, wn[k][1] = mn.y, wn[k][2] = mn.z, wn[k][3] = mn.w;
+    wx[k][0] = mx.x, wx[k][1] = mx.y, wx[k][2] = mx.z, wx[k][3] = mx.w;
+  }
+  const bool b = (l16 >> 3) & 1, c = (l16 >> 2) & 1;
   float total = 0.f;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    float s;
-    if (ScoreQ<G>::kSplit) {
-      s = __fmul_rn(Q.a[g][0], mx[0]);
-      s = __fmaf_rn(Q.c[ScoreQ<G>::kSplit ? g : 0][0], mn[0], s);
+    float v[NP];
 #pragma unroll
-      for (int j = 1; j < 8; ++j) {
-        s = __fmaf_rn(Q.a[g][j], mx[j], s);
-        s = __fmaf_rn(Q.c[ScoreQ<G>::kSplit ? g : 0][j], mn[j], s);
-      }
+    for (int k = 0; k < NP; ++k) v[k] = lane_partial<G>(Q, g, wn[k], wx[k]);
+    float r;
+    if (NP == 4) {
+      const float r0 = __shfl_xor_sync(hmask, b ? v[0] : v[2], 8, 16);
+      const float r1 = __shfl_xor_sync(hmask, b ? v[1] : v[3], 8, 16);
+      const float k0 = __fadd_rn(b ? v[2] : v[0], r0), k1 = __fadd_rn(b ? v[3] : v[1], r1);
+      r = __fadd_rn(c ? k1 : k0, __shfl_xor_sync(hmask, c ? k0 : k1, 4, 16));
     } else {
-      s = fmaxf(__fmul_rn(Q.a[g][0], mn[0]), __fmul_rn(Q.a[g][0], mx[0]));
-#pragma unroll
-      for (int j = 1; j < 8; ++j)
-        s = __fadd_rn(s, fmaxf(__fmul_rn(Q.a[g][j], mn[j]), __fmul_rn(Q.a[g][j], mx[j])));
+      r = __fadd_rn(b ? v[1] : v[0], __shfl_xor_sync(hmask, b ? v[0] : v[1], 8, 16));
+      r = __fadd_rn(r, __shfl_xor_sync(hmask, r, 4, 16));
     }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(hmask, s, o, 16));
-    total = (g == 0) ? s : __fadd_rn(total, s);
+    r = __fadd_rn(r, __shfl_xor_sync(hmask, r, 2, 16));
+    r = __fadd_rn(r, __shfl_xor_sync(hmask, r, 1, 16));
+    total = (g == 0) ? r : __fadd_rn(total, r);
   }
   return total;
 }
@@ -285,9 +349,14 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& f
     const uint32_t dm = (1u << width) - 1u;
     nb = shift;
 #pragma unroll 1
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = key_at(i);
-      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dm], 1);
+    for (int c = i0; c < i1; c += 8) {   // eight keys to registers, then their reductions
+      uint32_t kv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kv[i] = c + i < i1 ? key_at(c + i) : 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c + i < i1 && (kv[i] & pmask) == prefix)
+          sm_red_add_u32(smem_u32(hist) + 4u * (uint32_t)sp_pad((int)((kv[i] >> shift) & dm)), 1u);
     }
     __syncthreads();
     // thread t holds digits [t bpt, t bpt + bpt); suffix sums from the top
@@ -297,7 +366,7 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& f
     int mine = 0;
     if (holder) {
 #pragma unroll 1
-      for (int k = 0; k < bpt; ++k) mine += hist[tid * bpt + k];
+      for (int k = 0; k < bpt; ++k) mine += (int)sm_ld_u32(smem_u32(&hist[sp_pad(tid * bpt + k)]));
     }
     int incl = mine;
 #pragma unroll
@@ -318,7 +387,7 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& f
 #pragma unroll 1
       for (int k = bpt - 1; k >= 0; --k) {
         const int d = tid * bpt + k;
-        const int here = above + hist[d];
+        const int here = above + (int)sm_ld_u32(smem_u32(&hist[sp_pad(d)]));
         if (here >= need && above < need) {
           fx.sh_d = d;
           fx.sh_need = above;
@@ -330,7 +399,7 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& f
     __syncthreads();   // every thread is done reading the histogram
     if (holder) {
 #pragma unroll 1
-      for (int k = 0; k < bpt; ++k) hist[tid * bpt + k] = 0;
+      for (int k = 0; k < bpt; ++k) sm_st_u32(smem_u32(&hist[sp_pad(tid * bpt + k)]), 0u);
     }
     need -= fx.sh_need;
     prefix |= (uint32_t)fx.sh_d << shift;
@@ -408,54 +477,75 @@ __device__ __forceinline__ unsigned long long sp_join(uint32_t hi, uint32_t lo) 
 // consecutive positions [t R, t R + R) (-1 marks an invalid position).
 struct SpWeights {
   float* base;
-  bool pad;   // shared-memory positions padded one word per 32
+  bool pad;        // in shared memory, positions padded one word per 32
+  uint32_t sbase;  // shared address of base when pad
   int lp0, R, npos;
   __device__ __forceinline__ float at(int i) const {
     const int lp = lp0 + i;
-    return base[pad ? sp_pad(lp) : lp];
+    if (pad) return __uint_as_float(sm_ld_u32(sbase + 4u * (uint32_t)sp_pad(lp)));
+    return base[lp];
   }
 };
 
 // Histogram the masses of this thread's weights that lie in the current
-// prefix range by digit (key >> shift) & dm: exact 64-bit sums from native
-// 32-bit atomics on a low and a high word with an explicit carry.
+// prefix range by digit (key >> shift) & dm.  A bin is one 64-bit word
+// holding two 32-bit sums: the low kSpLoBits bits of each mass in the low
+// half, the rest in the high half, each added by a native 32-bit shared
+// reduction (a 64-bit one costs a compare-and-swap loop under contention).
+// Neither half overflows: a CTA holds at most kSpSharePages * kPage weights,
+// so the low sums stay below 2^(kSpLoBits + 13), and the weights of a set sum
+// to about 1, so the high sums stay near 2^(40 - kSpLoBits).  Weights are read
+// eight at a time before their reductions.
 __device__ __forceinline__ void mass_hist(const SpWeights& W, int shift, uint32_t dm,
-                                          const SpSearch& s, uint32_t* hlo, uint32_t* hhi) {
+                                          const SpSearch& s, unsigned long long* hist) {
+  const uint32_t h0 = smem_u32(hist);
 #pragma unroll 1
-  for (int i = 0; i < W.R; ++i) {
-    if (W.lp0 + i >= W.npos) break;
-    const float w = W.at(i);
-    if (w >= 0.f) {
-      const uint32_t key = __float_as_uint(w);
-      if ((key & s.pmask) == s.prefix) {
-        const unsigned long long F = sp_mass(w);
-        const uint32_t dg = (key >> shift) & dm;
-        const uint32_t lo = (uint32_t)F;
-        const uint32_t old = atomicAdd(&hlo[dg], lo);
-        const uint32_t up = (uint32_t)(F >> 32) + (old + lo < old ? 1u : 0u);
-        if (up) atomicAdd(&hhi[dg], up);
+  for (int c = 0; c < W.R; c += 8) {
+    float wv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      wv[i] = (c + i < W.R && W.lp0 + c + i < W.npos) ? W.at(c + i) : -1.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t key = __float_as_uint(wv[i]);
+      if (wv[i] >= 0.f && (key & s.pmask) == s.prefix) {
+        const unsigned long long m = sp_mass(wv[i]);
+        const uint32_t a = h0 + 8u * (uint32_t)sp_pad((int)((key >> shift) & dm));
+        sm_red_add_u32(a, (uint32_t)m & ((1u << kSpLoBits) - 1u));
+        sm_red_add_u32(a + 4u, (uint32_t)(m >> kSpLoBits));
       }
     }
   }
 }
 
-// Mass of digit d summed over every CTA of the cluster (the CTAs' words are
-// requested before any is added).
-__device__ __forceinline__ unsigned long long cluster_bin(const uint32_t* hlo,
-                                                          const uint32_t* hhi, int d, int CS) {
-  uint32_t lv[kSpMaxCluster], hv[kSpMaxCluster];
+// The mass of a bin word written by mass_hist.
+__device__ __forceinline__ unsigned long long sp_bin_mass(unsigned long long v) {
+  return ((v >> 32) << kSpLoBits) + (v & 0xFFFFFFFFull);
+}
+
+// The masses of digits base + k * kSpThreads + tid (k < nk) summed over the
+// CST CTAs of the cluster and written back, decoded, over this CTA's own
+// words of those digits (no peer reads them).  Consecutive threads read
+// consecutive words of a peer; nk * CST <= 16, and all of the remote words
+// are requested before any is added.
+template <int CST>
+__device__ __forceinline__ void cluster_bins(unsigned long long* hist, int base, int nk) {
+  constexpr int KMAX = 16 / CST;
+  const int tid = threadIdx.x;
+  unsigned long long v[KMAX][CST];
 #pragma unroll
-  for (int r = 0; r < kSpMaxCluster; ++r) {
-    lv[r] = hv[r] = 0u;
-    if (r < CS) {
-      lv[r] = ld_peer_u32(peer_addr(&hlo[d], r));
-      hv[r] = ld_peer_u32(peer_addr(&hhi[d], r));
-    }
+  for (int k = 0; k < KMAX; ++k)
+#pragma unroll
+    for (int r = 0; r < CST; ++r)
+      v[k][r] = k < nk ? ld_peer_u64(peer_addr(&hist[sp_pad(base + k * kSpThreads + tid)], (uint32_t)r))
+                       : 0ull;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    unsigned long long t = 0;
+#pragma unroll
+    for (int r = 0; r < CST; ++r) t += sp_bin_mass(v[k][r]);
+    if (k < nk) sm_st_u64(smem_u32(&hist[sp_pad(base + k * kSpThreads + tid)]), t);
   }
-  unsigned long long t = 0;
-#pragma unroll
-  for (int r = 0; r < kSpMaxCluster; ++r) t += sp_join(hv[r], lv[r]);
-  return t;
 }
 
 // One digit of the threshold search (NB digits; NB = 4096 for the first).
@@ -468,27 +558,37 @@ __device__ __forceinline__ unsigned long long cluster_bin(const uint32_t* hlo,
 // from the total mass and returns false if that is zero.  Leaves this CTA's
 // histogram zeroed.
 __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, double p, int CS,
-                           int cr, uint32_t* hlo, uint32_t* hhi, SpFixed& fx, SpSearch& s) {
+                           int cr, unsigned long long* hist, SpFixed& fx, SpSearch& s) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  mass_hist(W, shift, dm, s, hlo, hhi);
+  mass_hist(W, shift, dm, s, hist);
   if (CS > 1) cluster_sync();   // every CTA's histogram is complete
   else __syncthreads();
   const int SB = NB / CS;                                    // digits of this CTA's slice
   const int bpt = SB > kSpThreads ? SB / kSpThreads : 1;     // digits per thread (<= 16)
   const int first = cr * SB + tid * bpt;
   const bool holder = tid * bpt < SB;
+  // the slice's masses over the cluster, decoded in place: thread t reduces
+  // digits cr * SB + k * 256 + t (coalesced), then holds bpt consecutive ones
+  if (tid < SB) {
+    switch (CS) {
+      case 1:
+#pragma unroll 1
+        for (int k = 0; k < bpt; ++k) {
+          const uint32_t ad = smem_u32(&hist[sp_pad(k * kSpThreads + tid)]);
+          sm_st_u64(ad, sp_bin_mass(sm_ld_u64(ad)));
+        }
+        break;
+      case 2: cluster_bins<2>(hist, cr * SB, bpt); break;
+      case 4: cluster_bins<4>(hist, cr * SB, bpt); break;
+      case 8: cluster_bins<8>(hist, cr * SB, bpt); break;
+      default: cluster_bins<16>(hist, cr * SB, bpt); break;
+    }
+  }
+  __syncthreads();
   unsigned long long mine = 0;   // this thread's digits' mass
   if (holder) {
 #pragma unroll 1
-    for (int k = 0; k < bpt; ++k) {
-      const int d = first + k;
-      const unsigned long long v = CS == 1 ? sp_join(hhi[d], hlo[d]) : cluster_bin(hlo, hhi, d, CS);
-      if (CS > 1) {
-        hlo[d] = (uint32_t)v;
-        hhi[d] = (uint32_t)(v >> 32);
-      }
-      mine += v;
-    }
+    for (int k = 0; k < bpt; ++k) mine += sm_ld_u64(smem_u32(&hist[sp_pad(first + k)]));
   }
   unsigned long long incl = mine;   // suffix over this warp's higher lanes
 #pragma unroll
@@ -537,18 +637,23 @@ __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, d
 #pragma unroll 1
     for (int k = bpt - 1; k >= 0; --k) {
       const int d = first + k;
-      const unsigned long long here = above + sp_join(hhi[d], hlo[d]);
+      const unsigned long long here = above + sm_ld_u64(smem_u32(&hist[sp_pad(d)]));
       if (here >= s.T && above < s.T) {
-        for (int r = 0; r < CS; ++r) {
-          st_peer_u32(peer_addr(&fx.sh_d, r), (uint32_t)d);
-          st_peer_u64(peer_addr(&fx.sh_above, r), above - s.A);
+        if (CS == 1) {   // this CTA alone (also inside a larger cluster)
+          fx.sh_d = d;
+          fx.sh_above = above - s.A;
+        } else {
+          for (int r = 0; r < CS; ++r) {
+            st_peer_u32(peer_addr(&fx.sh_d, r), (uint32_t)d);
+            st_peer_u64(peer_addr(&fx.sh_above, r), above - s.A);
+          }
         }
       }
       above = here;
     }
   }
   __syncthreads();   // every thread is done with the histogram words it holds
-  for (int i = tid; i < NB; i += kSpThreads) hlo[i] = hhi[i] = 0u;
+  for (int i = tid; i < sp_pad(NB); i += kSpThreads) sm_st_u64(smem_u32(&hist[i]), 0ull);
   if (CS > 1) cluster_sync();   // the digit is in every CTA's shared memory
   else __syncthreads();
   if (ok) {
@@ -592,7 +697,7 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
   else __syncthreads();
   // every CTA's count (lanes r < CS), and the gathered list in warp 0
   int cnt = 0;
-  if (lane < CS) cnt = (int)ld_peer_u32(peer_addr(&fx.lst_n, (uint32_t)lane));
+  if (lane < CS) cnt = CS == 1 ? fx.lst_n : (int)ld_peer_u32(peer_addr(&fx.lst_n, (uint32_t)lane));
   int before = cnt;   // inclusive prefix over the CTAs
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -618,8 +723,8 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
       }
     }
     if (mine) {
-      key = ld_peer_u32(peer_addr(&fx.lst_key[lane - start], (uint32_t)src));
-      pos = ld_peer_u32(peer_addr(&fx.lst_pos[lane - start], (uint32_t)src));
+      key = CS == 1 ? fx.lst_key[lane] : ld_peer_u32(peer_addr(&fx.lst_key[lane - start], (uint32_t)src));
+      pos = CS == 1 ? fx.lst_pos[lane] : ld_peer_u32(peer_addr(&fx.lst_pos[lane - start], (uint32_t)src));
     }
     // rank in the order (weight descending, position ascending)
     int rank = 0;
@@ -656,7 +761,7 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
 
 // ---------------------------------------------------------------------------
 template <int G, int BITS>
-__global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
+__global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpArgs a) {
   using KW = SpKeyWidth<BITS>;
   extern __shared__ __align__(128) unsigned char sp_smem[];
   SpFixed& fx = *reinterpret_cast<SpFixed*>(sp_smem);
@@ -670,15 +775,17 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
   const bool paged = L.page_table != nullptr;
   if (tid == 0) {
     for (int s = 0; s < kSpMaxStages; ++s) {
-      mbar_init(&fx.full1[s], 1);
-      mbar_init(&fx.empty1[s], kSpWarps);
-      mbar_init(&fx.full2[s], 1 + 32);   // the byte-count arrival + warp 0's cp.async arrivals
-      mbar_init(&fx.empty2[s], kSpWarps);
+      mbar_init(&fx.full1[s], paged ? kSpThreads : 1);   // cp.async arrivals, or the byte count
+      mbar_init(&fx.full2[s], kSpThreads);   // every thread's cp.async arrival
     }
     mbar_fence_init();
   }
   __syncthreads();
   griddep_wait();
+  for (int i = tid; i < G * kHeadDim / 8; i += kSpThreads)   // 16-byte pieces of the G query rows
+    reinterpret_cast<uint4*>(&fx.qs[0][0])[i] =
+        __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.Hq + hk * G) * kHeadDim) + i);
+  __syncthreads();
   const int len = L.len(b);
   const int P = (len + kPage - 1) / kPage;
   int nsel = 0;          // candidate pages of the unit
@@ -689,98 +796,151 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     // ---------------- phase 1: page scores of pages [pA, pB) ----------------
     const int pA = (int)((int64_t)cr * P / CS), pB = (int)((int64_t)(cr + 1) * P / CS);
     const int npg = pB - pA;
-    const int nst = (npg + kMetaStagePages - 1) / kMetaStagePages;
+    const int mp = a.mp1;                       // pages per stage (32 or 64)
+    const int nst = (npg + mp - 1) / mp;
     unsigned char* ring = region;
-    uint32_t* skeys = reinterpret_cast<uint32_t*>(region + (size_t)a.s1 * kMetaStageBytes);
+    const size_t stage1 = (size_t)mp * kMetaRecBytes;
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(region + (size_t)a.s1 * stage1);
     const bool gk = a.gkeys != nullptr;   // keys in global memory (P above the shared capacity)
     uint32_t* gkeys = gk ? a.gkeys + (int64_t)u * L.max_pages : nullptr;
     const __half* meta = a.meta;
     const int64_t meta_unit = (int64_t)u * L.max_pages;   // contiguous record index of page 0
-    auto pt_of = [&](int k) -> int {   // warp 0: page-table entry of page lane of stage k
-      const int pg = pA + k * kMetaStagePages + lane;
-      if (!paged || k >= nst || pg >= pB) return 0;
-      const int e = L.page_table[(int64_t)b * L.max_pages + pg];
-      return (unsigned)e < (unsigned)L.pool_pages ? e : 0;
-    };
-    auto issue1 = [&](int k, int slot, int ptv) {   // warp 0
-      const int n = min(kMetaStagePages, npg - k * kMetaStagePages);
-      unsigned char* dst = ring + (size_t)slot * kMetaStageBytes;
-      if (paged) {
-        if (lane < n)
-          bulk_g2s(dst + lane * 512, meta + ((int64_t)ptv * L.Hk + hk) * (2 * kHeadDim), 512,
-                   &fx.full1[slot]);
-      } else if (lane == 0) {
-        bulk_g2s(dst, meta + (meta_unit + pA + (int64_t)k * kMetaStagePages) * (2 * kHeadDim),
-                 (uint32_t)n * 512u, &fx.full1[slot]);
+    // Stage k (up to 32 pages of the slice) into ring slot `slot`.  A
+    // contiguous cache's records of the slice are one run: one bulk copy by
+    // thread 0 completes on the stage's full barrier with its byte count.  A
+    // paged cache's records are 512-byte pieces spread over the pool: every
+    // thread copies two 16-byte parts by cp.async (pool pages from the
+    // page-table entries staged one iteration earlier) and arrives when they
+    // have landed.
+    // warp 0, lane i: the pool pages of pages i and i + 32 of stage k (0 past the slice)
+    auto fetch_pt = [&](int k) -> int2 {
+      int e[2] = {0, 0};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int pg = pA + k * mp + lane + 32 * h;
+        if (paged && k < nst && lane + 32 * h < mp && pg < pB) {
+          const int v = L.page_table[(int64_t)b * L.max_pages + pg];
+          e[h] = (unsigned)v < (unsigned)L.pool_pages ? v : 0;
+        }
       }
-      if (lane == 0) mbar_arrive_tx(&fx.full1[slot], (uint32_t)n * 512u);
+      return make_int2(e[0], e[1]);
     };
-    int ptn = 0;
-    if (warp == 0) {
-      int ptq[kSpMaxStages];
+    auto store_pt = [&](int slot, int2 e) {
+      fx.pt1[slot][lane] = e.x;
+      fx.pt1[slot][lane + 32] = e.y;
+    };
+    auto issue1 = [&](int k, int slot) {
+      const int n = k < nst ? min(mp, npg - k * mp) : 0;
+      unsigned char* dst = ring + (size_t)slot * stage1;
+      if (paged) {
 #pragma unroll
-      for (int k = 0; k < kSpMaxStages; ++k) ptq[k] = (k < a.s1) ? pt_of(k) : 0;
+        for (int x0 = 0; x0 < kMetaStagePages * 32; x0 += kSpThreads) {   // n <= mp pages of 32 parts
+          const int x = x0 + tid, i = x >> 5, c = x & 31;
+          if (i < n)
+            cp_async16_sm(dst + i * 512 + c * 16,
+                          meta + ((int64_t)fx.pt1[slot][i] * L.Hk + hk) * (2 * kHeadDim) + c * 8);
+        }
+        cp_async_arrive_noinc(&fx.full1[slot]);
+      } else if (tid == 0) {
+        fence_proxy_async();   // the slot's earlier readers are ordered before the copy
+        if (n > 0)
+          bulk_g2s(dst, meta + (meta_unit + pA + (int64_t)k * mp) * (2 * kHeadDim),
+                   (uint32_t)n * 512u, &fx.full1[slot]);
+        mbar_arrive_tx(&fx.full1[slot], (uint32_t)n * 512u);
+      }
+    };
+    // page-table entries: stages 0 .. S-1 staged now.  The entries of stage
+    // k >= S are loaded by warp k % 8 into its registers kPtAhead iterations
+    // before they are stored (at the end of iteration k - S, into the slot
+    // stage k - S used), so a load's latency spreads over several iterations
+    // and no barrier waits on one.
+    int2 ptn = make_int2(0, 0);
+    if (paged) {
+      if (warp == 0) {
+        int2 ptq[kSpMaxStages];
 #pragma unroll
-      for (int k = 0; k < kSpMaxStages; ++k)
-        if (k < a.s1 && k < nst) issue1(k, k, ptq[k]);
-      ptn = pt_of(a.s1);
+        for (int k = 0; k < kSpMaxStages; ++k) ptq[k] = k < a.s1 ? fetch_pt(k) : make_int2(0, 0);
+#pragma unroll
+        for (int k = 0; k < kSpMaxStages; ++k)
+          if (k < a.s1) store_pt(k, ptq[k]);
+      }
+#pragma unroll 1
+      for (int i = 0; i < kPtAhead; ++i)
+        if (warp == (a.s1 + i) % kSpWarps) ptn = fetch_pt(a.s1 + i);
     }
+    __syncthreads();
+#pragma unroll 1
+    for (int k = 0; k < a.s1 - 1; ++k) issue1(k, k);
     // the query channels of this lane (8 per head) for the group's heads
     const int l16 = lane & 15, hw = tid >> 4;
     const unsigned hmask = 0xFFFFu << (lane & 16);
     ScoreQ<G> Q;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const uint4 r = __ldg(reinterpret_cast<const uint4*>(
-          a.q + ((int64_t)b * a.Hq + hk * G + g) * kHeadDim + l16 * 8));
+      const uint4 r = *reinterpret_cast<const uint4*>(&fx.qs[g][l16 * 8]);
       const uint32_t wq[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        const unsigned short hbits = h_part(wq[j >> 1], j & 1);
         const float x = sp_h(wq[j >> 1], j & 1);
         if (ScoreQ<G>::kSplit) {
-          Q.a[g][j] = x >= 0.f ? x : 0.f;
-          Q.c[ScoreQ<G>::kSplit ? g : 0][j] = x >= 0.f ? 0.f : x;
+          const int gs = ScoreQ<G>::kSplit ? g : 0;
+          const uint32_t sh = 16u * (uint32_t)(j & 1);
+          if (!(j & 1)) Q.ap[gs][j >> 1] = Q.an[gs][j >> 1] = 0u;
+          // q+ (+0 when q < 0) and q- (+0 when q >= 0)
+          Q.ap[gs][j >> 1] |= (uint32_t)(x >= 0.f ? hbits : (unsigned short)0) << sh;
+          Q.an[gs][j >> 1] |= (uint32_t)(x >= 0.f ? (unsigned short)0 : hbits) << sh;
         } else {
-          Q.a[g][j] = x;
+          Q.a[ScoreQ<G>::kSplit ? 0 : g][j] = x;
         }
       }
     }
     for (int j = 0; j < nst; ++j) {
+      // refill: stage j + S - 1 into the slot stage j - 1 used (freed by the
+      // barrier that ended the previous iteration); then the page-table
+      // entries of stage j + S into the slot stage j's entries used
+      issue1(j + a.s1 - 1, (j + a.s1 - 1) % a.s1);
       const int slot = j % a.s1;
       const uint32_t par = (uint32_t)((j / a.s1) & 1);
       if (!failed) failed = !mbar_wait(&fx.full1[slot], par, a.status);
-      const int n = min(kMetaStagePages, npg - j * kMetaStagePages);
-      const unsigned char* st = ring + (size_t)slot * kMetaStageBytes;
-#pragma unroll
-      for (int k = 0; k < kMetaStagePages / 16; ++k) {
-        const int i = hw + 16 * k;
-        if (i < n) {   // uniform across the half-warp
-          const uint4* rec = reinterpret_cast<const uint4*>(st + i * 512);
-          const float score = page_score<G>(Q, rec[l16], rec[16 + l16], hmask);
-          const uint32_t key = f_key(score);
-          const int pg = pA + j * kMetaStagePages + i;
-          if (gk) {
-            if (l16 == 0) gkeys[pg] = key;
-          } else if (l16 < CS) {
-            st_peer_u32(peer_addr(&skeys[sp_pad(pg)], (uint32_t)l16), key);
-          }
+      const int n = min(mp, npg - j * mp);
+      const unsigned char* st = ring + (size_t)slot * stage1;
+      // every page of the stage is scored (records past n are stale and
+      // their scores unused); lane l16 then holds page hw + 16 kp, shared
+      // with the other lanes of its group of 16 / np, which split the stores
+      const bool four = mp == 4 * 16;
+      const float score = four ? page_scores<G, 4>(Q, st, hw, l16, hmask)
+                               : page_scores<G, 2>(Q, st, hw, l16, hmask);
+      const int kp = four ? (l16 >> 2) & 3 : (l16 >> 3) & 1;
+      const int rr = four ? (l16 & 3) : (l16 & 7), step = four ? 4 : 8;
+      const int i = hw + 16 * kp;
+      if (i < n) {
+        const uint32_t key = f_key(score);
+        const int pg = pA + j * mp + i;
+        if (gk) {
+          if (rr == 0) gkeys[pg] = key;
+        } else {
+          for (int r = rr; r < CS; r += step) st_peer_u32(peer_addr(&skeys[sp_pad(pg)], (uint32_t)r), key);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&fx.empty1[slot]);
-      if (warp == 0 && j + a.s1 < nst) {
-        if (!failed) failed = !mbar_wait(&fx.empty1[slot], par, a.status);
-        issue1(j + a.s1, slot, ptn);
-        ptn = pt_of(j + a.s1 + 1);
+      // the entries of stage j + S go where stage j's were (read when stage j
+      // was issued, S - 1 iterations ago); stage j + S + kPtAhead's are loaded
+      if (paged) {
+        if (warp == (j + a.s1) % kSpWarps) store_pt(j % a.s1, ptn);
+        if (warp == (j + a.s1 + kPtAhead) % kSpWarps) ptn = fetch_pt(j + a.s1 + kPtAhead);
       }
+      __syncthreads();   // slot j is free; the staged entries are visible
     }
     cluster_sync();   // every CTA holds all P keys (or they are in global memory)
 
     // ---------------- top-K_p and this CTA's share of the candidate list ----------------
     const int K = min(a.budget_pages, P);
-    auto key_at = [&](int i) -> uint32_t { return gk ? __ldcg(gkeys + i) : skeys[sp_pad(i)]; };
+    const uint32_t skeys_s = smem_u32(skeys);
+    auto key_at = [&](int i) -> uint32_t {
+      return gk ? __ldcg(gkeys + i) : sm_ld_u32(skeys_s + 4u * (uint32_t)sp_pad(i));
+    };
     int* hist = reinterpret_cast<int*>(ring);   // the meta ring is idle now
-    for (int i = tid; i < kSpBins; i += kSpThreads) hist[i] = 0;
+    for (int i = tid; i < kSpHistWords; i += kSpThreads) hist[i] = 0;
     __syncthreads();
     const bool all = K >= P;
     if (!all) topk_threshold(key_at, P, K, hist, fx);
@@ -838,6 +998,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     const int pg = (int)fx.pg[i];
     const bool valid = pg >= 0 && pg < P;
     fx.nrow[i] = valid ? min(kPage, len - pg * kPage) : 0;
+    fx.crow[i] = !valid ? 0 : ((!paged && pg * kPage + kPage > L.N) ? L.N - pg * kPage : kPage);
     fx.r0[i] = valid ? (uint32_t)L.page_row(b, hk, pg) : 0u;
   }
   __syncthreads();
@@ -846,7 +1007,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     // ---------------- phase 2: weight estimate of the share ----------------
     const int nst = (ns + kEstStagePages - 1) / kEstStagePages;
     unsigned char* ring = region;
-    const int ring_bytes = max(a.s2 * KW::kStageBytes, 2 * kSpBins * 4);
+    const int ring_bytes = max(a.s2 * KW::kStageBytes, kSpHistBytes + (a.local_pos ? sp_pad(a.local_pos) * 4 : 0));
     // logits [head][local position]: in shared memory (positions padded one
     // word per 32, so a thread's run of R consecutive positions is free of
     // bank conflicts) or at the set's positions [s0 * 16, ..) of the global
@@ -865,48 +1026,46 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     const uint8_t* codes = a.codes;
     const __half* scales = a.scales;
     const __half* zeros = a.zeros;
-    auto issue2 = [&](int k, int slot) {   // warp 0
-      const int npgs = min(kEstStagePages, ns - k * kEstStagePages);
-      unsigned char* st = ring + (size_t)slot * KW::kStageBytes;
-      unsigned char* st_codes = st;
-      unsigned char* st_scales = st + kEstStageTok * KW::kRowBytes;
-      unsigned char* st_zeros = st_scales + kEstStageTok * kGroups * 2;
-      // lane i < npgs: page i of the stage; rows copied = its valid rows
-      // rounded up to the page, except where the page runs past the cache's
-      // allocation (a contiguous cache whose length is not a multiple of 16)
-      int crow = 0;
-      uint32_t r0 = 0;
-      if (lane < npgs) {
-        const int e = k * kEstStagePages + lane;
-        const int pg = (int)fx.pg[e];
-        r0 = fx.r0[e];
-        if (fx.nrow[e] > 0) crow = (!paged && pg * kPage + kPage > L.N) ? L.N - pg * kPage : kPage;
-        if (crow > 0)
-          bulk_g2s(st_codes + lane * kPage * KW::kRowBytes, codes + (size_t)r0 * KW::kRowBytes,
-                   (uint32_t)(crow * KW::kRowBytes), &fx.full2[slot]);
-      }
-      // scales and zeros: 8 bytes per row by cp.async, row x of the stage per lane
+    // Stage k of the share (up to 16 candidate pages) into ring slot `slot`,
+    // by all threads with cp.async: the pages' code rows in 16-byte pieces,
+    // their scale and zero rows in 8-byte pieces; every thread then arrives
+    // on the stage's full barrier when its copies have landed.  Rows copied
+    // per page: the whole page, except where it runs past a contiguous
+    // cache's allocation (length not a multiple of 16); pages outside the
+    // sequence copy nothing.
+    auto issue2 = [&](int k, int slot) {
+      if (k < nst) {
+        const int npgs = min(kEstStagePages, ns - k * kEstStagePages);
+        unsigned char* st = ring + (size_t)slot * KW::kStageBytes;
+        unsigned char* st_codes = st;
+        unsigned char* st_scales = st + kEstStageTok * KW::kRowBytes;
+        unsigned char* st_zeros = st_scales + kEstStageTok * kGroups * 2;
+        constexpr int kPieces = KW::kRowBytes;   // 16-byte pieces of a page's code rows
 #pragma unroll
-      for (int x0 = 0; x0 < kEstStageTok; x0 += 32) {
-        const int x = x0 + lane, pi = x >> 4, r = x & 15;
-        const int cr_p = __shfl_sync(0xffffffffu, crow, pi);
-        const uint32_t r0_p = __shfl_sync(0xffffffffu, r0, pi);
-        if (r < cr_p) {
-          cp_async8_sm(st_scales + x * 8, scales + ((size_t)r0_p + r) * kGroups);
-          cp_async8_sm(st_zeros + x * 8, zeros + ((size_t)r0_p + r) * kGroups);
+        for (int x0 = 0; x0 < kEstStagePages * kPieces; x0 += kSpThreads) {
+          const int x = x0 + tid, pi = x / kPieces, c = x % kPieces;
+          if (pi < npgs) {
+            const int e = k * kEstStagePages + pi;
+            if (16 * c < fx.crow[e] * KW::kRowBytes)
+              cp_async16_sm(st_codes + pi * kPage * KW::kRowBytes + 16 * c,
+                            codes + (size_t)fx.r0[e] * KW::kRowBytes + 16 * c);
+          }
+        }
+        {
+          const int pi = tid >> 4, r = tid & 15;
+          if (pi < npgs) {
+            const int e = k * kEstStagePages + pi;
+            if (r < fx.crow[e]) {
+              cp_async8_sm(st_scales + tid * 8, scales + ((size_t)fx.r0[e] + r) * kGroups);
+              cp_async8_sm(st_zeros + tid * 8, zeros + ((size_t)fx.r0[e] + r) * kGroups);
+            }
+          }
         }
       }
       cp_async_arrive_noinc(&fx.full2[slot]);
-      uint32_t bytes = (uint32_t)(crow * KW::kRowBytes);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-      if (lane == 0) mbar_arrive_tx(&fx.full2[slot], bytes);
     };
-    if (warp == 0) {
-      fence_proxy_async();   // the ring was written by threads before; the copies come after
 #pragma unroll 1
-      for (int k = 0; k < a.s2 && k < nst; ++k) issue2(k, k);
-    }
+    for (int k = 0; k < a.s2 - 1; ++k) issue2(k, k);
     constexpr int HP = (G + 1) / 2;   // head pairs: one MMA N-block of 8 (head, group) columns each
     const int gid = lane >> 2, t = lane & 3;
     const int g0 = 2 * (t & 1);
@@ -916,7 +1075,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     for (int hp = 0; hp < HP; ++hp) {
       const int hb = 2 * hp + (gid >> 2);
       const bool on = ((gid & 3) == t) && hb < G;
-      const __half* qb = a.q + ((int64_t)b * a.Hq + hk * G + min(hb, G - 1)) * kHeadDim;
+      const __half* qb = fx.qs[min(hb, G - 1)];
       const __half z = __float2half_rn(0.f);
       const __half* qg = qb + kGroup * t;
 #pragma unroll
@@ -925,7 +1084,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
         for (int jj = 0; jj < 2; ++jj)
           bfr[hp][s][jj] = sp_pack_h2(on ? qg[KW::chan(s, jj, 0)] : z, on ? qg[KW::chan(s, jj, 1)] : z);
       const int he = 2 * hp + (t >> 1);
-      const __half* qe = a.q + ((int64_t)b * a.Hq + hk * G + min(he, G - 1)) * kHeadDim;
+      const __half* qe = fx.qs[min(he, G - 1)];
       float q0 = 0.f, q1 = 0.f;
       for (int d = 0; d < kGroup; ++d) {
         q0 += __half2float(qe[g0 * kGroup + d]);
@@ -942,6 +1101,9 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     }
     const bool owner = (t & 1) == 0;   // lanes t and t^1 hold the same logits
     for (int j = 0; j < nst; ++j) {
+      // refill: stage j + S - 1 into the slot stage j - 1 used (freed by the
+      // barrier that ended the previous iteration)
+      issue2(j + a.s2 - 1, (j + a.s2 - 1) % a.s2);
       const int slot = j % a.s2;
       const uint32_t par = (uint32_t)((j / a.s2) & 1);
       if (!failed) failed = !mbar_wait(&fx.full2[slot], par, a.status);
@@ -1043,12 +1205,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
           Mrun[hp] = mn;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&fx.empty2[slot]);
-      if (warp == 0 && j + a.s2 < nst) {
-        if (!failed) failed = !mbar_wait(&fx.empty2[slot], par, a.status);
-        issue2(j + a.s2, slot);
-      }
+      __syncthreads();   // every warp is done with this slot before it is refilled
     }
     // per-warp statistics -> the CTA's -> every CTA's, merged in rank order
 #pragma unroll
@@ -1090,9 +1247,9 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
     }
 
     // ---------------- top-p per selection set ----------------
-    uint32_t* hlo = reinterpret_cast<uint32_t*>(ring);   // the estimate ring is idle now
-    uint32_t* hhi = hlo + kSpBins;
-    uint32_t* obuf = hlo;
+    // the estimate ring is idle now: the digit histogram, then the staged output
+    unsigned long long* hist = reinterpret_cast<unsigned long long*>(ring);
+    uint32_t* obuf = reinterpret_cast<uint32_t*>(ring);
     const int npos = ns * kPage;                                  // local positions of the share
     const int R = (npos + kSpThreads - 1) / kSpThreads;   // <= 32 (host-checked)
     const int lp0 = tid * R;
@@ -1101,10 +1258,11 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
       const int set = a.group_sets ? u : b * a.Hq + hk * G + hs;
       const int h0 = a.group_sets ? 0 : hs, nh = a.group_sets ? G : 1;
       __syncthreads();   // the ring (or the previous set's staged output) is free
-      for (int i = tid; i < 2 * kSpBins; i += kSpThreads) hlo[i] = 0u;
+      for (int i = tid; i < kSpHistWords; i += kSpThreads) hist[i] = 0ull;
       // the set's weights, written over the logits of its first head (each
       // thread reads and writes only its own positions)
-      SpWeights W{lbase + h0 * hstride, lpad, lp0, R, npos};
+      SpWeights W{lbase + h0 * hstride, lpad,
+                  lpad ? smem_u32(lbase + h0 * hstride) : 0u, lp0, R, npos};
 #pragma unroll 1
       for (int i = 0; i < R; ++i) {
         const int lp = lp0 + i;
@@ -1119,6 +1277,28 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
         }
         lbase[lidx(h0, lp)] = ok ? acc : -1.0f;
       }
+      // A set of at most local_pos positions is gathered whole into every
+      // CTA of the cluster (after the histogram words of the ring), and each
+      // CTA searches and compacts it alone: one cluster barrier instead of
+      // several per digit.  Each CTA then writes the outputs of its own share.
+      const bool local = CS > 1 && nsel * kPage <= a.local_pos;
+      SpWeights WS = W;
+      int CSs = CS, crs = cr, pos0s = s0 * kPage;
+      if (local) {
+        float* wall = reinterpret_cast<float*>(ring + kSpHistBytes);
+        __syncthreads();   // this CTA's weights are complete
+        for (int i = tid; i < npos; i += kSpThreads) {
+          const uint32_t w = __float_as_uint(lbase[lidx(h0, i)]);
+          const float* dst = wall + sp_pad(s0 * kPage + i);
+          for (int r = 0; r < CS; ++r) st_peer_u32(peer_addr(dst, (uint32_t)r), w);
+        }
+        cluster_sync();   // every CTA holds the whole set
+        const int npa = nsel * kPage, Ra = (npa + kSpThreads - 1) / kSpThreads;
+        WS = SpWeights{wall, true, smem_u32(wall), tid * Ra, Ra, npa};
+        CSs = 1;
+        crs = 0;
+        pos0s = 0;
+      }
       const bool keep_all = a.p >= 1.0;
       uint32_t theta = 0;
       unsigned long long r_need = 0;
@@ -1129,12 +1309,12 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
         bool done_small = false;
 #pragma unroll 1
         for (int step = 0; step < 3; ++step) {
-          const bool ok = digit_step(W, step == 0 ? 18 : (step == 1 ? 9 : 0),
+          const bool ok = digit_step(WS, step == 0 ? 18 : (step == 1 ? 9 : 0),
                                      step == 0 ? 0xFFFu : 0x1FFu, step == 0 ? kSpBins : 512, a.p,
-                                     CS, cr, hlo, hhi, fx, sr);
+                                     CSs, crs, hist, fx, sr);
           if (step == 0) {
             have = ok;
-            if (have) done_small = resolve_small_bin(W, sr, s0 * kPage, CS, fx, &theta, &r_need);
+            if (have) done_small = resolve_small_bin(WS, sr, pos0s, CSs, fx, &theta, &r_need);
           }
           if (!have || done_small) break;   // the same in every CTA of the cluster
         }
@@ -1148,9 +1328,9 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
       // compaction in ascending position order
       unsigned n_gt = 0, n_eq = 0;
 #pragma unroll 1
-      for (int i = 0; i < R; ++i) {
-        if (lp0 + i >= npos) break;
-        const float w = W.at(i);
+      for (int i = 0; i < WS.R; ++i) {
+        if (WS.lp0 + i >= WS.npos) break;
+        const float w = WS.at(i);
         if (w < 0.f) continue;
         const uint32_t key = __float_as_uint(w);
         if (keep_all || (have && key > theta)) ++n_gt;
@@ -1159,7 +1339,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
       unsigned blk_total;
       const unsigned ex = sp_scan((n_gt << 16) | n_eq, fx.scan, &blk_total);
       unsigned gt_before = 0, eq_before = 0, gt_all = blk_total >> 16, eq_all = blk_total & 0xFFFFu;
-      if (CS > 1) {
+      if (CSs > 1) {
         if (tid == 0) {
           fx.blk[0] = blk_total >> 16;
           fx.blk[1] = blk_total & 0xFFFFu;
@@ -1202,13 +1382,13 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
           (r_need > eq_before ? (unsigned)min((unsigned long long)eq_blk, r_need - eq_before) : 0u);
       const unsigned lpos0 = (ex >> 16) + (unsigned)min(r_need, ties_before) -
                              (unsigned)min(r_need, (unsigned long long)eq_before);
-      unsigned sel = 0;   // bit i: local position lp0 + i is kept (R <= 32)
+      unsigned sel = 0;   // bit i: position WS.lp0 + i is kept (R <= 32)
       {
         unsigned taken = 0;
 #pragma unroll 1
-        for (int i = 0; i < R; ++i) {
-          if (lp0 + i >= npos) break;
-          const float w = W.at(i);
+        for (int i = 0; i < WS.R; ++i) {
+          if (WS.lp0 + i >= WS.npos) break;
+          const float w = WS.at(i);
           if (w < 0.f) continue;
           const uint32_t key = __float_as_uint(w);
           bool keep = keep_all || (have && key > theta);
@@ -1219,7 +1399,27 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
           if (keep) sel |= 1u << i;
         }
       }
-      for (int pass = 0; pass < (a.rows ? 2 : 1); ++pass) {
+      if (local) {
+        // the kept positions of this CTA's share, straight to their output
+        // slots (the whole set's order is known to every CTA)
+        int32_t* oidx = a.idx + (int64_t)set * a.icap;
+        uint32_t* orow = a.rows ? a.rows + (int64_t)set * a.icap : nullptr;
+        unsigned o = lpos0;
+        unsigned m = sel;
+#pragma unroll 1
+        while (m) {
+          const int i = __ffs(m) - 1;
+          m &= m - 1;
+          const int x = WS.lp0 + i - s0 * kPage;   // position within this CTA's share
+          if (x >= 0 && x < npos) {
+            const int e = x >> 4, r = x & 15;
+            oidx[o] = (int32_t)(fx.pg[e] * kPage + (uint32_t)r);
+            if (orow) orow[o] = fx.r0[e] + (uint32_t)r;
+          }
+          ++o;
+        }
+      }
+      for (int pass = 0; pass < (local ? 0 : (a.rows ? 2 : 1)); ++pass) {
         unsigned lp = lpos0;
         unsigned m = sel;
 #pragma unroll 1
@@ -1239,7 +1439,9 @@ __global__ void __launch_bounds__(kSpThreads, 1) k_select_prune(SpArgs a) {
         a.count[set] = (int32_t)(gt_all + (unsigned)min(r_need, (unsigned long long)eq_all));
         if (a.done) a.done[set] = 0;   // the attention kernel's per-set completion counter
       }
-      if (CS > 1) cluster_sync();   // peers are done reading this CTA's totals
+      // peers are done reading this CTA's totals, or (gathered sets) with
+      // this CTA's copy of the set before the next set overwrites it
+      if (CS > 1 && (!local || hs + 1 < nsets_u)) cluster_sync();
     }
   }
   if (failed) {   // a wait gave up: give any copy still in flight time to land before exit
@@ -1322,10 +1524,10 @@ static size_t sp_smem_bytes(const SpShape& s, int kbits, int G, int max_pages, b
   const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * kbits / 8 + 2 * kGroups * 2);
   size_t ra = 0, rb = 0;
   if (do_select)
-    ra = (size_t)s.s1 * kMetaStageBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
+    ra = (size_t)s.s1 * s.mp1 * kMetaRecBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
   if (do_prune) {
-    rb = (size_t)s.s2 * stage2 > (size_t)2 * kSpBins * 4 ? (size_t)s.s2 * stage2
-                                                         : (size_t)2 * kSpBins * 4;
+    const size_t search = (size_t)kSpHistBytes + (s.local_pos ? (size_t)sp_pad(s.local_pos) * 4 : 0);
+    rb = (size_t)s.s2 * stage2 > search ? (size_t)s.s2 * stage2 : search;
     if (s.logits_in_smem) rb += (size_t)sp_pad(s.share_cap * kPage) * G * sizeof(float);
   }
   return (kSpFixedBytes + (ra > rb ? ra : rb) + 127) / 128 * 128;
@@ -1345,16 +1547,18 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
   while (cs_min < kSpMaxCluster && (sel_pages + cs_min - 1) / cs_min > kSpSharePages) cs_min *= 2;
   if ((sel_pages + cs_min - 1) / cs_min > kSpSharePages) return -1;
   const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * BITS / 8 + 2 * kGroups * 2);
-  auto fill = [&](int cs, size_t budget, SpShape* s) {
+  auto fill = [&](int cs, size_t budget, int mp1, SpShape* s) {
     s->cs = cs;
+    s->mp1 = mp1;
     s->share_cap = (sel_pages + cs - 1) / cs;
+    s->local_pos = (do_prune && cs > 1 && sel_pages * kPage <= kSpLocalPos) ? sel_pages * kPage : 0;
     s->keys_in_smem = max_pages <= kSpKeysCap;
     s->logits_in_smem = (size_t)sp_pad(s->share_cap * kPage) * G * 4 <= (size_t)kSpLogitsSmem;
     const size_t keys = s->keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0;
     const size_t logits = s->logits_in_smem ? (size_t)sp_pad(s->share_cap * kPage) * G * 4 : 0;
     const size_t room1 = budget > kSpFixedBytes + keys ? budget - kSpFixedBytes - keys : 0;
     const size_t room2 = budget > kSpFixedBytes + logits ? budget - kSpFixedBytes - logits : 0;
-    s->s1 = (int)(room1 / kMetaStageBytes);
+    s->s1 = (int)(room1 / ((size_t)s->mp1 * kMetaRecBytes));
     s->s2 = (int)(room2 / stage2);
     const int need2 = (s->share_cap + kEstStagePages - 1) / kEstStagePages;   // stages of a share
     s->s1 = s->s1 < 2 ? 2 : (s->s1 > kSpMaxStages ? kSpMaxStages : s->s1);
@@ -1364,16 +1568,33 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
   };
   SpShape s;
   const size_t big = 200 * 1024, two_per_sm = 110 * 1024;
+  // two CTAs per SM when the registers allow it (more warps to hide latency)
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    regs = cudaFuncGetAttributes(&fa, k_select_prune<G, BITS>) == cudaSuccess ? fa.numRegs : 255;
+  }
+  if (regs * kSpThreads * 2 <= 65536) {
+    for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
+      if ((long long)units * cs > 2LL * num_sms) continue;
+      fill(cs, two_per_sm, kMetaStagePages / 2, &s);
+      if (s.smem > kSpMaxSmem) continue;
+      if (sp_max_clusters<G, BITS>(cs, s.smem) >= units) {
+        *out = s;
+        return 0;
+      }
+    }
+  }
   for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
     if ((long long)units * cs > num_sms) continue;
-    fill(cs, big, &s);
+    fill(cs, big, kMetaStagePages, &s);
     if (s.smem > kSpMaxSmem) continue;
     if (sp_max_clusters<G, BITS>(cs, s.smem) >= units) {
       *out = s;
       return 0;
     }
   }
-  fill(cs_min, two_per_sm, &s);
+  fill(cs_min, two_per_sm, kMetaStagePages / 2, &s);
   if (s.smem > kSpMaxSmem) return -1;
   *out = s;
   return 0;
@@ -1390,7 +1611,9 @@ static cudaError_t sp_launch_t(SpArgs a, int sel_pages, int num_sms, cudaStream_
     return cudaErrorInvalidValue;
   a.s1 = sh.s1;
   a.s2 = sh.s2;
+  a.mp1 = sh.mp1;
   a.share_cap = sh.share_cap;
+  a.local_pos = sh.local_pos;
   if (sh.keys_in_smem) a.gkeys = nullptr;
   if (sh.logits_in_smem) a.glogits = nullptr;
   cudaLaunchAttribute attr[2];

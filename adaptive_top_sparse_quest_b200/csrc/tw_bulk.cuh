@@ -1,11 +1,11 @@
-// Bulk-copy (non-tensor TMA) streaming, mbarriers and thread-block-cluster
-// helpers shared by the streaming kernels.
+// Bulk-copy (non-tensor TMA) streaming, mbarriers, explicit shared-memory
+// accesses and thread-block-cluster helpers shared by the streaming kernels.
 //
-// A stage of a shared-memory ring is filled by cp.async.bulk copies that
-// complete on the stage's "full" mbarrier (one arrival that carries the
-// stage's byte count); the consumer warps release it on its "empty" mbarrier
-// (one arrival per warp).  No copy uses cluster multicast: every source is
-// this GPU's own global memory.
+// A stage of a shared-memory ring is filled either by one cp.async.bulk copy
+// that completes on the stage's "full" mbarrier together with the stage's
+// byte count, or by cp.async copies from every thread, each thread arriving on
+// the barrier when its copies have landed.  No copy uses cluster multicast:
+// every source is this GPU's own global memory.
 //
 // Every mbarrier wait is bounded: a wait that has not seen its phase complete
 // after kWaitNs of polling sets kDevErrWait in the caller's status word and
@@ -92,6 +92,33 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           "r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// --------------------------------------------------------------------------
+// Explicit shared-memory accesses (addresses from smem_u32), for code paths
+// where a pointer's state space would otherwise be generic.
+
+__device__ __forceinline__ void sm_red_add_u64(uint32_t addr, unsigned long long v) {
+  asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ void sm_red_add_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long sm_ld_u64(uint32_t addr) {
+  unsigned long long v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sm_st_u64(uint32_t addr, unsigned long long v) {
+  asm volatile("st.shared.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t sm_ld_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sm_st_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // --------------------------------------------------------------------------
