@@ -63,7 +63,7 @@ constexpr int kMetaRecBytes = 2 * kHeadDim * 2;          // one page's min and m
 constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
 constexpr int kEstStageTok = kEstStagePages * kPage;
 constexpr int kSpBins = 4096;                            // first digit of the searches: 12 bits
-constexpr int kSpBinList = 32;                           // a first-digit bin this small is resolved directly
+constexpr int kSpBinList = 256;                          // a first-digit bin this small is resolved directly
 constexpr float kEstL2Scale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
 constexpr double kSpMassEps = 1e-12;           // exact ties at p resolve as in real arithmetic
 constexpr float kSpMassScale = 1099511627776.0f;   // 2^40
@@ -104,6 +104,7 @@ struct SpFixed {
   int2 scan2[kSpWarps + 1];
   unsigned scan[kSpWarps + 1];
   uint32_t wmin[kSpWarps], wmax[kSpWarps];
+  uint32_t kmin[kSpMaxCluster * kSpWarps], kmax[kSpMaxCluster * kSpWarps];   // per CTA and warp
   unsigned blk[2];
   unsigned pre[4];
   uint32_t lst_key[kSpBinList];   // the weights of the threshold's first-digit bin
@@ -147,6 +148,13 @@ __host__ __device__ __forceinline__ int sp_pad(int i) { return i + (i >> 5); }
 constexpr int kSpHistWords = kSpBins + kSpBins / 32;
 constexpr int kSpHistBytes = kSpHistWords * 8;   // a digit histogram of 64-bit words
 constexpr int kSpLoBits = 19;
+// First digit of the top-p search: bits 29..18 of the weight's fp32 pattern.
+// A weight of nonzero mass is at least 2^-40, so its digit is at least
+// 87 * 32; the histogram covers digits [2048, 4096) only.
+constexpr int kSpShift0 = 18;
+constexpr int kTopkDigitBits = 10;   // digit width of the page top-k rounds
+constexpr int kSpDigit0Base = 2048;
+constexpr int kSpBins0 = kSpBins - kSpDigit0Base;
 constexpr int kPtAhead = 6;   // iterations between a page-table load and its store (< kSpWarps)   // low bits of a mass in a bin word's low half
 
 __device__ __forceinline__ float sp_h(uint32_t w, int hi) {
@@ -308,34 +316,15 @@ __device__ __forceinline__ float page_scores(const ScoreQ<G>& Q, const unsigned 
 // Radix select of the K largest of P keys (ties to the lower index), by the
 // whole CTA: returns through fx the threshold key and the number of keys
 // equal to it that are kept (the lowest-index ones).  Thread t owns the E
-// consecutive keys [t E, t E + E).  hist: kSpBins ints, zero on entry and exit.
+// consecutive keys [t E, t E + E); kmin / kmax: the smallest and largest of
+// the P keys.  Digits of kTopkDigitBits bits below the keys' common prefix.
+// hist: 2^kTopkDigitBits ints (padded), zero on entry and exit.
 template <typename KeyAt>
-__device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& fx) {
+__device__ void topk_threshold(KeyAt key_at, int P, int K, uint32_t kmin, uint32_t kmax, int* hist,
+                               SpFixed& fx) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = (P + kSpThreads - 1) / kSpThreads;
   const int i0 = tid * E, i1 = min(P, i0 + E);
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll 1
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t k = key_at(i);
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    fx.wmin[warp] = kmin;
-    fx.wmax[warp] = kmax;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int w = 0; w < kSpWarps; ++w) {
-    kmin = min(kmin, fx.wmin[w]);
-    kmax = max(kmax, fx.wmax[w]);
-  }
   // the keys share the bits above the highest bit where the smallest and
   // largest differ; the digits start below that common prefix
   int nb = 32 - __clz((int)(kmin ^ kmax));
@@ -344,7 +333,7 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, int* hist, SpFixed& f
   int need = K;
 #pragma unroll 1
   for (int round = 0; nb > 0; ++round) {
-    const int width = min(round == 0 ? 12 : 10, nb);
+    const int width = min(kTopkDigitBits, nb);
     const int shift = nb - width;
     const uint32_t dm = (1u << width) - 1u;
     nb = shift;
@@ -430,11 +419,20 @@ __device__ __forceinline__ void sp_mma16816(float (&d)[4], const uint32_t (&a)[4
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Nibbles e and e+4 of W as the half2 (c_e - 8, c_{e+4} - 8), exact.
+// Nibbles e and e+4 of W as the half2 (c_e - 8, c_{e+4} - 8), exact.  A low
+// nibble of a byte is masked into the mantissa of 1024 (giving 1024 + c, then
+// minus 1032); a high nibble is masked in place (1024 + 16 c, then times 1/16
+// minus 72), so bytes 2 and 3 need one shift of W by 8 and no other shifts.
 __device__ __forceinline__ uint32_t sp_nib_pair(uint32_t W, int e) {
-  uint32_t x = ((W >> (4 * e)) & 0x000F000Fu) | 0x64006400u;   // (1024 + c) as fp16
+  const uint32_t src = e >= 2 ? (W >> 8) : W;
   uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64086408u));   // minus 1032
+  if ((e & 1) == 0) {
+    const uint32_t x = (src & 0x000F000Fu) | 0x64006400u;   // 1024 + c
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64086408u));   // minus 1032
+  } else {
+    const uint32_t x = (src & 0x00F000F0u) | 0x64006400u;   // 1024 + 16 c
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(0x2C002C00u), "r"(0xD480D480u));   // x / 16 - 72
+  }
   return r;
 }
 
@@ -495,8 +493,9 @@ struct SpWeights {
 // Neither half overflows: a CTA holds at most kSpSharePages * kPage weights,
 // so the low sums stay below 2^(kSpLoBits + 13), and the weights of a set sum
 // to about 1, so the high sums stay near 2^(40 - kSpLoBits).  Weights are read
-// eight at a time before their reductions.
-__device__ __forceinline__ void mass_hist(const SpWeights& W, int shift, uint32_t dm,
+// eight at a time before their reductions.  Histogram word d holds digit
+// d + dbase; every weight of nonzero mass has a digit >= dbase.
+__device__ __forceinline__ void mass_hist(const SpWeights& W, int shift, uint32_t dm, int dbase,
                                           const SpSearch& s, unsigned long long* hist) {
   const uint32_t h0 = smem_u32(hist);
 #pragma unroll 1
@@ -508,11 +507,14 @@ __device__ __forceinline__ void mass_hist(const SpWeights& W, int shift, uint32_
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t key = __float_as_uint(wv[i]);
-      if (wv[i] >= 0.f && (key & s.pmask) == s.prefix) {
-        const unsigned long long m = sp_mass(wv[i]);
-        const uint32_t a = h0 + 8u * (uint32_t)sp_pad((int)((key >> shift) & dm));
-        sm_red_add_u32(a, (uint32_t)m & ((1u << kSpLoBits) - 1u));
-        sm_red_add_u32(a + 4u, (uint32_t)(m >> kSpLoBits));
+      const unsigned long long m = wv[i] >= 0.f ? sp_mass(wv[i]) : 0ull;
+      // a weight of zero mass changes no sum (and lies below digit dbase)
+      if (m != 0ull && (key & s.pmask) == s.prefix) {
+        const int d = (int)((key >> shift) & dm) - dbase;
+        const uint32_t a = h0 + 8u * (uint32_t)sp_pad(d);
+        const uint32_t lo = (uint32_t)m & ((1u << kSpLoBits) - 1u), hi = (uint32_t)(m >> kSpLoBits);
+        if (lo) sm_red_add_u32(a, lo);
+        if (hi) sm_red_add_u32(a + 4u, hi);
       }
     }
   }
@@ -555,12 +557,12 @@ __device__ __forceinline__ void cluster_bins(unsigned long long* hist, int base,
 // CTA's own words of those digits (no peer reads them).  The mass scan runs
 // from the top digit down; the one thread whose digit holds the crossing of
 // the target writes it into every CTA.  The first step also sets the target
-// from the total mass and returns false if that is zero.  Leaves this CTA's
-// histogram zeroed.
-__device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, double p, int CS,
-                           int cr, unsigned long long* hist, SpFixed& fx, SpSearch& s) {
+// from the total mass and returns false if that is zero.  Leaves the low 512
+// digits of this CTA's histogram zeroed.
+__device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, int dbase, double p,
+                           int CS, int cr, unsigned long long* hist, SpFixed& fx, SpSearch& s) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  mass_hist(W, shift, dm, s, hist);
+  mass_hist(W, shift, dm, dbase, s, hist);
   if (CS > 1) cluster_sync();   // every CTA's histogram is complete
   else __syncthreads();
   const int SB = NB / CS;                                    // digits of this CTA's slice
@@ -610,19 +612,18 @@ __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, d
   if (CS > 1) {
     if (tid == 0) fx.slice_tot = slice;
     cluster_sync();   // slice totals published; no peer reads this CTA's histogram any more
-    unsigned long long tots[kSpMaxCluster];
+    unsigned long long t = lane < CS ? ld_peer_u64(peer_addr(&fx.slice_tot, (uint32_t)lane)) : 0ull;
+    unsigned long long th = lane > cr ? t : 0ull;
 #pragma unroll
-    for (int r = 0; r < kSpMaxCluster; ++r)
-      tots[r] = r < CS ? ld_peer_u64(peer_addr(&fx.slice_tot, r)) : 0ull;
-    total = 0;
-#pragma unroll
-    for (int r = 0; r < kSpMaxCluster; ++r) {
-      total += tots[r];
-      if (r > cr) higher += tots[r];
+    for (int o = 16; o > 0; o >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, o);
+      th += __shfl_xor_sync(0xffffffffu, th, o);
     }
+    total = t;
+    higher = th;
   }
   bool ok = true;
-  if (NB == kSpBins) {
+  if (shift == kSpShift0) {
     if (total == 0) {
       ok = false;
     } else {
@@ -653,12 +654,14 @@ __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, d
     }
   }
   __syncthreads();   // every thread is done with the histogram words it holds
-  for (int i = tid; i < sp_pad(NB); i += kSpThreads) sm_st_u64(smem_u32(&hist[i]), 0ull);
+  // the later digits (512 bins) need only the low words zeroed; the next set
+  // zeroes the whole histogram
+  for (int i = tid; i < sp_pad(512); i += kSpThreads) sm_st_u64(smem_u32(&hist[i]), 0ull);
   if (CS > 1) cluster_sync();   // the digit is in every CTA's shared memory
   else __syncthreads();
   if (ok) {
     s.A += fx.sh_above;
-    s.prefix |= (uint32_t)fx.sh_d << shift;
+    s.prefix |= (uint32_t)(fx.sh_d + dbase) << shift;
     s.pmask |= dm << shift;
   }
   __syncthreads();   // sh_d / sh_above / wsuf are rewritten by the next step
@@ -673,9 +676,12 @@ __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, d
 // r_need the number of weights equal to it up to and including it (the same
 // theta and tie count as the remaining digit steps would give).  Returns
 // false (the same in every CTA) when the digit holds more weights.  pos0:
-// this CTA's first set position.
+// this CTA's first set position.  scratch: the (zeroed) digit histogram,
+// used as work space only when the digit is resolved here; the next set
+// zeroes it again.
 __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos0, int CS,
-                                  SpFixed& fx, uint32_t* theta, unsigned long long* r_need) {
+                                  SpFixed& fx, unsigned long long* scratch, uint32_t* theta,
+                                  unsigned long long* r_need) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) fx.lst_n = 0;
   __syncthreads();
@@ -695,10 +701,10 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
   }
   if (CS > 1) cluster_sync();   // every CTA's list is complete
   else __syncthreads();
-  // every CTA's count (lanes r < CS), and the gathered list in warp 0
+  // every CTA's count (lanes r < CS, in every warp) and their inclusive prefix
   int cnt = 0;
   if (lane < CS) cnt = CS == 1 ? fx.lst_n : (int)ld_peer_u32(peer_addr(&fx.lst_n, (uint32_t)lane));
-  int before = cnt;   // inclusive prefix over the CTAs
+  int before = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int t = __shfl_up_sync(0xffffffffu, before, o);
@@ -706,57 +712,66 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
   }
   const int n = __shfl_sync(0xffffffffu, before, 31);
   const bool over = __any_sync(0xffffffffu, cnt > kSpBinList);
-  const bool small = !over && n <= kSpBinList;
-  if (small && warp == 0) {
-    // lane i < n takes element i of the concatenated lists (CTA r holds
-    // elements [before_r - cnt_r, before_r))
-    uint32_t key = 0, pos = 0xFFFFFFFFu;
-    const bool mine = lane < n;
-    int src = 0, start = 0;
+  if (over || n == 0 || n > kSpBinList) return false;   // uniform over the cluster
+  // element t of the concatenated lists (CTA r holds [before_r - cnt_r, before_r))
+  uint32_t* gkey = reinterpret_cast<uint32_t*>(scratch);
+  uint32_t* gpos = gkey + kSpBinList;
+  uint32_t* skey = gpos + kSpBinList;                    // by rank
+  int* sgt = reinterpret_cast<int*>(skey + kSpBinList);  // by rank: weights above its value
+  unsigned long long* sF = reinterpret_cast<unsigned long long*>(sgt + kSpBinList);   // by rank
+  int src = 0, start = 0;
 #pragma unroll 1
-    for (int r = 0; r < CS; ++r) {
-      const int end = __shfl_sync(0xffffffffu, before, r);
-      const int c = __shfl_sync(0xffffffffu, cnt, r);
-      if (lane >= end - c && lane < end) {
-        src = r;
-        start = end - c;
-      }
+  for (int r = 0; r < CS; ++r) {   // every lane, so the shuffles are uniform
+    const int end = __shfl_sync(0xffffffffu, before, r);
+    const int c = __shfl_sync(0xffffffffu, cnt, r);
+    if (tid >= end - c && tid < end) {
+      src = r;
+      start = end - c;
     }
-    if (mine) {
-      key = CS == 1 ? fx.lst_key[lane] : ld_peer_u32(peer_addr(&fx.lst_key[lane - start], (uint32_t)src));
-      pos = CS == 1 ? fx.lst_pos[lane] : ld_peer_u32(peer_addr(&fx.lst_pos[lane - start], (uint32_t)src));
+  }
+  if (tid < n) {
+    gkey[tid] = CS == 1 ? fx.lst_key[tid] : ld_peer_u32(peer_addr(&fx.lst_key[tid - start], (uint32_t)src));
+    gpos[tid] = CS == 1 ? fx.lst_pos[tid] : ld_peer_u32(peer_addr(&fx.lst_pos[tid - start], (uint32_t)src));
+  }
+  __syncthreads();
+  // rank in the order (weight descending, position ascending); the ranks are
+  // a permutation of 0 .. n-1 (positions are distinct)
+  if (tid < n) {
+    const uint32_t key = gkey[tid], pos = gpos[tid];
+    int rank = 0, gt = 0;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+      const uint32_t kj = gkey[j];
+      gt += kj > key;
+      rank += kj > key || (kj == key && gpos[j] < pos);
     }
-    // rank in the order (weight descending, position ascending)
-    int rank = 0;
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
-      const uint32_t pj = __shfl_sync(0xffffffffu, pos, j);
-      if (j < n && mine && (kj > key || (kj == key && pj < pos))) ++rank;
-    }
-    const unsigned long long F = mine ? sp_mass(__uint_as_float(key)) : 0ull;
-    unsigned long long cum = s.A;   // mass above the digit plus every weight up to this one
-    int ties = 0;                   // weights equal to this one up to and including it
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) {
-      const int rj = __shfl_sync(0xffffffffu, rank, j);
-      const unsigned long long Fj = __shfl_sync(0xffffffffu, F, j);
-      const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
-      if (j < n && mine && rj <= rank) {
-        cum += Fj;
-        if (kj == key) ++ties;
-      }
-    }
-    const bool cut = mine && cum >= s.T && cum - F < s.T;
-    if (cut) {
-      fx.res_theta = key;
-      fx.res_need = (unsigned long long)ties;
-    }
+    skey[rank] = key;
+    sgt[rank] = gt;
+    sF[rank] = sp_mass(__uint_as_float(key));
+  }
+  __syncthreads();
+  // running mass in rank order: inclusive scan over threads 0 .. n-1
+  const unsigned long long F = tid < n ? sF[tid] : 0ull;
+  unsigned long long inc = F;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) fx.wsuf[warp] = inc;
+  __syncthreads();
+#pragma unroll
+  for (int w2 = 0; w2 < kSpWarps; ++w2)
+    if (w2 < warp) inc += fx.wsuf[w2];
+  const unsigned long long cum = s.A + inc;   // mass above the digit plus ranks 0 .. tid
+  if (tid < n && cum >= s.T && cum - F < s.T) {
+    fx.res_theta = skey[tid];
+    fx.res_need = (unsigned long long)(tid - sgt[tid] + 1);
   }
   __syncthreads();
   *theta = fx.res_theta;
   *r_need = fx.res_need;
-  return small;
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -895,6 +910,7 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
         }
       }
     }
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;   // over the keys this lane computed
     for (int j = 0; j < nst; ++j) {
       // refill: stage j + S - 1 into the slot stage j - 1 used (freed by the
       // barrier that ended the previous iteration); then the page-table
@@ -916,6 +932,8 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       const int i = hw + 16 * kp;
       if (i < n) {
         const uint32_t key = f_key(score);
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
         const int pg = pA + j * mp + i;
         if (gk) {
           if (rr == 0) gkeys[pg] = key;
@@ -931,7 +949,33 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       }
       __syncthreads();   // slot j is free; the staged entries are visible
     }
+    // every warp's smallest and largest key, into every CTA
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane < CS) {
+      st_peer_u32(peer_addr(&fx.kmin[cr * kSpWarps + warp], (uint32_t)lane), kmin);
+      st_peer_u32(peer_addr(&fx.kmax[cr * kSpWarps + warp], (uint32_t)lane), kmax);
+    }
     cluster_sync();   // every CTA holds all P keys (or they are in global memory)
+    {
+      const int nw = CS * kSpWarps;   // <= 128: four per lane
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int i = lane + 32 * x;
+        if (i < nw) {
+          kmin = min(kmin, fx.kmin[i]);
+          kmax = max(kmax, fx.kmax[i]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+      }
+    }
 
     // ---------------- top-K_p and this CTA's share of the candidate list ----------------
     const int K = min(a.budget_pages, P);
@@ -940,36 +984,59 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       return gk ? __ldcg(gkeys + i) : sm_ld_u32(skeys_s + 4u * (uint32_t)sp_pad(i));
     };
     int* hist = reinterpret_cast<int*>(ring);   // the meta ring is idle now
-    for (int i = tid; i < kSpHistWords; i += kSpThreads) hist[i] = 0;
+    for (int i = tid; i < sp_pad(1 << kTopkDigitBits); i += kSpThreads) hist[i] = 0;
     __syncthreads();
     const bool all = K >= P;
-    if (!all) topk_threshold(key_at, P, K, hist, fx);
+    if (!all) topk_threshold(key_at, P, K, kmin, kmax, hist, fx);
     const uint32_t thr = all ? 0u : fx.sh_pref;
     const int need = all ? 0 : fx.sh_need;
     const int E = (P + kSpThreads - 1) / kSpThreads;
     const int i0 = tid * E, i1 = min(P, i0 + E);
-    int n_gt = 0, n_eq = 0;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = all ? 1u : key_at(i);
-      if (all || k > thr) ++n_gt;
-      else if (k == thr) ++n_eq;
+    // bit i - c of the masks: key i of the chunk [c, c + 32) above / at the
+    // threshold; the first chunk's masks are kept for the second pass (a
+    // thread has one chunk unless P > 8192)
+    auto chunk_masks = [&](int c, uint32_t& gtm, uint32_t& eqm) {
+      gtm = eqm = 0u;
+      const int ce = min(i1, c + 32);
+#pragma unroll 1
+      for (int i = c; i < ce; ++i) {
+        const uint32_t k = all ? 1u : key_at(i);
+        if (all || k > thr) gtm |= 1u << (i - c);
+        else if (k == thr) eqm |= 1u << (i - c);
+      }
+    };
+    uint32_t gtm0, eqm0;
+    chunk_masks(i0, gtm0, eqm0);
+    int n_gt = __popc(gtm0), n_eq = __popc(eqm0);
+#pragma unroll 1
+    for (int c = i0 + 32; c < i1; c += 32) {
+      uint32_t g, e;
+      chunk_masks(c, g, e);
+      n_gt += __popc(g);
+      n_eq += __popc(e);
     }
     int2 tot;
     const int2 ex = sp_scan2(make_int2(n_gt, n_eq), fx.scan2, &tot);
     nsel = K;
     s0 = (int)((int64_t)cr * K / CS);
     ns = (int)((int64_t)(cr + 1) * K / CS) - s0;
+    // the kept keys: all above, and the lowest-index ones at the threshold
     int take = ex.y < need ? min(n_eq, need - ex.y) : 0;
     int pos = ex.x + min(need, ex.y);
     int32_t* cand_u = a.cand + (int64_t)u * a.cand_stride;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = all ? 1u : key_at(i);
-      bool sel = all || k > thr;
-      if (!sel && k == thr && take > 0) {
-        sel = true;
-        --take;
+#pragma unroll 1
+    for (int c = i0; c < i1; c += 32) {
+      uint32_t sel = gtm0, m = eqm0;
+      if (c != i0) chunk_masks(c, sel, m);
+#pragma unroll 1
+      for (; take > 0 && m; --take) {
+        sel |= m & (0u - m);
+        m &= m - 1;
       }
-      if (sel) {
+#pragma unroll 1
+      while (sel) {
+        const int i = c + __ffs(sel) - 1;
+        sel &= sel - 1;
         if (pos >= s0 && pos < s0 + ns) {
           fx.pg[pos - s0] = (uint32_t)i;
           cand_u[pos] = i;
@@ -1007,7 +1074,7 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     // ---------------- phase 2: weight estimate of the share ----------------
     const int nst = (ns + kEstStagePages - 1) / kEstStagePages;
     unsigned char* ring = region;
-    const int ring_bytes = max(a.s2 * KW::kStageBytes, kSpHistBytes + (a.local_pos ? sp_pad(a.local_pos) * 4 : 0));
+    const int ring_bytes = max(a.s2 * KW::kStageBytes, kSpHistBytes);
     // logits [head][local position]: in shared memory (positions padded one
     // word per 32, so a thread's run of R consecutive positions is free of
     // bank conflicts) or at the set's positions [s0 * 16, ..) of the global
@@ -1247,9 +1314,8 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     }
 
     // ---------------- top-p per selection set ----------------
-    // the estimate ring is idle now: the digit histogram, then the staged output
+    // the estimate ring is idle now: the digit histogram (and the small-bin work space)
     unsigned long long* hist = reinterpret_cast<unsigned long long*>(ring);
-    uint32_t* obuf = reinterpret_cast<uint32_t*>(ring);
     const int npos = ns * kPage;                                  // local positions of the share
     const int R = (npos + kSpThreads - 1) / kSpThreads;   // <= 32 (host-checked)
     const int lp0 = tid * R;
@@ -1277,28 +1343,6 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
         }
         lbase[lidx(h0, lp)] = ok ? acc : -1.0f;
       }
-      // A set of at most local_pos positions is gathered whole into every
-      // CTA of the cluster (after the histogram words of the ring), and each
-      // CTA searches and compacts it alone: one cluster barrier instead of
-      // several per digit.  Each CTA then writes the outputs of its own share.
-      const bool local = CS > 1 && nsel * kPage <= a.local_pos;
-      SpWeights WS = W;
-      int CSs = CS, crs = cr, pos0s = s0 * kPage;
-      if (local) {
-        float* wall = reinterpret_cast<float*>(ring + kSpHistBytes);
-        __syncthreads();   // this CTA's weights are complete
-        for (int i = tid; i < npos; i += kSpThreads) {
-          const uint32_t w = __float_as_uint(lbase[lidx(h0, i)]);
-          const float* dst = wall + sp_pad(s0 * kPage + i);
-          for (int r = 0; r < CS; ++r) st_peer_u32(peer_addr(dst, (uint32_t)r), w);
-        }
-        cluster_sync();   // every CTA holds the whole set
-        const int npa = nsel * kPage, Ra = (npa + kSpThreads - 1) / kSpThreads;
-        WS = SpWeights{wall, true, smem_u32(wall), tid * Ra, Ra, npa};
-        CSs = 1;
-        crs = 0;
-        pos0s = 0;
-      }
       const bool keep_all = a.p >= 1.0;
       uint32_t theta = 0;
       unsigned long long r_need = 0;
@@ -1309,12 +1353,12 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
         bool done_small = false;
 #pragma unroll 1
         for (int step = 0; step < 3; ++step) {
-          const bool ok = digit_step(WS, step == 0 ? 18 : (step == 1 ? 9 : 0),
-                                     step == 0 ? 0xFFFu : 0x1FFu, step == 0 ? kSpBins : 512, a.p,
-                                     CSs, crs, hist, fx, sr);
+          const bool ok = digit_step(W, step == 0 ? kSpShift0 : (step == 1 ? 9 : 0),
+                                     step == 0 ? 0xFFFu : 0x1FFu, step == 0 ? kSpBins0 : 512,
+                                     step == 0 ? kSpDigit0Base : 0, a.p, CS, cr, hist, fx, sr);
           if (step == 0) {
             have = ok;
-            if (have) done_small = resolve_small_bin(WS, sr, pos0s, CSs, fx, &theta, &r_need);
+            if (have) done_small = resolve_small_bin(W, sr, s0 * kPage, CS, fx, hist, &theta, &r_need);
           }
           if (!have || done_small) break;   // the same in every CTA of the cluster
         }
@@ -1325,21 +1369,23 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
           r_need = (sr.T - sr.A + Ft - 1) / Ft;
         }
       }
-      // compaction in ascending position order
-      unsigned n_gt = 0, n_eq = 0;
+      // compaction in ascending position order: bit i of gtm / eqm marks
+      // local position lp0 + i above / at theta
+      unsigned gtm = 0, eqm = 0;
 #pragma unroll 1
-      for (int i = 0; i < WS.R; ++i) {
-        if (WS.lp0 + i >= WS.npos) break;
-        const float w = WS.at(i);
+      for (int i = 0; i < R; ++i) {
+        if (lp0 + i >= npos) break;
+        const float w = W.at(i);
         if (w < 0.f) continue;
         const uint32_t key = __float_as_uint(w);
-        if (keep_all || (have && key > theta)) ++n_gt;
-        else if (have && key == theta) ++n_eq;
+        if (keep_all || (have && key > theta)) gtm |= 1u << i;
+        else if (have && key == theta) eqm |= 1u << i;
       }
+      const unsigned n_gt = __popc(gtm), n_eq = __popc(eqm);
       unsigned blk_total;
       const unsigned ex = sp_scan((n_gt << 16) | n_eq, fx.scan, &blk_total);
       unsigned gt_before = 0, eq_before = 0, gt_all = blk_total >> 16, eq_all = blk_total & 0xFFFFu;
-      if (CSs > 1) {
+      if (CS > 1) {
         if (tid == 0) {
           fx.blk[0] = blk_total >> 16;
           fx.blk[1] = blk_total & 0xFFFFu;
@@ -1376,72 +1422,36 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       unsigned take = 0;
       if (ties_before < r_need) take = (unsigned)min((unsigned long long)n_eq, r_need - ties_before);
       const unsigned first = gt_before + (unsigned)min(r_need, (unsigned long long)eq_before);
-      const unsigned eq_blk = blk_total & 0xFFFFu;
-      const unsigned n_out =
-          (blk_total >> 16) +
-          (r_need > eq_before ? (unsigned)min((unsigned long long)eq_blk, r_need - eq_before) : 0u);
       const unsigned lpos0 = (ex >> 16) + (unsigned)min(r_need, ties_before) -
                              (unsigned)min(r_need, (unsigned long long)eq_before);
-      unsigned sel = 0;   // bit i: position WS.lp0 + i is kept (R <= 32)
+      unsigned sel = gtm;   // and the `take` lowest positions at theta
       {
-        unsigned taken = 0;
+        unsigned m = eqm;
 #pragma unroll 1
-        for (int i = 0; i < WS.R; ++i) {
-          if (WS.lp0 + i >= WS.npos) break;
-          const float w = WS.at(i);
-          if (w < 0.f) continue;
-          const uint32_t key = __float_as_uint(w);
-          bool keep = keep_all || (have && key > theta);
-          if (!keep && have && key == theta && taken < take) {
-            keep = true;
-            ++taken;
-          }
-          if (keep) sel |= 1u << i;
-        }
-      }
-      if (local) {
-        // the kept positions of this CTA's share, straight to their output
-        // slots (the whole set's order is known to every CTA)
-        int32_t* oidx = a.idx + (int64_t)set * a.icap;
-        uint32_t* orow = a.rows ? a.rows + (int64_t)set * a.icap : nullptr;
-        unsigned o = lpos0;
-        unsigned m = sel;
-#pragma unroll 1
-        while (m) {
-          const int i = __ffs(m) - 1;
+        for (unsigned t = 0; t < take; ++t) {
+          sel |= m & (0u - m);
           m &= m - 1;
-          const int x = WS.lp0 + i - s0 * kPage;   // position within this CTA's share
-          if (x >= 0 && x < npos) {
-            const int e = x >> 4, r = x & 15;
-            oidx[o] = (int32_t)(fx.pg[e] * kPage + (uint32_t)r);
-            if (orow) orow[o] = fx.r0[e] + (uint32_t)r;
-          }
-          ++o;
         }
       }
-      for (int pass = 0; pass < (local ? 0 : (a.rows ? 2 : 1)); ++pass) {
-        unsigned lp = lpos0;
+      {
+        // the thread's kept positions are consecutive outputs
+        int32_t* oidx = a.idx + (int64_t)set * a.icap + first + lpos0;
+        uint32_t* orow = a.rows ? a.rows + (int64_t)set * a.icap + first + lpos0 : nullptr;
         unsigned m = sel;
 #pragma unroll 1
-        while (m) {
+        for (int o = 0; m; ++o) {
           const int i = __ffs(m) - 1;
           m &= m - 1;
           const int e = (lp0 + i) >> 4, r = (lp0 + i) & 15;
-          obuf[lp++] = pass == 0 ? fx.pg[e] * kPage + (uint32_t)r : fx.r0[e] + (uint32_t)r;
+          oidx[o] = (int32_t)(fx.pg[e] * kPage + (uint32_t)r);
+          if (orow) orow[o] = fx.r0[e] + (uint32_t)r;
         }
-        __syncthreads();
-        uint32_t* dst = pass == 0 ? reinterpret_cast<uint32_t*>(a.idx + (int64_t)set * a.icap + first)
-                                  : a.rows + (int64_t)set * a.icap + first;
-        for (unsigned i = tid; i < n_out; i += kSpThreads) dst[i] = obuf[i];
-        __syncthreads();   // obuf is rewritten by the next pass
       }
       if (cr == 0 && tid == 0) {
         a.count[set] = (int32_t)(gt_all + (unsigned)min(r_need, (unsigned long long)eq_all));
         if (a.done) a.done[set] = 0;   // the attention kernel's per-set completion counter
       }
-      // peers are done reading this CTA's totals, or (gathered sets) with
-      // this CTA's copy of the set before the next set overwrites it
-      if (CS > 1 && (!local || hs + 1 < nsets_u)) cluster_sync();
+      if (CS > 1) cluster_sync();   // peers are done reading this CTA's totals
     }
   }
   if (failed) {   // a wait gave up: give any copy still in flight time to land before exit
@@ -1526,8 +1536,7 @@ static size_t sp_smem_bytes(const SpShape& s, int kbits, int G, int max_pages, b
   if (do_select)
     ra = (size_t)s.s1 * s.mp1 * kMetaRecBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
   if (do_prune) {
-    const size_t search = (size_t)kSpHistBytes + (s.local_pos ? (size_t)sp_pad(s.local_pos) * 4 : 0);
-    rb = (size_t)s.s2 * stage2 > search ? (size_t)s.s2 * stage2 : search;
+    rb = (size_t)s.s2 * stage2 > (size_t)kSpHistBytes ? (size_t)s.s2 * stage2 : (size_t)kSpHistBytes;
     if (s.logits_in_smem) rb += (size_t)sp_pad(s.share_cap * kPage) * G * sizeof(float);
   }
   return (kSpFixedBytes + (ra > rb ? ra : rb) + 127) / 128 * 128;
@@ -1551,7 +1560,6 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
     s->cs = cs;
     s->mp1 = mp1;
     s->share_cap = (sel_pages + cs - 1) / cs;
-    s->local_pos = (do_prune && cs > 1 && sel_pages * kPage <= kSpLocalPos) ? sel_pages * kPage : 0;
     s->keys_in_smem = max_pages <= kSpKeysCap;
     s->logits_in_smem = (size_t)sp_pad(s->share_cap * kPage) * G * 4 <= (size_t)kSpLogitsSmem;
     const size_t keys = s->keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0;
@@ -1613,7 +1621,6 @@ static cudaError_t sp_launch_t(SpArgs a, int sel_pages, int num_sms, cudaStream_
   a.s2 = sh.s2;
   a.mp1 = sh.mp1;
   a.share_cap = sh.share_cap;
-  a.local_pos = sh.local_pos;
   if (sh.keys_in_smem) a.gkeys = nullptr;
   if (sh.logits_in_smem) a.glogits = nullptr;
   cudaLaunchAttribute attr[2];

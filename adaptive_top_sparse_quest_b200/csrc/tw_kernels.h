@@ -70,7 +70,6 @@ constexpr int kSpMaxCluster = 16;
 constexpr int kSpKeysCap = 8192;         // pages whose score keys a CTA keeps in shared memory
 constexpr int kSpLogitsSmem = 32 * 1024; // a share's logits stay in shared memory up to this size
 constexpr int kSpMaxSmem = 227 * 1024;
-constexpr int kSpLocalPos = 8192;       // largest set gathered whole into every CTA of a cluster
 
 struct SpArgs {
   Layout L;
@@ -100,12 +99,10 @@ struct SpArgs {
   int s1, s2;               // ring stages of the two phases
   int mp1;                  // page records per score stage (32 or 64)
   int share_cap;            // candidate pages per CTA share (shared-memory logits stride / 16)
-  int local_pos;            // sets of at most this many positions are searched whole in every CTA
 };
 
 struct SpShape {
   int cs, share_cap, s1, s2, mp1;
-  int local_pos;            // 0, or the positions a set may have to be gathered into every CTA
   bool keys_in_smem, logits_in_smem;
   size_t smem;
 };

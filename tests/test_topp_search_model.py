@@ -3,9 +3,10 @@
 The kernel finds theta on the fp32 bit pattern of the weights with exact
 integer masses (each weight truncated to a multiple of 2^-40): a first 12-bit
 digit, then either two more digits (9 + 9 bits) or, when the first digit's
-bin holds at most 32 weights, a direct resolution of that bin (sort by weight
-descending and position ascending, cut where the running mass reaches the
-target).  Both must give the same theta and tie count as a brute-force sort of
+bin holds at most 256 weights, a direct resolution of that bin (each weight's
+rank in the order weight descending, position ascending, and the count of
+weights above it; a scan of the masses in rank order; the cut where the
+running mass reaches the target, its tie count = rank - count above + 1).  Both must give the same theta and tie count as a brute-force sort of
 the integer masses; the kept set is every weight above theta plus the r_need
 lowest-position weights equal to it."""
 import math
@@ -15,7 +16,7 @@ import pytest
 
 SCALE = float(2 ** 40)
 EPS = 1e-12
-BIN_LIST = 32
+BIN_LIST = 256
 
 
 def masses(w32):
@@ -49,15 +50,23 @@ def digit_search(keys, F, T, first_only=False):
 
 def small_bin(keys, F, T, prefix, pmask, A):
     idx = np.nonzero((keys & pmask) == prefix)[0]
-    if len(idx) > BIN_LIST:
+    if len(idx) == 0 or len(idx) > BIN_LIST:
         return None
-    order = sorted(idx, key=lambda i: (-int(keys[i]), i))
+    n = len(idx)
+    k = [int(keys[i]) for i in idx]
+    pos = [int(i) for i in idx]
+    rank = [sum(1 for j in range(n) if k[j] > k[t] or (k[j] == k[t] and pos[j] < pos[t]))
+            for t in range(n)]
+    gt = [sum(1 for j in range(n) if k[j] > k[t]) for t in range(n)]
+    assert sorted(rank) == list(range(n))
+    skey, sgt, sF = [0] * n, [0] * n, [0] * n
+    for t in range(n):
+        skey[rank[t]], sgt[rank[t]], sF[rank[t]] = k[t], gt[t], int(F[idx[t]])
     cum = A
-    for j, i in enumerate(order):
-        cum += int(F[i])
-        if cum >= T and cum - int(F[i]) < T:
-            ties = sum(1 for i2 in order[:j + 1] if keys[i2] == keys[i])
-            return int(keys[i]), ties
+    for r in range(n):
+        cum += sF[r]
+        if cum >= T and cum - sF[r] < T:
+            return skey[r], r - sgt[r] + 1
     raise AssertionError("no cut")
 
 
@@ -133,3 +142,27 @@ def test_small_bin_path_is_taken_on_spread_weights():
     T = target(int(F.sum()), 0.85)
     prefix1, pmask1, A1 = digit_search(keys, F, T, first_only=True)
     assert small_bin(keys, F, T, prefix1, pmask1, A1) is not None
+
+
+def test_small_bin_path_is_taken_on_unit_variance_logits():
+    """8192 candidates with logits of unit spread (the Llama-shaped workloads)
+    put about 70 weights in the threshold's first-digit bin: more than a warp,
+    within the 256 the CTA-wide resolution takes."""
+    rng = np.random.default_rng(5)
+    taken = 0
+    for trial in range(8):
+        l = rng.standard_normal(8192)
+        w = np.exp(l - l.max())
+        w32 = (w / w.sum()).astype(np.float32)
+        keys = w32.view(np.uint32).astype(np.int64)
+        F = masses(w32)
+        T = target(int(F.sum()), 0.85)
+        prefix1, pmask1, A1 = digit_search(keys, F, T, first_only=True)
+        in_bin = int(((keys & pmask1) == prefix1).sum())
+        res = small_bin(keys, F, T, prefix1, pmask1, A1)
+        if res is not None:
+            taken += 1
+            theta_b, ties_b, sel_b = brute(keys, F, T)
+            assert res == (theta_b, ties_b)
+        assert in_bin > 32
+    assert taken == 8
