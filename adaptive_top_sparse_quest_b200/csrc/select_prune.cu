@@ -63,7 +63,7 @@ constexpr int kMetaRecBytes = 2 * kHeadDim * 2;          // one page's min and m
 constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
 constexpr int kEstStageTok = kEstStagePages * kPage;
 constexpr int kSpBins = 4096;                            // first digit of the searches: 12 bits
-constexpr int kSpBinList = 256;                          // a first-digit bin this small is resolved directly
+constexpr int kSpBinList = 1024;                         // a first-digit bin this small is resolved in every CTA
 constexpr float kEstL2Scale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e)/sqrt(128)
 constexpr double kSpMassEps = 1e-12;           // exact ties at p resolve as in real arithmetic
 constexpr float kSpMassScale = 1099511627776.0f;   // 2^40
@@ -107,11 +107,7 @@ struct SpFixed {
   uint32_t kmin[kSpMaxCluster * kSpWarps], kmax[kSpMaxCluster * kSpWarps];   // per CTA and warp
   unsigned blk[2];
   unsigned pre[4];
-  uint32_t lst_key[kSpBinList];   // the weights of the threshold's first-digit bin
-  uint32_t lst_pos[kSpBinList];   // and their positions in the set
   int lst_n;
-  uint32_t res_theta;
-  unsigned long long res_need;
 };
 
 constexpr size_t kSpFixedBytes = (sizeof(SpFixed) + 127) / 128 * 128;
@@ -147,6 +143,7 @@ __host__ __device__ __forceinline__ int sp_pad(int i) { return i + (i >> 5); }
 // are consecutive, so their padded words are conflict-free across a warp).
 constexpr int kSpHistWords = kSpBins + kSpBins / 32;
 constexpr int kSpHistBytes = kSpHistWords * 8;   // a digit histogram of 64-bit words
+constexpr int kSpListWord = 1024;   // 64-bit word of the histogram storage where the bin lists start
 constexpr int kSpLoBits = 19;
 // First digit of the top-p search: bits 29..18 of the weight's fp32 pattern.
 // A weight of nonzero mass is at least 2^-40, so its digit is at least
@@ -668,21 +665,19 @@ __device__ bool digit_step(const SpWeights& W, int shift, uint32_t dm, int NB, i
   return ok;
 }
 
-// After the first digit: when the weights inside the threshold's digit (over
-// the whole cluster) number at most kSpBinList, gather them into every CTA
-// and resolve the threshold directly.  Sorted by weight descending, ties by
-// ascending set position, the cut is the first weight at which the mass above
-// the digit plus the running mass reaches the target; theta is its value and
-// r_need the number of weights equal to it up to and including it (the same
-// theta and tie count as the remaining digit steps would give).  Returns
-// false (the same in every CTA) when the digit holds more weights.  pos0:
-// this CTA's first set position.  scratch: the (zeroed) digit histogram,
-// used as work space only when the digit is resolved here; the next set
-// zeroes it again.
-__device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos0, int CS,
-                                  SpFixed& fx, unsigned long long* scratch, uint32_t* theta,
-                                  unsigned long long* r_need) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// After the first digit: when the weights inside the threshold's digit number
+// at most kSpBinList over the cluster, every CTA gathers all of them and runs
+// the two remaining digits (9 + 9 bits) on that list alone, with block
+// barriers only; otherwise (false, the same in every CTA) the caller runs them
+// over the whole set, reduced across the cluster.  Both give the same digits:
+// weights outside the first digit never match the prefix.  The CTA's own list
+// and the gathered list live in the histogram's storage above the 512 words
+// the later digits use (`ring`, at least kSpHistBytes).
+__device__ bool resolve_small_bin(const SpWeights& W, SpSearch& s, int CS, double p, SpFixed& fx,
+                                  unsigned long long* hist) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t* own = reinterpret_cast<uint32_t*>(hist + kSpListWord);   // this CTA's list
+  uint32_t* all = own + kSpBinList;                                  // the gathered list
   if (tid == 0) fx.lst_n = 0;
   __syncthreads();
 #pragma unroll 1
@@ -693,10 +688,7 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
     const uint32_t key = __float_as_uint(w);
     if ((key & s.pmask) == s.prefix) {
       const int slot = atomicAdd(&fx.lst_n, 1);
-      if (slot < kSpBinList) {
-        fx.lst_key[slot] = key;
-        fx.lst_pos[slot] = (uint32_t)(pos0 + W.lp0 + i);
-      }
+      if (slot < kSpBinList) own[slot] = key;
     }
   }
   if (CS > 1) cluster_sync();   // every CTA's list is complete
@@ -713,64 +705,26 @@ __device__ bool resolve_small_bin(const SpWeights& W, const SpSearch& s, int pos
   const int n = __shfl_sync(0xffffffffu, before, 31);
   const bool over = __any_sync(0xffffffffu, cnt > kSpBinList);
   if (over || n == 0 || n > kSpBinList) return false;   // uniform over the cluster
-  // element t of the concatenated lists (CTA r holds [before_r - cnt_r, before_r))
-  uint32_t* gkey = reinterpret_cast<uint32_t*>(scratch);
-  uint32_t* gpos = gkey + kSpBinList;
-  uint32_t* skey = gpos + kSpBinList;                    // by rank
-  int* sgt = reinterpret_cast<int*>(skey + kSpBinList);  // by rank: weights above its value
-  unsigned long long* sF = reinterpret_cast<unsigned long long*>(sgt + kSpBinList);   // by rank
-  int src = 0, start = 0;
+  // element t of the concatenated lists: CTA r holds [before_r - cnt_r, before_r)
+  int ends[kSpMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kSpMaxCluster; ++r) ends[r] = __shfl_sync(0xffffffffu, before, r);
 #pragma unroll 1
-  for (int r = 0; r < CS; ++r) {   // every lane, so the shuffles are uniform
-    const int end = __shfl_sync(0xffffffffu, before, r);
-    const int c = __shfl_sync(0xffffffffu, cnt, r);
-    if (tid >= end - c && tid < end) {
-      src = r;
-      start = end - c;
-    }
-  }
-  if (tid < n) {
-    gkey[tid] = CS == 1 ? fx.lst_key[tid] : ld_peer_u32(peer_addr(&fx.lst_key[tid - start], (uint32_t)src));
-    gpos[tid] = CS == 1 ? fx.lst_pos[tid] : ld_peer_u32(peer_addr(&fx.lst_pos[tid - start], (uint32_t)src));
-  }
-  __syncthreads();
-  // rank in the order (weight descending, position ascending); the ranks are
-  // a permutation of 0 .. n-1 (positions are distinct)
-  if (tid < n) {
-    const uint32_t key = gkey[tid], pos = gpos[tid];
-    int rank = 0, gt = 0;
-#pragma unroll 4
-    for (int j = 0; j < n; ++j) {
-      const uint32_t kj = gkey[j];
-      gt += kj > key;
-      rank += kj > key || (kj == key && gpos[j] < pos);
-    }
-    skey[rank] = key;
-    sgt[rank] = gt;
-    sF[rank] = sp_mass(__uint_as_float(key));
-  }
-  __syncthreads();
-  // running mass in rank order: inclusive scan over threads 0 .. n-1
-  const unsigned long long F = tid < n ? sF[tid] : 0ull;
-  unsigned long long inc = F;
+  for (int t = tid; t < n; t += kSpThreads) {
+    int src = 0, start = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  if (lane == 31) fx.wsuf[warp] = inc;
-  __syncthreads();
-#pragma unroll
-  for (int w2 = 0; w2 < kSpWarps; ++w2)
-    if (w2 < warp) inc += fx.wsuf[w2];
-  const unsigned long long cum = s.A + inc;   // mass above the digit plus ranks 0 .. tid
-  if (tid < n && cum >= s.T && cum - F < s.T) {
-    fx.res_theta = skey[tid];
-    fx.res_need = (unsigned long long)(tid - sgt[tid] + 1);
+    for (int r = 0; r < kSpMaxCluster; ++r)
+      if (r < CS && t >= ends[r]) {
+        src = r + 1;
+        start = ends[r];
+      }
+    all[t] = CS == 1 ? own[t] : ld_peer_u32(peer_addr(&own[t - start], (uint32_t)src));
   }
   __syncthreads();
-  *theta = fx.res_theta;
-  *r_need = fx.res_need;
+  const int Rl = (n + kSpThreads - 1) / kSpThreads;
+  const SpWeights L{reinterpret_cast<float*>(all), false, 0u, tid * Rl, Rl, n};
+  digit_step(L, 9, 0x1FFu, 512, 0, p, 1, 0, hist, fx, s);
+  digit_step(L, 0, 0x1FFu, 512, 0, p, 1, 0, hist, fx, s);
   return true;
 }
 
@@ -1358,11 +1312,11 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
                                      step == 0 ? kSpDigit0Base : 0, a.p, CS, cr, hist, fx, sr);
           if (step == 0) {
             have = ok;
-            if (have) done_small = resolve_small_bin(W, sr, s0 * kPage, CS, fx, hist, &theta, &r_need);
+            if (have) done_small = resolve_small_bin(W, sr, CS, a.p, fx, hist);
           }
           if (!have || done_small) break;   // the same in every CTA of the cluster
         }
-        if (have && !done_small) {
+        if (have) {
           theta = sr.prefix;
           unsigned long long Ft = sp_mass(__uint_as_float(theta));
           if (Ft == 0) Ft = 1;

@@ -3,10 +3,8 @@
 The kernel finds theta on the fp32 bit pattern of the weights with exact
 integer masses (each weight truncated to a multiple of 2^-40): a first 12-bit
 digit, then either two more digits (9 + 9 bits) or, when the first digit's
-bin holds at most 256 weights, a direct resolution of that bin (each weight's
-rank in the order weight descending, position ascending, and the count of
-weights above it; a scan of the masses in rank order; the cut where the
-running mass reaches the target, its tie count = rank - count above + 1).  Both must give the same theta and tie count as a brute-force sort of
+bin holds at most 1024 weights over the cluster, the same two digits run on a
+gathered list of that bin's weights alone (no cluster reduction).  Both must give the same theta and tie count as a brute-force sort of
 the integer masses; the kept set is every weight above theta plus the r_need
 lowest-position weights equal to it."""
 import math
@@ -16,7 +14,7 @@ import pytest
 
 SCALE = float(2 ** 40)
 EPS = 1e-12
-BIN_LIST = 256
+BIN_LIST = 1024
 
 
 def masses(w32):
@@ -49,25 +47,27 @@ def digit_search(keys, F, T, first_only=False):
 
 
 def small_bin(keys, F, T, prefix, pmask, A):
+    """The GPU's resolution of a small first-digit bin: digits 2 and 3 over the
+    bin's weights gathered into one list (their order in the list is
+    arbitrary: the CTAs' lists are concatenated)."""
     idx = np.nonzero((keys & pmask) == prefix)[0]
     if len(idx) == 0 or len(idx) > BIN_LIST:
         return None
-    n = len(idx)
-    k = [int(keys[i]) for i in idx]
-    pos = [int(i) for i in idx]
-    rank = [sum(1 for j in range(n) if k[j] > k[t] or (k[j] == k[t] and pos[j] < pos[t]))
-            for t in range(n)]
-    gt = [sum(1 for j in range(n) if k[j] > k[t]) for t in range(n)]
-    assert sorted(rank) == list(range(n))
-    skey, sgt, sF = [0] * n, [0] * n, [0] * n
-    for t in range(n):
-        skey[rank[t]], sgt[rank[t]], sF[rank[t]] = k[t], gt[t], int(F[idx[t]])
-    cum = A
-    for r in range(n):
-        cum += sF[r]
-        if cum >= T and cum - sF[r] < T:
-            return skey[r], r - sgt[r] + 1
-    raise AssertionError("no cut")
+    perm = np.random.default_rng(len(idx)).permutation(len(idx))
+    lk, lF = keys[idx][perm], F[idx][perm]
+    for shift, dm in ((9, 0x1FF), (0, 0x1FF)):
+        sel = (lk & pmask) == prefix
+        hist = np.zeros(dm + 1, dtype=object)
+        for k, f in zip(lk[sel], lF[sel]):
+            hist[(int(k) >> shift) & dm] += int(f)
+        suffix = np.cumsum(hist[::-1])[::-1]
+        above = np.concatenate([suffix[1:], [0]])
+        d = int(np.nonzero((A + suffix >= T) & (A + above < T))[0][0])
+        A += int(above[d])
+        prefix |= d << shift
+        pmask |= dm << shift
+    Ft = max(1, int(masses(np.array([prefix], np.uint32).view(np.float32))[0]))
+    return prefix, (T - A + Ft - 1) // Ft
 
 
 def brute(keys, F, T):
