@@ -47,6 +47,7 @@ class TwStep(ctypes.Structure):
 _SIGS = {
     "tw_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "tw_last_cuda_error": (ctypes.c_int, []),
+    "tw_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "tw_version": (ctypes.c_int, []),
     "tw_quantize_keys": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_vp, c_vp, c_vp]),
     "tw_page_meta": (ctypes.c_int, [ctypes.POINTER(TwKv), c_vp, c_vp]),

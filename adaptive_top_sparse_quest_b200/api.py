@@ -192,8 +192,18 @@ def workspace_bytes(B: int, Hq: int, Hk: int, N: int, capacity: int) -> int:
 
 
 def new_workspace(B, Hq, Hk, N, capacity, device) -> torch.Tensor:
-    return torch.empty(max(workspace_bytes(B, Hq, Hk, N, capacity), 256), dtype=torch.uint8,
-                       device=device)
+    """A workspace with its device status word (the first 4 bytes) zeroed."""
+    ws = torch.empty(max(workspace_bytes(B, Hq, Hk, N, capacity), 256), dtype=torch.uint8,
+                     device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def device_status(ws: torch.Tensor) -> int:
+    """The workspace's device status word (synchronises): 0, or bit 0 set when a
+    bounded wait of the selection kernel gave up (that call's outputs are
+    invalid; the C API calls it TW_ERR_TIMEOUT)."""
+    return int(ws[:4].view(torch.int32).item())
 
 
 def budget_pages(budget_tokens: Optional[int], kv: KVCache) -> int:
@@ -438,7 +448,9 @@ def token_workspace_bytes(B, Hq, Hk, N, cand_stride, capacity, key_bits=4) -> in
 
 def _token_ws(kv, Hq, stride, capacity, device):
     n = max(token_workspace_bytes(kv.B, Hq, kv.Hk, kv.N, stride, capacity, kv.key_bits), 256)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()   # the device status word
+    return ws
 
 
 def select_tokens(q: torch.Tensor, kv: KVCache, labels: torch.Tensor, channels: torch.Tensor,
@@ -516,6 +528,7 @@ class LabelDecodeStep:
                                       kv.key_bits),
                 workspace_bytes(kv.B, Hq, kv.Hk, kv.N, self.capacity), 256)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.ws[:256].zero_()   # the device status word
         self._kvs = kv.struct()
         self._q_stage = None
 

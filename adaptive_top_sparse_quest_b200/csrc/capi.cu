@@ -389,6 +389,12 @@ int tw_last_cuda_error(void) { return g_last_cuda; }
 
 int tw_version(void) { return 101; }
 
+int tw_selftest_bounded_wait(int32_t* status, void* stream) {
+  if (!status || (reinterpret_cast<uintptr_t>(status) & 3)) return TW_ERR_INVALID_ARG;
+  const cudaError_t e = tw::launch_wait_selftest(status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TW_OK : cuda_fail(e);
+}
+
 int tw_quantize_keys(const tw_kv* kv, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
                      void* stream) {
   tw::Layout L;

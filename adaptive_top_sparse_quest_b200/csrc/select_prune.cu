@@ -85,6 +85,7 @@ struct SpKeyWidth {
 // Fixed part of the shared memory; the phase regions follow it.
 struct SpFixed {
   __align__(16) __half qs[8][kHeadDim];   // the unit's query heads
+  int seq;                                // the unit's sequence
   uint64_t full1[kSpMaxStages];
   int32_t pt1[kSpMaxStages][kMetaStagePages];   // paged: pool pages of each ring stage
   uint64_t full2[kSpMaxStages];
@@ -108,6 +109,8 @@ struct SpFixed {
   unsigned blk[2];
   unsigned pre[4];
   int lst_n;
+  uint32_t res_theta;             // small-bin resolution: theta
+  unsigned long long res_above;   // and the bin's mass above it
 };
 
 constexpr size_t kSpFixedBytes = (sizeof(SpFixed) + 127) / 128 * 128;
@@ -143,7 +146,10 @@ __host__ __device__ __forceinline__ int sp_pad(int i) { return i + (i >> 5); }
 // are consecutive, so their padded words are conflict-free across a warp).
 constexpr int kSpHistWords = kSpBins + kSpBins / 32;
 constexpr int kSpHistBytes = kSpHistWords * 8;   // a digit histogram of 64-bit words
-constexpr int kSpListWord = 1024;   // 64-bit word of the histogram storage where the bin lists start
+constexpr int kSpListWord = 1024;
+constexpr int kMetaBulkLanes = 8;  // lanes per warp issuing a paged stage's record copies
+static_assert(kMetaBulkLanes * kSpWarps >= kMetaStagePages, "a lane per record of a stage");
+constexpr int kSpSortPerLane = 4;   // a bin list of at most 32 * this is sorted by one warp   // 64-bit word of the histogram storage where the bin lists start
 constexpr int kSpLoBits = 19;
 // First digit of the top-p search: bits 29..18 of the weight's fp32 pattern.
 // A weight of nonzero mass is at least 2^-40, so its digit is at least
@@ -709,8 +715,7 @@ __device__ bool resolve_small_bin(const SpWeights& W, SpSearch& s, int CS, doubl
   int ends[kSpMaxCluster];
 #pragma unroll
   for (int r = 0; r < kSpMaxCluster; ++r) ends[r] = __shfl_sync(0xffffffffu, before, r);
-#pragma unroll 1
-  for (int t = tid; t < n; t += kSpThreads) {
+  auto fetch = [&](int t) -> uint32_t {
     int src = 0, start = 0;
 #pragma unroll
     for (int r = 0; r < kSpMaxCluster; ++r)
@@ -718,8 +723,74 @@ __device__ bool resolve_small_bin(const SpWeights& W, SpSearch& s, int CS, doubl
         src = r + 1;
         start = ends[r];
       }
-    all[t] = CS == 1 ? own[t] : ld_peer_u32(peer_addr(&own[t - start], (uint32_t)src));
+    return CS == 1 ? own[t] : ld_peer_u32(peer_addr(&own[t - start], (uint32_t)src));
+  };
+  if (n <= 32 * kSpSortPerLane) {
+    // one warp: the <= 128 weights (element lane + 32 k in v[k]) sorted
+    // descending by a bitonic network, their masses scanned in that order;
+    // theta is the weight at which the running mass reaches the target, and
+    // the mass of the list's weights above theta joins A
+    if (threadIdx.x < 32) {
+      constexpr int NK = kSpSortPerLane;
+      uint32_t v[NK];
+#pragma unroll
+      for (int k = 0; k < NK; ++k) v[k] = lane + 32 * k < n ? fetch(lane + 32 * k) : 0u;
+#pragma unroll
+      for (int size = 2; size <= 32 * NK; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          uint32_t o[NK];
+#pragma unroll
+          for (int k = 0; k < NK; ++k)
+            o[k] = stride >= 32 ? v[k ^ (stride >> 5)] : __shfl_xor_sync(0xffffffffu, v[k], stride);
+#pragma unroll
+          for (int k = 0; k < NK; ++k) {
+            const int e = lane + 32 * k;
+            const bool lower = (e & stride) == 0, desc = (e & size) == 0;
+            v[k] = (lower == desc) ? max(v[k], o[k]) : min(v[k], o[k]);
+          }
+        }
+      }
+      // element e of the sorted order is v[e / 32] of lane e % 32
+      unsigned long long F[NK], inc[NK], base = 0ull;
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        F[k] = v[k] ? sp_mass(__uint_as_float(v[k])) : 0ull;
+        inc[k] = F[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long t = __shfl_up_sync(0xffffffffu, inc[k], o);
+          if (lane >= o) inc[k] += t;
+        }
+        inc[k] += base;
+        base = __shfl_sync(0xffffffffu, inc[k], 31);
+      }
+      uint32_t cut = 0u;
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        const unsigned long long cum = s.A + inc[k];
+        if (F[k] && cum >= s.T && cum - F[k] < s.T) cut = v[k];
+      }
+      const uint32_t theta = __reduce_max_sync(0xffffffffu, cut);   // the one cut (others 0)
+      unsigned long long above = 0ull;
+#pragma unroll
+      for (int k = 0; k < NK; ++k)
+        if (v[k] > theta) above += F[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+      if (lane == 0) {
+        fx.res_theta = theta;
+        fx.res_above = above;
+      }
+    }
+    __syncthreads();
+    s.prefix = fx.res_theta;
+    s.pmask = 0xFFFFFFFFu;
+    s.A += fx.res_above;
+    return true;
   }
+#pragma unroll 1
+  for (int t = tid; t < n; t += kSpThreads) all[t] = fetch(t);
   __syncthreads();
   const int Rl = (n + kSpThreads - 1) / kSpThreads;
   const SpWeights L{reinterpret_cast<float*>(all), false, 0u, tid * Rl, Rl, n};
@@ -737,20 +808,39 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
   unsigned char* region = sp_smem + kSpFixedBytes;
   const Layout& L = a.L;
   const int CS = (int)cluster_size(), cr = (int)cluster_rank();
-  const int u = blockIdx.x / CS;
-  const int b = u / L.Hk, hk = u % L.Hk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool do_select = a.meta != nullptr, do_prune = a.codes != nullptr;
   const bool paged = L.page_table != nullptr;
   if (tid == 0) {
     for (int s = 0; s < kSpMaxStages; ++s) {
-      mbar_init(&fx.full1[s], paged ? kSpThreads : 1);   // cp.async arrivals, or the byte count
+      mbar_init(&fx.full1[s], paged ? kSpWarps * kMetaBulkLanes : 1);   // arrivals with bytes
       mbar_init(&fx.full2[s], kSpThreads);   // every thread's cp.async arrival
     }
     mbar_fence_init();
   }
   __syncthreads();
   griddep_wait();
+  // Cluster c takes KV head c % Hk of the sequence of rank c / Hk in the order
+  // longest first (ties to the lower index): when the clusters run in more
+  // than one wave, the shortest sequences make up the last.
+  const int hk = (int)((blockIdx.x / CS) % L.Hk), rb = (int)((blockIdx.x / CS) / L.Hk);
+  int b = rb;
+  if (L.B > 1 && L.seq_lens) {
+#pragma unroll 1
+    for (int j = tid; j < L.B; j += kSpThreads) {
+      const int lj = L.len(j);
+      int rank = 0;
+#pragma unroll 1
+      for (int i = 0; i < L.B; ++i) {
+        const int li = L.len(i);
+        rank += li > lj || (li == lj && i < j);
+      }
+      if (rank == rb) fx.seq = j;
+    }
+    __syncthreads();
+    b = fx.seq;
+  }
+  const int u = b * L.Hk + hk;
   for (int i = tid; i < G * kHeadDim / 8; i += kSpThreads)   // 16-byte pieces of the G query rows
     reinterpret_cast<uint4*>(&fx.qs[0][0])[i] =
         __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.Hq + hk * G) * kHeadDim) + i);
@@ -774,13 +864,12 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     uint32_t* gkeys = gk ? a.gkeys + (int64_t)u * L.max_pages : nullptr;
     const __half* meta = a.meta;
     const int64_t meta_unit = (int64_t)u * L.max_pages;   // contiguous record index of page 0
-    // Stage k (up to 32 pages of the slice) into ring slot `slot`.  A
-    // contiguous cache's records of the slice are one run: one bulk copy by
-    // thread 0 completes on the stage's full barrier with its byte count.  A
-    // paged cache's records are 512-byte pieces spread over the pool: every
-    // thread copies two 16-byte parts by cp.async (pool pages from the
-    // page-table entries staged one iteration earlier) and arrives when they
-    // have landed.
+    // Stage k (up to mp pages of the slice) into ring slot `slot`, completing
+    // on the stage's full barrier with its byte count.  A contiguous cache's
+    // records of the slice are one run: one bulk copy by thread 0.  A paged
+    // cache's records are 512-byte pieces spread over the pool: one bulk copy
+    // per record from warp 0 (pool pages from the staged page-table entries);
+    // few large requests instead of 16-byte pieces from every thread.
     // warp 0, lane i: the pool pages of pages i and i + 32 of stage k (0 past the slice)
     auto fetch_pt = [&](int k) -> int2 {
       int e[2] = {0, 0};
@@ -802,14 +891,18 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       const int n = k < nst ? min(mp, npg - k * mp) : 0;
       unsigned char* dst = ring + (size_t)slot * stage1;
       if (paged) {
-#pragma unroll
-        for (int x0 = 0; x0 < kMetaStagePages * 32; x0 += kSpThreads) {   // n <= mp pages of 32 parts
-          const int x = x0 + tid, i = x >> 5, c = x & 31;
-          if (i < n)
-            cp_async16_sm(dst + i * 512 + c * 16,
-                          meta + ((int64_t)fx.pt1[slot][i] * L.Hk + hk) * (2 * kHeadDim) + c * 8);
+        // one bulk copy per page record, spread over the warps: lane j < 8 of
+        // warp w copies page 8 w + j (mp <= 64), arriving on the stage's
+        // barrier with its bytes (0 past the stage) before issuing the copy
+        const int i = warp * 8 + lane;
+        if (lane < kMetaBulkLanes) {
+          mbar_arrive_tx(&fx.full1[slot], i < n ? 512u : 0u);
+          if (i < n) {
+            fence_proxy_async();   // the slot's earlier readers are ordered before the copy
+            bulk_g2s(dst + i * 512, meta + ((int64_t)fx.pt1[slot][i] * L.Hk + hk) * (2 * kHeadDim),
+                     512u, &fx.full1[slot]);
+          }
         }
-        cp_async_arrive_noinc(&fx.full1[slot]);
       } else if (tid == 0) {
         fence_proxy_async();   // the slot's earlier readers are ordered before the copy
         if (n > 0)
@@ -1600,5 +1693,20 @@ cudaError_t launch_select_prune(const SpArgs& a, int sel_pages, int num_sms, cud
 
 // Largest candidate pages per unit the selection stages accept.
 int select_prune_max_pages() { return kSpSharePages * kSpMaxCluster; }
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives on; the wait must give up after kWaitNs and set kDevErrWait in
+// *status, and the kernel must then return normally.
+__global__ void k_wait_selftest(int* status) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  mbar_fence_init();
+  if (mbar_wait(&bar, 0u, status)) atomicOr(status, 2);   // 2: the wait did not give up
+}
+
+cudaError_t launch_wait_selftest(int* status, cudaStream_t st) {
+  k_wait_selftest<<<1, 1, 0, st>>>(status);
+  return cudaGetLastError();
+}
 
 }  // namespace tw

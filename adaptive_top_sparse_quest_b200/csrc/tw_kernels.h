@@ -107,6 +107,8 @@ struct SpShape {
   size_t smem;
 };
 
+cudaError_t launch_wait_selftest(int* status, cudaStream_t st);
+
 // Launch the selection stages (shape chosen from the sizes and the device):
 // sel_pages = candidate pages per unit at most.  a.gkeys / a.glogits point to
 // workspace regions, used only when the keys / logits exceed shared memory.

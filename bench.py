@@ -64,11 +64,19 @@ def parse():
     ap.add_argument("--selector", default="quest", choices=["quest", "label"],
                     help="base selector: Quest pages, or token-level label channels "
                          "(synthetic Double Sparsity, 16 channels per KV head)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="batched_paged only: this many sequences instead of 16 (a smaller "
+                         "case of the same workload, for profiler captures that must stay "
+                         "small on the device)")
     return ap.parse_args()
 
 
-def make_workload(name, device):
+def make_workload(name, device, batch=0):
     import workloads as W
+    if batch > 0:
+        if name != "batched_paged":
+            raise SystemExit("--batch applies to batched_paged only")
+        return W.batched_paged(device=device, B=batch)
     return W.CONFIGS[name](device=device)
 
 
@@ -306,7 +314,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import torch
-    w = make_workload(args.config, "cpu")
+    w = make_workload(args.config, "cpu", args.batch)
     chans = None
     if args.selector == "label":
         import workloads as W
@@ -480,7 +488,7 @@ def main():
     _b.build()
     _capi.load()
 
-    w = make_workload(args.config, dev)
+    w = make_workload(args.config, dev, args.batch)
     kv0 = KVCache.from_workload(w, args.key_bits)
     keys0 = quantize_keys(kv0)
     meta0 = page_meta(kv0)

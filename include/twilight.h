@@ -20,6 +20,11 @@
  *   - All data pointers are DEVICE pointers owned by the caller, 16-byte
  *     aligned.  The library allocates no memory; scratch comes from a caller
  *     workspace sized by tw_workspace_size().
+ *   - The first 4 bytes of a workspace are a device status word.  Zero it
+ *     once after allocating; the kernels only set bits in it.  Bit 0: a
+ *     bounded wait of the selection kernel (0.2 s on one pipeline stage) gave
+ *     up, and that call's outputs are invalid; a caller that reads the word
+ *     after synchronising reports it as TW_ERR_TIMEOUT.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     only enqueue work and return; they never synchronise and never read
  *     device results on the host.
@@ -70,7 +75,7 @@ typedef enum tw_status {
                                candidates per set > 131072, device not sm_100 */
   TW_ERR_CAPACITY = 3,      /* an output or workspace buffer is too small */
   TW_ERR_CUDA = 4,          /* a CUDA call failed; see tw_last_cuda_error() */
-  TW_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up */
+  TW_ERR_TIMEOUT = 5        /* a bounded device wait gave up (workspace status word) */
 } tw_status;
 
 /* KV-cache descriptor (see "Layouts" above).  Used by every call. */
@@ -97,6 +102,16 @@ const char* tw_status_string(int status);
 
 /* The cudaError_t of the last TW_ERR_CUDA returned on this host thread. */
 int tw_last_cuda_error(void);
+
+/*
+ * Diagnostic: runs one device wait that nothing completes, bounded as the
+ * selection kernel's ring waits are (0.2 s).  The wait gives up, sets bit 0
+ * of *status (a device int32 the caller zeroed) and the kernel returns
+ * normally; bit 1 would mean the wait did not give up.  The CUDA context stays
+ * usable.  Enqueues on `stream` and returns; read *status after
+ * synchronising.
+ */
+int tw_selftest_bounded_wait(int32_t* status, void* stream);
 
 /* Library ABI version (major * 100 + minor). */
 int tw_version(void);

@@ -145,3 +145,8 @@ def test_product_package_does_not_import_oracle():
             if f.endswith(".py"):
                 src = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), f
+
+
+def test_bounded_wait_selftest_argument_checks(lib):
+    assert lib.tw_selftest_bounded_wait(None, None) == _capi.TW_ERR_INVALID_ARG
+    assert lib.tw_selftest_bounded_wait(ctypes.c_void_p(2), None) == _capi.TW_ERR_INVALID_ARG

@@ -4,7 +4,9 @@ The kernel finds theta on the fp32 bit pattern of the weights with exact
 integer masses (each weight truncated to a multiple of 2^-40): a first 12-bit
 digit, then either two more digits (9 + 9 bits) or, when the first digit's
 bin holds at most 1024 weights over the cluster, the same two digits run on a
-gathered list of that bin's weights alone (no cluster reduction).  Both must give the same theta and tie count as a brute-force sort of
+gathered list of that bin's weights alone (no cluster reduction); a list of at
+most 128 is sorted by one warp instead and cut where the running mass reaches
+the target.  Both must give the same theta and tie count as a brute-force sort of
 the integer masses; the kept set is every weight above theta plus the r_need
 lowest-position weights equal to it."""
 import math
@@ -53,6 +55,20 @@ def small_bin(keys, F, T, prefix, pmask, A):
     idx = np.nonzero((keys & pmask) == prefix)[0]
     if len(idx) == 0 or len(idx) > BIN_LIST:
         return None
+    if len(idx) <= 128:
+        # one warp sorts the list descending and cuts where the running mass
+        # reaches the target; the list's mass above theta joins A
+        order = sorted((int(keys[i]) for i in idx), reverse=True)
+        cum = A
+        for k in order:
+            f = int(masses(np.array([k], np.uint32).view(np.float32))[0])
+            cum += f
+            if cum >= T and cum - f < T:
+                theta = k
+                break
+        A += sum(int(F[i]) for i in idx if int(keys[i]) > theta)
+        Ft = max(1, int(masses(np.array([theta], np.uint32).view(np.float32))[0]))
+        return theta, (T - A + Ft - 1) // Ft
     perm = np.random.default_rng(len(idx)).permutation(len(idx))
     lk, lF = keys[idx][perm], F[idx][perm]
     for shift, dm in ((9, 0x1FF), (0, 0x1FF)):
