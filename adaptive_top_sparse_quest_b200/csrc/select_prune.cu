@@ -57,8 +57,7 @@
 namespace tw {
 
 constexpr int kSpWarps = kSpThreads / 32;
-constexpr int kMetaStagePages = 64;     // page records per score stage at most (32 KB); a launch
-                                        // uses 64, or 32 when two CTAs share an SM
+constexpr int kMetaStagePages = 64;     // page records per score stage (32 KB): four per half-warp
 constexpr int kMetaRecBytes = 2 * kHeadDim * 2;          // one page's min and max rows
 constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
 constexpr int kEstStageTok = kEstStagePages * kPage;
@@ -855,7 +854,7 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     // ---------------- phase 1: page scores of pages [pA, pB) ----------------
     const int pA = (int)((int64_t)cr * P / CS), pB = (int)((int64_t)(cr + 1) * P / CS);
     const int npg = pB - pA;
-    const int mp = a.mp1;                       // pages per stage (32 or 64)
+    constexpr int mp = kMetaStagePages;         // page records per stage
     const int nst = (npg + mp - 1) / mp;
     unsigned char* ring = region;
     const size_t stage1 = (size_t)mp * kMetaRecBytes;
@@ -870,22 +869,23 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     // cache's records are 512-byte pieces spread over the pool: one bulk copy
     // per record from warp 0 (pool pages from the staged page-table entries);
     // few large requests instead of 16-byte pieces from every thread.
-    // warp 0, lane i: the pool pages of pages i and i + 32 of stage k (0 past the slice)
+    // lane i of a warp: the page-table entries of pages i and i + 32 of stage
+    // k (0 past the slice), as loaded; nothing uses them until store_pt, so
+    // the load's latency is not waited for here
     auto fetch_pt = [&](int k) -> int2 {
       int e[2] = {0, 0};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int pg = pA + k * mp + lane + 32 * h;
-        if (paged && k < nst && lane + 32 * h < mp && pg < pB) {
-          const int v = L.page_table[(int64_t)b * L.max_pages + pg];
-          e[h] = (unsigned)v < (unsigned)L.pool_pages ? v : 0;
-        }
+        if (paged && k < nst && lane + 32 * h < mp && pg < pB)
+          e[h] = L.page_table[(int64_t)b * L.max_pages + pg];
       }
       return make_int2(e[0], e[1]);
     };
+    // pool pages of the stage into the slot (an id outside the pool reads pool page 0)
     auto store_pt = [&](int slot, int2 e) {
-      fx.pt1[slot][lane] = e.x;
-      fx.pt1[slot][lane + 32] = e.y;
+      fx.pt1[slot][lane] = (unsigned)e.x < (unsigned)L.pool_pages ? e.x : 0;
+      fx.pt1[slot][lane + 32] = (unsigned)e.y < (unsigned)L.pool_pages ? e.y : 0;
     };
     auto issue1 = [&](int k, int slot) {
       const int n = k < nst ? min(mp, npg - k * mp) : 0;
@@ -969,24 +969,30 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       const int n = min(mp, npg - j * mp);
       const unsigned char* st = ring + (size_t)slot * stage1;
       // every page of the stage is scored (records past n are stale and
-      // their scores unused); lane l16 then holds page hw + 16 kp, shared
-      // with the other lanes of its group of 16 / np, which split the stores
-      const bool four = mp == 4 * 16;
-      const float score = four ? page_scores<G, 4>(Q, st, hw, l16, hmask)
-                               : page_scores<G, 2>(Q, st, hw, l16, hmask);
-      const int kp = four ? (l16 >> 2) & 3 : (l16 >> 3) & 1;
-      const int rr = four ? (l16 & 3) : (l16 & 7), step = four ? 4 : 8;
-      const int i = hw + 16 * kp;
-      if (i < n) {
-        const uint32_t key = f_key(score);
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
-        const int pg = pA + j * mp + i;
-        if (gk) {
-          if (rr == 0) gkeys[pg] = key;
-        } else {
-          for (int r = rr; r < CS; r += step) st_peer_u32(peer_addr(&skeys[sp_pad(pg)], (uint32_t)r), key);
+      // their scores unused); lane l16 then holds page hw + 16 kp (+ 32 for
+      // the second pass of G >= 4, which takes two pages per half-warp at a
+      // time to stay in registers), shared with the other lanes of its group,
+      // which split the stores
+      auto emit = [&](float score, int i, int rr, int step) {
+        if (i < n) {
+          const uint32_t key = f_key(score);
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+          const int pg = pA + j * mp + i;
+          if (gk) {
+            if (rr == 0) gkeys[pg] = key;
+          } else {
+            for (int r = rr; r < CS; r += step) st_peer_u32(peer_addr(&skeys[sp_pad(pg)], (uint32_t)r), key);
+          }
         }
+      };
+      if (G >= 4) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+          emit(page_scores<G, 2>(Q, st + half * 32 * kMetaRecBytes, hw, l16, hmask),
+               hw + 16 * ((l16 >> 3) & 1) + 32 * half, l16 & 7, 8);
+      } else {
+        emit(page_scores<G, 4>(Q, st, hw, l16, hmask), hw + 16 * ((l16 >> 2) & 3), l16 & 3, 4);
       }
       // the entries of stage j + S go where stage j's were (read when stage j
       // was issued, S - 1 iterations ago); stage j + S + kPtAhead's are loaded
@@ -1581,7 +1587,7 @@ static size_t sp_smem_bytes(const SpShape& s, int kbits, int G, int max_pages, b
   const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * kbits / 8 + 2 * kGroups * 2);
   size_t ra = 0, rb = 0;
   if (do_select)
-    ra = (size_t)s.s1 * s.mp1 * kMetaRecBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
+    ra = (size_t)s.s1 * kMetaStagePages * kMetaRecBytes + (s.keys_in_smem ? (size_t)sp_pad(max_pages) * 4 + 4 : 0);
   if (do_prune) {
     rb = (size_t)s.s2 * stage2 > (size_t)kSpHistBytes ? (size_t)s.s2 * stage2 : (size_t)kSpHistBytes;
     if (s.logits_in_smem) rb += (size_t)sp_pad(s.share_cap * kPage) * G * sizeof(float);
@@ -1603,9 +1609,8 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
   while (cs_min < kSpMaxCluster && (sel_pages + cs_min - 1) / cs_min > kSpSharePages) cs_min *= 2;
   if ((sel_pages + cs_min - 1) / cs_min > kSpSharePages) return -1;
   const size_t stage2 = (size_t)kEstStageTok * (kHeadDim * BITS / 8 + 2 * kGroups * 2);
-  auto fill = [&](int cs, size_t budget, int mp1, SpShape* s) {
+  auto fill = [&](int cs, size_t budget, SpShape* s) {
     s->cs = cs;
-    s->mp1 = mp1;
     s->share_cap = (sel_pages + cs - 1) / cs;
     s->keys_in_smem = max_pages <= kSpKeysCap;
     s->logits_in_smem = (size_t)sp_pad(s->share_cap * kPage) * G * 4 <= (size_t)kSpLogitsSmem;
@@ -1613,7 +1618,7 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
     const size_t logits = s->logits_in_smem ? (size_t)sp_pad(s->share_cap * kPage) * G * 4 : 0;
     const size_t room1 = budget > kSpFixedBytes + keys ? budget - kSpFixedBytes - keys : 0;
     const size_t room2 = budget > kSpFixedBytes + logits ? budget - kSpFixedBytes - logits : 0;
-    s->s1 = (int)(room1 / ((size_t)s->mp1 * kMetaRecBytes));
+    s->s1 = (int)(room1 / ((size_t)kMetaStagePages * kMetaRecBytes));
     s->s2 = (int)(room2 / stage2);
     const int need2 = (s->share_cap + kEstStagePages - 1) / kEstStagePages;   // stages of a share
     s->s1 = s->s1 < 2 ? 2 : (s->s1 > kSpMaxStages ? kSpMaxStages : s->s1);
@@ -1632,7 +1637,7 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
   if (regs * kSpThreads * 2 <= 65536) {
     for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
       if ((long long)units * cs > 2LL * num_sms) continue;
-      fill(cs, two_per_sm, kMetaStagePages / 2, &s);
+      fill(cs, two_per_sm, &s);
       if (s.smem > kSpMaxSmem) continue;
       if (sp_max_clusters<G, BITS>(cs, s.smem) >= units) {
         *out = s;
@@ -1642,14 +1647,14 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
   }
   for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
     if ((long long)units * cs > num_sms) continue;
-    fill(cs, big, kMetaStagePages, &s);
+    fill(cs, big, &s);
     if (s.smem > kSpMaxSmem) continue;
     if (sp_max_clusters<G, BITS>(cs, s.smem) >= units) {
       *out = s;
       return 0;
     }
   }
-  fill(cs_min, two_per_sm, kMetaStagePages / 2, &s);
+  fill(cs_min, two_per_sm, &s);
   if (s.smem > kSpMaxSmem) return -1;
   *out = s;
   return 0;
@@ -1666,7 +1671,6 @@ static cudaError_t sp_launch_t(SpArgs a, int sel_pages, int num_sms, cudaStream_
     return cudaErrorInvalidValue;
   a.s1 = sh.s1;
   a.s2 = sh.s2;
-  a.mp1 = sh.mp1;
   a.share_cap = sh.share_cap;
   if (sh.keys_in_smem) a.gkeys = nullptr;
   if (sh.logits_in_smem) a.glogits = nullptr;

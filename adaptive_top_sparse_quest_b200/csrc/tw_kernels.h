@@ -97,12 +97,11 @@ struct SpArgs {
   int lcap;
   int* status;              // device status word (bounded waits that gave up)
   int s1, s2;               // ring stages of the two phases
-  int mp1;                  // page records per score stage (32 or 64)
   int share_cap;            // candidate pages per CTA share (shared-memory logits stride / 16)
 };
 
 struct SpShape {
-  int cs, share_cap, s1, s2, mp1;
+  int cs, share_cap, s1, s2;
   bool keys_in_smem, logits_in_smem;
   size_t smem;
 };
