@@ -45,6 +45,7 @@ constexpr int kDecHW = kDecThreads / 16;       // half-warps
 constexpr int kStageTok = 16;                  // tokens per pipeline stage
 constexpr int kStages = 6;                     // 5 stages (40 KB) in flight per CTA
 constexpr int kWin = 512;                      // token rows staged per window
+constexpr int kMinTokPerCta = 64;              // few-set path: tokens per CTA at least
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void h8_to_f8(uint4 r, float* f) {
@@ -478,12 +479,17 @@ k_sparse_decode(Layout L, const __half* __restrict__ q, int Hq, int G, int group
     // Few sets: every set gets whole CTAs, so no CTA's range straddles two
     // sets (a straddling CTA pays a second row staging and ring ramp-up, and
     // the set's merge waits for it).  A set with cnt tokens gets
-    // 1 + floor(cnt * (n - E) / S) CTAs, E the number of non-empty sets, so the
-    // shares add up to at most n and no CTA holds more than about S / (n - E).
+    // 1 + floor(cnt * np / S) CTAs, E the number of non-empty sets and
+    // np = min(n - E, S / kMinTokPerCta), so the shares add up to at most n;
+    // CTAs past them have no set and exit.
     int64_t ne = 0;
     for (int s = tid; s < nsets; s += kDecThreads) ne += count[s] > 0 && icap > 0 ? 1 : 0;
     const int64_t E = block_sum_i64(ne, sm.red64);
-    const int64_t np = n - E;
+    // at least kMinTokPerCta tokens per CTA: a few small sets leave CTAs
+    // idle rather than split into ranges whose fixed costs (row staging,
+    // ring ramp-up, one more record in the merge) outweigh their tokens
+    int64_t np = n - E;
+    if (np > S / kMinTokPerCta) np = S / kMinTokPerCta;
     if (tid == 0) sm.nlist = -1;
     int64_t before = 0;   // CTAs given to the sets of earlier chunks
     for (int base = 0; base < nsets; base += kDecThreads) {

@@ -414,7 +414,7 @@ __device__ void topk_threshold(KeyAt key_at, int P, int K, uint32_t kmin, uint32
 
 __device__ __forceinline__ void sp_mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                             uint32_t b1) {
-  asm volatile(
+  asm(   // no side effects: the compiler may interleave independent tiles
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -686,14 +686,17 @@ __device__ bool resolve_small_bin(const SpWeights& W, SpSearch& s, int CS, doubl
   if (tid == 0) fx.lst_n = 0;
   __syncthreads();
 #pragma unroll 1
-  for (int i = 0; i < W.R; ++i) {
-    if (W.lp0 + i >= W.npos) break;
-    const float w = W.at(i);
-    if (w < 0.f) continue;
-    const uint32_t key = __float_as_uint(w);
-    if ((key & s.pmask) == s.prefix) {
-      const int slot = atomicAdd(&fx.lst_n, 1);
-      if (slot < kSpBinList) own[slot] = key;
+  for (int c = 0; c < W.R; c += 8) {   // eight weights loaded, then tested
+    float wv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wv[i] = (c + i < W.R && W.lp0 + c + i < W.npos) ? W.at(c + i) : -1.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t key = __float_as_uint(wv[i]);
+      if (wv[i] >= 0.f && (key & s.pmask) == s.prefix) {
+        const int slot = atomicAdd(&fx.lst_n, 1);
+        if (slot < kSpBinList) own[slot] = key;
+      }
     }
   }
   if (CS > 1) cluster_sync();   // every CTA's list is complete
@@ -1378,23 +1381,67 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       const int h0 = a.group_sets ? 0 : hs, nh = a.group_sets ? G : 1;
       __syncthreads();   // the ring (or the previous set's staged output) is free
       for (int i = tid; i < kSpHistWords; i += kSpThreads) hist[i] = 0ull;
-      // the set's weights, written over the logits of its first head (each
-      // thread reads and writes only its own positions)
-      SpWeights W{lbase + h0 * hstride, lpad,
-                  lpad ? smem_u32(lbase + h0 * hstride) : 0u, lp0, R, npos};
-#pragma unroll 1
-      for (int i = 0; i < R; ++i) {
-        const int lp = lp0 + i;
-        if (lp >= npos) break;
-        const bool ok = (lp & 15) < fx.nrow[lp >> 4];
+      // The set's weights.  Logits in shared memory: written over the logits
+      // of the set's first head, each thread on its own positions (CH at a
+      // time, loads first).  Logits in global memory: read with consecutive
+      // threads on consecutive positions, and the weights written to shared
+      // memory above the histogram when the idle ring has room (else over
+      // the first head's logits); the search then reads them from there.
+      const bool wsm = !lpad && ring_bytes >= kSpHistBytes + sp_pad(npos) * 4;
+      float* wb = lpad ? lbase + h0 * hstride
+                       : (wsm ? reinterpret_cast<float*>(ring + kSpHistBytes) : lbase + h0 * hstride);
+      SpWeights W{wb, lpad || wsm, (lpad || wsm) ? smem_u32(wb) : 0u, lp0, R, npos};
+      auto weight = [&](int lp, const float (&l)[G]) -> float {
+        if ((lp & 15) >= fx.nrow[lp >> 4]) return -1.0f;
         float acc = 0.f;
-        if (ok) {
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-            if (h >= h0 && h < h0 + nh) acc += exp2f(lbase[lidx(h, lp)] - Mh[h]) * iZ[h];
-          if (nh > 1) acc *= 1.0f / (float)nh;
+        for (int h = 0; h < G; ++h)
+          if (h >= h0 && h < h0 + nh) acc += exp2f(l[h] - Mh[h]) * iZ[h];
+        if (nh > 1) acc *= 1.0f / (float)nh;
+        return acc;
+      };
+      if (lpad) {
+        constexpr int CH = G >= 8 ? 4 : 8;
+#pragma unroll 1
+        for (int c = 0; c < R; c += CH) {
+          float lv[CH][G];
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int lp = lp0 + c + i;
+            const bool in = c + i < R && lp < npos;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              lv[i][h] = (in && h >= h0 && h < h0 + nh) ? lbase[lidx(h, lp)] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int lp = lp0 + c + i;
+            if (c + i >= R || lp >= npos) break;
+            lbase[lidx(h0, lp)] = weight(lp, lv[i]);
+          }
         }
-        lbase[lidx(h0, lp)] = ok ? acc : -1.0f;
+      } else {
+        constexpr int CH = G >= 8 ? 2 : 4;
+#pragma unroll 1
+        for (int lp0c = 0; lp0c < npos; lp0c += CH * kSpThreads) {
+          float lv[CH][G];
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int lp = lp0c + i * kSpThreads + tid;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              lv[i][h] = (lp < npos && h >= h0 && h < h0 + nh) ? lbase[lidx(h, lp)] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int lp = lp0c + i * kSpThreads + tid;
+            if (lp >= npos) break;
+            const float w = weight(lp, lv[i]);
+            if (wsm) sm_st_u32(W.sbase + 4u * (uint32_t)sp_pad(lp), __float_as_uint(w));
+            else lbase[lidx(h0, lp)] = w;
+          }
+        }
+        __syncthreads();   // the search reads positions other threads wrote
       }
       const bool keep_all = a.p >= 1.0;
       uint32_t theta = 0;
@@ -1426,13 +1473,17 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       // local position lp0 + i above / at theta
       unsigned gtm = 0, eqm = 0;
 #pragma unroll 1
-      for (int i = 0; i < R; ++i) {
-        if (lp0 + i >= npos) break;
-        const float w = W.at(i);
-        if (w < 0.f) continue;
-        const uint32_t key = __float_as_uint(w);
-        if (keep_all || (have && key > theta)) gtm |= 1u << i;
-        else if (have && key == theta) eqm |= 1u << i;
+      for (int c = 0; c < R; c += 8) {   // eight weights loaded, then tested
+        float wv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wv[i] = (c + i < R && lp0 + c + i < npos) ? W.at(c + i) : -1.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (wv[i] < 0.f) continue;
+          const uint32_t key = __float_as_uint(wv[i]);
+          if (keep_all || (have && key > theta)) gtm |= 1u << (c + i);
+          else if (have && key == theta) eqm |= 1u << (c + i);
+        }
       }
       const unsigned n_gt = __popc(gtm), n_eq = __popc(eqm);
       unsigned blk_total;
@@ -1487,17 +1538,40 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
         }
       }
       {
-        // the thread's kept positions are consecutive outputs
-        int32_t* oidx = a.idx + (int64_t)set * a.icap + first + lpos0;
-        uint32_t* orow = a.rows ? a.rows + (int64_t)set * a.icap + first + lpos0 : nullptr;
+        // The thread's kept positions are consecutive outputs from lpos0 on.
+        // They are staged in shared memory (the histogram's storage: ids,
+        // then rows) when the CTA's outputs fit it, and copied out with
+        // consecutive threads on consecutive words; else each thread stores
+        // its own run.
+        int32_t* oidx = a.idx + (int64_t)set * a.icap + first;
+        uint32_t* orow = a.rows ? a.rows + (int64_t)set * a.icap + first : nullptr;
+        const unsigned eq_blk = blk_total & 0xFFFFu;
+        const unsigned n_out = (blk_total >> 16) +
+            (r_need > eq_before ? (unsigned)min((unsigned long long)eq_blk, r_need - eq_before) : 0u);
+        const bool staged = 2 * npos * 4 <= ring_bytes;   // uniform in the CTA
+        uint32_t* sidx = reinterpret_cast<uint32_t*>(ring);
+        uint32_t* srow = sidx + npos;
         unsigned m = sel;
 #pragma unroll 1
-        for (int o = 0; m; ++o) {
+        for (unsigned o = lpos0; m; ++o) {
           const int i = __ffs(m) - 1;
           m &= m - 1;
           const int e = (lp0 + i) >> 4, r = (lp0 + i) & 15;
-          oidx[o] = (int32_t)(fx.pg[e] * kPage + (uint32_t)r);
-          if (orow) orow[o] = fx.r0[e] + (uint32_t)r;
+          const uint32_t id = fx.pg[e] * kPage + (uint32_t)r, row = fx.r0[e] + (uint32_t)r;
+          if (staged) {
+            sidx[o] = id;
+            srow[o] = row;
+          } else {
+            oidx[o] = (int32_t)id;
+            if (orow) orow[o] = row;
+          }
+        }
+        if (staged) {
+          __syncthreads();
+          for (unsigned o = tid; o < n_out; o += kSpThreads) {
+            oidx[o] = (int32_t)sidx[o];
+            if (orow) orow[o] = srow[o];
+          }
         }
       }
       if (cr == 0 && tid == 0) {
@@ -1634,8 +1708,13 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
     cudaFuncAttributes fa;
     regs = cudaFuncGetAttributes(&fa, k_select_prune<G, BITS>) == cudaSuccess ? fa.numRegs : 255;
   }
+  // clusters no larger than the unit's pages allow 64 per CTA (a small unit
+  // spread wider pays more in cluster barriers than it saves)
+  const int work = do_select ? max_pages : sel_pages;
+  int cs_top = kSpMaxCluster;
+  while (cs_top > cs_min && cs_top * 64 > work) cs_top /= 2;
   if (regs * kSpThreads * 2 <= 65536) {
-    for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
+    for (int cs = cs_top; cs >= cs_min; cs /= 2) {
       if ((long long)units * cs > 2LL * num_sms) continue;
       fill(cs, two_per_sm, &s);
       if (s.smem > kSpMaxSmem) continue;
@@ -1645,7 +1724,7 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
       }
     }
   }
-  for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
+  for (int cs = cs_top; cs >= cs_min; cs /= 2) {
     if ((long long)units * cs > num_sms) continue;
     fill(cs, big, &s);
     if (s.smem > kSpMaxSmem) continue;
