@@ -1708,13 +1708,8 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
     cudaFuncAttributes fa;
     regs = cudaFuncGetAttributes(&fa, k_select_prune<G, BITS>) == cudaSuccess ? fa.numRegs : 255;
   }
-  // clusters no larger than the unit's pages allow 64 per CTA (a small unit
-  // spread wider pays more in cluster barriers than it saves)
-  const int work = do_select ? max_pages : sel_pages;
-  int cs_top = kSpMaxCluster;
-  while (cs_top > cs_min && cs_top * 64 > work) cs_top /= 2;
   if (regs * kSpThreads * 2 <= 65536) {
-    for (int cs = cs_top; cs >= cs_min; cs /= 2) {
+    for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
       if ((long long)units * cs > 2LL * num_sms) continue;
       fill(cs, two_per_sm, &s);
       if (s.smem > kSpMaxSmem) continue;
@@ -1724,7 +1719,7 @@ static int sp_shape(int units, int max_pages, int sel_pages, bool do_select, boo
       }
     }
   }
-  for (int cs = cs_top; cs >= cs_min; cs /= 2) {
+  for (int cs = kSpMaxCluster; cs >= cs_min; cs /= 2) {
     if ((long long)units * cs > num_sms) continue;
     fill(cs, big, &s);
     if (s.smem > kSpMaxSmem) continue;
