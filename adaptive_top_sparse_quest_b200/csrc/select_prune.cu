@@ -685,18 +685,24 @@ __device__ bool resolve_small_bin(const SpWeights& W, SpSearch& s, int CS, doubl
   uint32_t* all = own + kSpBinList;                                  // the gathered list
   if (tid == 0) fx.lst_n = 0;
   __syncthreads();
+  auto add = [&](float w) {
+    const uint32_t key = __float_as_uint(w);
+    if (w >= 0.f && (key & s.pmask) == s.prefix) {
+      const int slot = atomicAdd(&fx.lst_n, 1);
+      if (slot < kSpBinList) own[slot] = key;
+    }
+  };
+  if (W.pad) {   // shared memory: one weight at a time
 #pragma unroll 1
-  for (int c = 0; c < W.R; c += 8) {   // eight weights loaded, then tested
-    float wv[8];
+    for (int i = 0; i < W.R && W.lp0 + i < W.npos; ++i) add(W.at(i));
+  } else {       // global memory: eight weights loaded, then tested
+#pragma unroll 1
+    for (int c = 0; c < W.R; c += 8) {
+      float wv[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) wv[i] = (c + i < W.R && W.lp0 + c + i < W.npos) ? W.at(c + i) : -1.0f;
+      for (int i = 0; i < 8; ++i) wv[i] = (c + i < W.R && W.lp0 + c + i < W.npos) ? W.at(c + i) : -1.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t key = __float_as_uint(wv[i]);
-      if (wv[i] >= 0.f && (key & s.pmask) == s.prefix) {
-        const int slot = atomicAdd(&fx.lst_n, 1);
-        if (slot < kSpBinList) own[slot] = key;
-      }
+      for (int i = 0; i < 8; ++i) add(wv[i]);
     }
   }
   if (CS > 1) cluster_sync();   // every CTA's list is complete
@@ -1382,8 +1388,7 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       __syncthreads();   // the ring (or the previous set's staged output) is free
       for (int i = tid; i < kSpHistWords; i += kSpThreads) hist[i] = 0ull;
       // The set's weights.  Logits in shared memory: written over the logits
-      // of the set's first head, each thread on its own positions (CH at a
-      // time, loads first).  Logits in global memory: read with consecutive
+      // of the set's first head, each thread on its own positions.  Logits in global memory: read with consecutive
       // threads on consecutive positions, and the weights written to shared
       // memory above the histogram when the idle ring has room (else over
       // the first head's logits); the search then reads them from there.
@@ -1401,24 +1406,14 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
         return acc;
       };
       if (lpad) {
-        constexpr int CH = G >= 8 ? 4 : 8;
 #pragma unroll 1
-        for (int c = 0; c < R; c += CH) {
-          float lv[CH][G];
+        for (int i = 0; i < R; ++i) {
+          const int lp = lp0 + i;
+          if (lp >= npos) break;
+          float lv[G];
 #pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            const int lp = lp0 + c + i;
-            const bool in = c + i < R && lp < npos;
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-              lv[i][h] = (in && h >= h0 && h < h0 + nh) ? lbase[lidx(h, lp)] : 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            const int lp = lp0 + c + i;
-            if (c + i >= R || lp >= npos) break;
-            lbase[lidx(h0, lp)] = weight(lp, lv[i]);
-          }
+          for (int h = 0; h < G; ++h) lv[h] = (h >= h0 && h < h0 + nh) ? lbase[lidx(h, lp)] : 0.f;
+          lbase[lidx(h0, lp)] = weight(lp, lv);
         }
       } else {
         constexpr int CH = G >= 8 ? 2 : 4;
@@ -1472,17 +1467,23 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
       // compaction in ascending position order: bit i of gtm / eqm marks
       // local position lp0 + i above / at theta
       unsigned gtm = 0, eqm = 0;
+      auto mark = [&](int i, float w) {
+        if (w < 0.f) return;
+        const uint32_t key = __float_as_uint(w);
+        if (keep_all || (have && key > theta)) gtm |= 1u << i;
+        else if (have && key == theta) eqm |= 1u << i;
+      };
+      if (W.pad) {   // shared memory: one weight at a time
 #pragma unroll 1
-      for (int c = 0; c < R; c += 8) {   // eight weights loaded, then tested
-        float wv[8];
+        for (int i = 0; i < R && lp0 + i < npos; ++i) mark(i, W.at(i));
+      } else {       // global memory: eight weights loaded, then tested
+#pragma unroll 1
+        for (int c = 0; c < R; c += 8) {
+          float wv[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) wv[i] = (c + i < R && lp0 + c + i < npos) ? W.at(c + i) : -1.0f;
+          for (int i = 0; i < 8; ++i) wv[i] = (c + i < R && lp0 + c + i < npos) ? W.at(c + i) : -1.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (wv[i] < 0.f) continue;
-          const uint32_t key = __float_as_uint(wv[i]);
-          if (keep_all || (have && key > theta)) gtm |= 1u << (c + i);
-          else if (have && key == theta) eqm |= 1u << (c + i);
+          for (int i = 0; i < 8; ++i) mark(c + i, wv[i]);
         }
       }
       const unsigned n_gt = __popc(gtm), n_eq = __popc(eqm);
