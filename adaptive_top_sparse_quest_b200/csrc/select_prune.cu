@@ -26,12 +26,16 @@
 //   every query head of the group on the tensor cores (mma.sync, codes as the
 //   A operand) into shared memory and keeps per-head (max, sum 2^(l - max)).
 //   One exchange of those pairs gives every CTA the unit's softmax statistics.
-//   Each thread then holds the weights of R consecutive candidates of its
-//   CTA's share in registers, and the threshold is found most significant
-//   digit first (12 + 9 + 9 bits of the fp32 weight) over exact integer
-//   masses; the CTAs reduce-scatter their digit histograms through
-//   distributed shared memory.  The kept tokens are compacted in ascending
-//   order with their physical K/V rows for the attention kernel.
+//   Each thread then owns the weights of R consecutive candidates of its
+//   CTA's share (in shared memory), and the threshold is found most
+//   significant digit first (12 + 9 + 9 bits of the fp32 weight) over exact
+//   integer masses.  The first digit's histograms are reduce-scattered over
+//   the cluster through distributed shared memory; when that digit holds few
+//   enough weights over the cluster, every CTA gathers them and finishes on
+//   its own (a one-warp sort up to 128 weights, the remaining two digits on
+//   the list up to 1024), else the remaining digits are reduced like the
+//   first.  The kept tokens are compacted in ascending order with their
+//   physical K/V rows for the attention kernel.
 //
 // The score of a page is a deterministic fp32 sum in one fixed order, so the
 // selected page ids are an exact integer result: products of two fp16 values
@@ -43,12 +47,12 @@
 // (one of the two products is zero), so it is accumulated with two fused
 // multiply-adds whose single rounding is the rounding of the sum.
 //
-// Streaming: cp.async.bulk copies complete on a stage's "full" mbarrier
-// together with their byte count; the consumer warps release the stage on
-// its "empty" mbarrier and warp 0 refills it.  The scales and zeros of the
-// quantised rows (8 bytes per row, whose start need not be 16-byte aligned in
-// a contiguous cache) arrive by 8-byte cp.async that signal the same full
-// mbarrier.  No copy uses cluster multicast.  Every wait is bounded
+// Streaming: each ring stage completes on its "full" mbarrier: bulk copies
+// (cp.async.bulk) with their byte counts for the metadata records, or every
+// thread's cp.async pieces (one arrival per thread when they have landed) for
+// the quantised rows, whose scales and zeros need not start 16-byte aligned
+// in a contiguous cache.  A stage is refilled after the block barrier that
+// ends its use.  No copy uses cluster multicast.  Every wait is bounded
 // (tw_bulk.cuh).
 #include "tw_bulk.cuh"
 #include "tw_common.cuh"

@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -101,12 +102,21 @@ TRAFFIC_SOURCES = ("cache_build.cu", "decode.cu", "host_io.cu", "resolve.cu", "s
                    "tw_bulk.cuh", "tw_common.cuh", "tw_kernels.h")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments or blank lines: what a comment edit leaves alone."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def src_hash():
+    """Hash of the measured kernels' device sources (code only), so that an ncu
+    capture stays attached to the code it was taken on."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "adaptive_top_sparse_quest_b200", "csrc")
     for f in TRAFFIC_SOURCES:
         h.update(f.encode())
-        h.update(open(os.path.join(d, f), "rb").read())
+        h.update(_code_only(open(os.path.join(d, f)).read()).encode())
     return h.hexdigest()[:16]
 
 
