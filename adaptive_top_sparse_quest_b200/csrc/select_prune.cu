@@ -61,7 +61,8 @@
 namespace tw {
 
 constexpr int kSpWarps = kSpThreads / 32;
-constexpr int kMetaStagePages = 64;     // page records per score stage (32 KB): four per half-warp
+constexpr int kMetaStagePages = 64;     // page records per score stage (32 KB); 32 or 64
+static_assert(kMetaStagePages == 32 || kMetaStagePages == 64, "two or four pages per half-warp");
 constexpr int kMetaRecBytes = 2 * kHeadDim * 2;          // one page's min and max rows
 constexpr int kEstStagePages = 16;                       // 256 candidate tokens per stage
 constexpr int kEstStageTok = kEstStagePages * kPage;
@@ -898,7 +899,8 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
     // pool pages of the stage into the slot (an id outside the pool reads pool page 0)
     auto store_pt = [&](int slot, int2 e) {
       fx.pt1[slot][lane] = (unsigned)e.x < (unsigned)L.pool_pages ? e.x : 0;
-      fx.pt1[slot][lane + 32] = (unsigned)e.y < (unsigned)L.pool_pages ? e.y : 0;
+      constexpr int kHi = kMetaStagePages > 32 ? 32 : 0;   // the second half of a 64-page stage
+      if (kHi) fx.pt1[slot][lane + kHi] = (unsigned)e.y < (unsigned)L.pool_pages ? e.y : 0;
     };
     auto issue1 = [&](int k, int slot) {
       const int n = k < nst ? min(mp, npg - k * mp) : 0;
@@ -999,9 +1001,9 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
           }
         }
       };
-      if (G >= 4) {
+      if (kMetaStagePages == 32 || G >= 4) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < kMetaStagePages / 32; ++half)
           emit(page_scores<G, 2>(Q, st + half * 32 * kMetaRecBytes, hw, l16, hmask),
                hw + 16 * ((l16 >> 3) & 1) + 32 * half, l16 & 7, 8);
       } else {
@@ -1314,31 +1316,35 @@ __global__ void __launch_bounds__(kSpThreads, G <= 4 ? 2 : 1) k_select_prune(SpA
             if (c0 + 8 < ns * kPage) lbase[lidx(he, c0 + 8)] = lg[k][hp][1];
           }
         }
-        float m = -INFINITY;
+        // this lane's running (max, sum 2^(l - max)) over its own logits; the
+        // lanes are merged once after the stream
         if (owner && hv) {
+          const float m = fmaxf(fmaxf(lg[0][hp][0], lg[0][hp][1]), fmaxf(lg[1][hp][0], lg[1][hp][1]));
+          if (m != -INFINITY) {
+            const float mn = fmaxf(Mrun[hp], m);
+            float z = Mrun[hp] == -INFINITY ? 0.f : Zrun[hp] * exp2f(Mrun[hp] - mn);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) m = fmaxf(m, fmaxf(lg[k][hp][0], lg[k][hp][1]));
-        }
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float z = 0.f;
-        if (owner && hv && m != -INFINITY) {
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            z += exp2f(lg[k][hp][0] - m);
-            z += exp2f(lg[k][hp][1] - m);
+            for (int k = 0; k < 2; ++k) z += exp2f(lg[k][hp][0] - mn) + exp2f(lg[k][hp][1] - mn);
+            Zrun[hp] = z;
+            Mrun[hp] = mn;
           }
-        }
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        if (m != -INFINITY) {
-          const float mn = fmaxf(Mrun[hp], m);
-          Zrun[hp] = (Mrun[hp] == -INFINITY ? 0.f : Zrun[hp] * exp2f(Mrun[hp] - mn)) +
-                     z * exp2f(m - mn);
-          Mrun[hp] = mn;
         }
       }
       __syncthreads();   // every warp is done with this slot before it is refilled
+    }
+    // merge the lanes' pairs of each head (lanes of one head differ in bits 2..4)
+#pragma unroll
+    for (int hp = 0; hp < HP; ++hp) {
+      float m = Mrun[hp], z = Zrun[hp];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o), zo = __shfl_xor_sync(0xffffffffu, z, o);
+        const float mn = fmaxf(m, mo);
+        z = (m == -INFINITY ? 0.f : z * exp2f(m - mn)) + (mo == -INFINITY ? 0.f : zo * exp2f(mo - mn));
+        m = mn;
+      }
+      Mrun[hp] = m;
+      Zrun[hp] = z;
     }
     // per-warp statistics -> the CTA's -> every CTA's, merged in rank order
 #pragma unroll
