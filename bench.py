@@ -324,7 +324,14 @@ def run_reference(args):
     if rank != 0:
         return 0
     import torch
-    w = make_workload(args.config, "cpu", args.batch)
+    # the same seeded workload as the GPU arm: generated where that arm generates
+    # it (the device generator draws other numbers than the host one), then
+    # brought to the host for the oracle
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
+    w = make_workload(args.config, gen, args.batch)
+    if gen != "cpu":
+        w = w.to("cpu")
+        torch.cuda.empty_cache()
     chans = None
     if args.selector == "label":
         import workloads as W
