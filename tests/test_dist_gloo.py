@@ -54,3 +54,16 @@ def test_single_rank_is_identity():
     import bench
     assert bench.reduce_max(3.5, 1, None) == 3.5
     assert bench.whole_job_us_per_step(3.5, 7, 1) == pytest.approx(3500 / 7)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun the reference arm runs and prints on rank 0 alone; the
+    other ranks return 0 without work or output."""
+    import argparse
+
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    args = argparse.Namespace(config="tiny", batch=0, selector="quest", key_bits=4, steps=1,
+                              warmup=0, gpus=2)
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
